@@ -1,0 +1,607 @@
+/*
+ * hq_oracle.c -- plain, slow CPU oracle of the HyperQuant per-tile codec.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library) shares no code, header, table or constant with it.
+ *
+ * Sources, cited by page title and section:
+ *   [V1] "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline for
+ *        Large Language and Diffusion Models" (mlsanity.com paper page),
+ *        section "Abstract (arXiv)", ingredients (i)-(iv).
+ *   [V2] "HyperQuant: A Near-Entropy-Optimal Lattice Quantization Pipeline
+ *        for Large Language and Diffusion Models" (acceptodds.com ICLR 2027
+ *        page), abstract.
+ *   [CS82] Conway & Sloane, "Fast quantizing and decoding algorithms for
+ *        lattice quantizers and codes", IEEE Trans. IT 28(2), 1982:
+ *        nearest point of Z^n, D_n and of a union of cosets.
+ *   [SM64] Steele, Lea & Flood, "Fast splittable pseudorandom number
+ *        generators", OOPSLA 2014: the SplitMix64 output function.
+ *
+ * The pages state the pipeline (per-tile random-sign Hadamard rotation,
+ * lattice E8/D4/A2/Z, lossless strip of the bits membership fixes, Rice code
+ * of the remainder, subtractive dither for the KV cache) but none of its
+ * constants, tie rules or the stream layout.  Every such choice below is a
+ * stated reading; the same readings are listed, with reasons, in the design
+ * notes that ship with the repository.
+ *
+ * Precision: every step whose floating-point result decides an integer (the
+ * lattice point, the Rice parameter, the stream) runs in IEEE binary32 with
+ * round-to-nearest-even, one rounding per operation (compile with
+ * -ffp-contract=off, no fast-math).  The decode reconstruction and the GEMV
+ * reference run in binary64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define HQO_MAX_TILE 1024
+
+/* status bits shared by encode/decode (values are this oracle's own) */
+#define HQO_NONFINITE 1
+#define HQO_CAPACITY 2
+#define HQO_CORRUPT 4
+
+/* ------------------------------------------------------------------ */
+/* Counter-based randomness [SM64]: the pages only say "random signs" and
+ * "seeded dither"; the generator is this reading's choice. */
+
+uint64_t hqo_mix64(uint64_t z)
+{
+    z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ULL;
+    z = (z ^ (z >> 27)) * 0x94d049bb133111ebULL;
+    return z ^ (z >> 31);
+}
+
+/* H(seed, tag, a, b): three chained mixes of a golden-gamma offset seed. */
+uint64_t hqo_hash(uint64_t seed, uint64_t tag, uint64_t a, uint64_t b)
+{
+    uint64_t h = hqo_mix64(seed + 0x9E3779B97F4A7C15ULL * (tag + 1));
+    h = hqo_mix64(h ^ a);
+    return hqo_mix64(h ^ b);
+}
+
+/* Random sign of coordinate i of column tile j [V1 (i), V2 "per-tile
+ * Walsh-Hadamard rotation"]: bit (i mod 64) of H(seed, 1, j, i / 64), set
+ * bit = -1.  Signs depend on the column tile only, so every row of a
+ * column tile shares them. */
+int hqo_sign(uint64_t seed, uint64_t j, uint32_t i)
+{
+    uint64_t h = hqo_hash(seed, 1, j, i >> 6);
+    return ((h >> (i & 63)) & 1) ? -1 : 1;
+}
+
+/* Uniform r_i in [0,1) with 24 bits, for coordinate i of tile t (dither).
+ * One hash serves coordinates 2m and 2m+1: bits 40..63 and 16..39. */
+float hqo_uniform(uint64_t seed, uint64_t t, uint32_t i)
+{
+    uint64_t h = hqo_hash(seed, 2, t, i >> 1);
+    uint32_t r = (i & 1) ? (uint32_t)((h >> 16) & 0xFFFFFFu) : (uint32_t)(h >> 40);
+    return (float)r * 0x1p-24f;
+}
+
+/* ------------------------------------------------------------------ */
+/* Walsh-Hadamard transform [V1 (i), V2]: unnormalised Sylvester matrix
+ * H[a][b] = (-1)^popcount(a & b).  Butterfly stages h = 1, 2, 4, ..., n/2
+ * in that order; the pair (a, a+h) with bit h of a clear becomes
+ * (v_a + v_{a+h}, v_a - v_{a+h}). */
+void hqo_fwht_f32(float *v, int n)
+{
+    for (int h = 1; h < n; h <<= 1)
+        for (int a = 0; a < n; a++)
+            if (!(a & h)) {
+                float p = v[a], q = v[a + h];
+                v[a] = p + q;
+                v[a + h] = p - q;
+            }
+}
+
+void hqo_fwht_f64(double *v, int n)
+{
+    for (int h = 1; h < n; h <<= 1)
+        for (int a = 0; a < n; a++)
+            if (!(a & h)) {
+                double p = v[a], q = v[a + h];
+                v[a] = p + q;
+                v[a + h] = p - q;
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-tile scale for the target rate (pages silent beyond "a per-tile
+ * scale"; reading): the high-resolution entropy of a lattice quantizer of
+ * cell volume V and step D on i.i.d. N(0, s^2) coordinates is
+ * log2(sqrt(2 pi e) s) - log2(D V^(1/d)) bits per dimension; setting it to
+ * R gives D = s sqrt(2 pi e) 2^-R V^(-1/d).  With the unnormalised
+ * Hadamard transform the rotated coordinates have variance sum_i w_i^2. */
+
+static double cell_volume(int lattice)
+{
+    switch (lattice) {
+    case 8: return 1.0;             /* E8: unimodular */
+    case 4: return 2.0;             /* D4: index 2 in Z^4 */
+    case 2: return sqrt(3.0) / 2.0; /* A2 with minimal norm 1 */
+    default: return 1.0;            /* Z */
+    }
+}
+
+float hqo_rate_constant(int lattice, float bps)
+{
+    double c = sqrt(2.0 * M_PI * M_E) * pow(2.0, -(double)bps) *
+               pow(cell_volume(lattice), -1.0 / (double)lattice);
+    return (float)c;
+}
+
+/* sum of squares by a fixed pairwise tree: level l adds the partial sums of
+ * indices that differ in bit l (l = 0 first). */
+float hqo_sumsq(const float *w, int n)
+{
+    float a[HQO_MAX_TILE];
+    for (int i = 0; i < n; i++) a[i] = w[i] * w[i];
+    for (int h = 1; h < n; h <<= 1)
+        for (int i = 0; i < n; i++)
+            if (!(i & h)) a[i] = a[i] + a[i + h];
+    return a[0];
+}
+
+/* binary32 -> bfloat16 bit pattern, round to nearest even (finite input) */
+static uint16_t bf16_bits(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Delta = bf16(c * sqrt(S)).  A non-finite S marks the tile non-finite;
+ * a zero or subnormal Delta (and any non-finite tile) is stored as 0 and the
+ * tile's lattice points are all zero. */
+uint16_t hqo_tile_scale(float S, float c, int *nonfinite)
+{
+    *nonfinite = !isfinite(S);
+    if (*nonfinite) return 0;
+    float sigma = sqrtf(S);
+    float d32 = c * sigma;
+    uint16_t b = bf16_bits(d32);
+    if ((b & 0x7F80u) == 0) return 0;
+    return b;
+}
+
+/* ------------------------------------------------------------------ */
+/* Nearest lattice points [CS82].  Each returns the coset bit c (E8, A2;
+ * else 0), the integer coordinates z that the stream stores before the
+ * strip, and the point itself in binary32.
+ *   Z  : points Z;           z = y.
+ *   D_n: points of Z^n with even sum; z = y.
+ *   E8 : D8 u (D8 + 1/2);    z = y - c/2 (in D8).
+ *   A2 : points (a + c/2, (b + c/2) sqrt3);  z = (a, b).
+ * Tie rules (reading): rint ties to even; D_n flips the first coordinate of
+ * largest |x - rint(x)|, towards x (upwards when x is an integer); E8 keeps
+ * the integer coset when the two squared distances are equal; A2 likewise. */
+
+static void dn_round(const float *x, int d, int32_t *f)
+{
+    float e[8];
+    int32_t sum = 0;
+    for (int i = 0; i < d; i++) {
+        float r = rintf(x[i]);
+        f[i] = (int32_t)r;
+        e[i] = x[i] - r;
+        sum += f[i];
+    }
+    if (sum & 1) {
+        int b = 0;
+        for (int i = 1; i < d; i++)
+            if (fabsf(e[i]) > fabsf(e[b])) b = i;
+        f[b] += (e[b] >= 0.0f) ? 1 : -1;
+    }
+}
+
+static float sqdist(const float *x, const float *p, int d)
+{
+    float s = 0.0f;
+    for (int i = 0; i < d; i++) {
+        float t = x[i] - p[i];
+        s = s + t * t;
+    }
+    return s;
+}
+
+void hqo_nearest(int lattice, const float *x, int *c, int32_t *z, float *pt)
+{
+    *c = 0;
+    if (lattice == 1) {
+        float r = rintf(x[0]);
+        z[0] = (int32_t)r;
+        pt[0] = r;
+    } else if (lattice == 4) {
+        dn_round(x, 4, z);
+        for (int i = 0; i < 4; i++) pt[i] = (float)z[i];
+    } else if (lattice == 8) {
+        int32_t a[8], b[8];
+        float xs[8], pa[8], pb[8];
+        dn_round(x, 8, a);
+        for (int i = 0; i < 8; i++) xs[i] = x[i] - 0.5f;
+        dn_round(xs, 8, b);
+        for (int i = 0; i < 8; i++) {
+            pa[i] = (float)a[i];
+            pb[i] = (float)b[i] + 0.5f;
+        }
+        float d0 = sqdist(x, pa, 8), d1 = sqdist(x, pb, 8);
+        if (d0 <= d1) {
+            for (int i = 0; i < 8; i++) { z[i] = a[i]; pt[i] = pa[i]; }
+        } else {
+            *c = 1;
+            for (int i = 0; i < 8; i++) { z[i] = b[i]; pt[i] = pb[i]; }
+        }
+    } else { /* A2 */
+        const float S3 = (float)sqrt(3.0);
+        const float T = (float)(1.0 / sqrt(3.0));
+        float y1 = x[1] * T;
+        float a0 = rintf(x[0]), b0 = rintf(y1);
+        float a1 = rintf(x[0] - 0.5f), b1 = rintf(y1 - 0.5f);
+        float p0[2] = { a0, b0 * S3 };
+        float p1[2] = { a1 + 0.5f, (b1 + 0.5f) * S3 };
+        float d0 = sqdist(x, p0, 2), d1 = sqdist(x, p1, 2);
+        if (d0 <= d1) {
+            z[0] = (int32_t)a0; z[1] = (int32_t)b0; pt[0] = p0[0]; pt[1] = p0[1];
+        } else {
+            *c = 1;
+            z[0] = (int32_t)a1; z[1] = (int32_t)b1; pt[0] = p1[0]; pt[1] = p1[1];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Subtractive dither for the KV cache [V2]: delta uniform on the Voronoi
+ * cell, drawn as a uniform point x0 of a box that tiles space under a
+ * sublattice of the lattice (2Z^d for E8 and D4, Z for Z, Z x sqrt3 Z for
+ * A2), reduced by the lattice: delta = x0 - Q(x0).  Vector v of tile t. */
+void hqo_dither(int lattice, uint64_t seed, uint64_t t, uint32_t v, float *delta)
+{
+    int d = lattice;
+    float x0[8] = { 0 }, pt[8];
+    int32_t z[8];
+    int c;
+    for (int m = 0; m < d; m++) {
+        float r = hqo_uniform(seed, t, v * (uint32_t)d + (uint32_t)m);
+        if (lattice == 8 || lattice == 4) x0[m] = 2.0f * r;
+        else if (lattice == 1) x0[m] = r;
+        else x0[m] = (m == 0) ? r : r * (float)sqrt(3.0);
+    }
+    hqo_nearest(lattice, x0, &c, z, pt);
+    for (int m = 0; m < d; m++) delta[m] = x0[m] - pt[m];
+}
+
+/* ------------------------------------------------------------------ */
+/* Lossless strip and zigzag [V1 (iii), V2 "a lossless strip discards the
+ * bits lattice membership already fixes"].  Reading: for D-type vectors
+ * (D4, and E8 after its coset bit is removed) the coordinate sum is even,
+ * so the parity of the last coordinate is implied: it is stored halved
+ * (floor).  A2 keeps the coset bit c and its two integers.  Z strips
+ * nothing.  Zigzag maps 0,-1,1,-2,... to 0,1,2,3,... */
+
+static int32_t floor_half(int32_t z) { return (z - (z & 1)) / 2; }
+
+static uint32_t zigzag(int32_t z) { return z >= 0 ? 2u * (uint32_t)z : 2u * (uint32_t)(-(int64_t)z) - 1u; }
+
+static int32_t unzigzag(uint32_t u) { return (u & 1) ? -(int32_t)((u + 1) / 2) : (int32_t)(u / 2); }
+
+void hqo_symbols(int lattice, const int32_t *z, uint32_t *u)
+{
+    int d = lattice;
+    for (int i = 0; i < d; i++) {
+        int32_t s = z[i];
+        if ((lattice == 8 || lattice == 4) && i == d - 1) s = floor_half(z[i]);
+        u[i] = zigzag(s);
+    }
+}
+
+void hqo_unsymbols(int lattice, const uint32_t *u, int32_t *z)
+{
+    int d = lattice;
+    int32_t sum = 0;
+    for (int i = 0; i < d; i++) z[i] = unzigzag(u[i]);
+    if (lattice == 8 || lattice == 4) {
+        for (int i = 0; i < d - 1; i++) sum += z[i];
+        z[d - 1] = 2 * z[d - 1] + (sum & 1);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Rice code [V1 (iii), V2 "a Rice code carries the remainder"]:
+ * code(u, k) = q = floor(u / 2^k) zero bits, one 1 bit, and the k low bits
+ * of u; length q + 1 + k.  Per-tile k in [0, 15] minimising the tile's total
+ * length, smallest k on ties (brute force over all 16 values). */
+uint64_t hqo_rice_cost(const uint32_t *u, int n, int k)
+{
+    uint64_t s = 0;
+    for (int i = 0; i < n; i++) s += (uint64_t)(u[i] >> k) + 1u + (uint64_t)k;
+    return s;
+}
+
+int hqo_best_k(const uint32_t *u, int n)
+{
+    int bk = 0;
+    uint64_t best = hqo_rice_cost(u, n, 0);
+    for (int k = 1; k <= 15; k++) {
+        uint64_t c = hqo_rice_cost(u, n, k);
+        if (c < best) { best = c; bk = k; }
+    }
+    return bk;
+}
+
+/* Tile stream layout (this build's format; the pages print none).  Bits are
+ * numbered LSB-first within little-endian 32-bit words.
+ *   [0, C)            coset bit of vector v at bit v (C = n/d for E8, A2)
+ *   [C, C + n k)      low k bits of code i at C + i k, LSB first
+ *   [C + n k, ...)    unary parts: q_i zero bits then a one bit, i = 0..n-1
+ * then zero padding to a whole word.  Same bits as the interleaved Rice
+ * code, grouped by kind. */
+static int put_bit(uint32_t *w, uint64_t cap_bits, uint64_t pos, int b)
+{
+    if (pos >= cap_bits) return 0;
+    if (b) w[pos >> 5] |= 1u << (pos & 31);
+    return 1;
+}
+
+static int get_bit(const uint32_t *w, uint64_t pos) { return (int)((w[pos >> 5] >> (pos & 31)) & 1u); }
+
+/* returns the number of words, or -1 if cap_words is too small */
+int hqo_pack_tile(int lattice, int n, int k, const uint8_t *coset, const uint32_t *u,
+                  uint32_t *words, int cap_words)
+{
+    uint64_t cap = (uint64_t)cap_words * 32u, pos = 0;
+    int d = lattice;
+    int nv = n / d;
+    memset(words, 0, sizeof(uint32_t) * (size_t)cap_words);
+    if (lattice == 8 || lattice == 2)
+        for (int v = 0; v < nv; v++)
+            if (!put_bit(words, cap, pos++, coset[v])) return -1;
+    for (int i = 0; i < n; i++)
+        for (int b = 0; b < k; b++)
+            if (!put_bit(words, cap, pos++, (int)((u[i] >> b) & 1u))) return -1;
+    for (int i = 0; i < n; i++) {
+        pos += u[i] >> k;
+        if (!put_bit(words, cap, pos++, 1)) return -1;
+    }
+    return (int)((pos + 31) / 32);
+}
+
+/* Parse one tile; 0 on success, HQO_CORRUPT if the words do not hold a
+ * canonical tile (a read past the end, a one bit in the padding, or a word
+ * count other than ceil(bits / 32)). */
+int hqo_unpack_tile(int lattice, int n, int k, const uint32_t *words, int nwords,
+                    uint8_t *coset, uint32_t *u)
+{
+    uint64_t end = (uint64_t)nwords * 32u, pos = 0;
+    int d = lattice;
+    int nv = n / d;
+    if (k < 0 || k > 15) return HQO_CORRUPT;
+    if (lattice == 8 || lattice == 2) {
+        for (int v = 0; v < nv; v++) {
+            if (pos >= end) return HQO_CORRUPT;
+            coset[v] = (uint8_t)get_bit(words, pos++);
+        }
+    } else {
+        for (int v = 0; v < nv; v++) coset[v] = 0;
+    }
+    for (int i = 0; i < n; i++) {
+        uint32_t low = 0;
+        for (int b = 0; b < k; b++) {
+            if (pos >= end) return HQO_CORRUPT;
+            low |= (uint32_t)get_bit(words, pos++) << b;
+        }
+        u[i] = low;
+    }
+    for (int i = 0; i < n; i++) {
+        uint32_t q = 0;
+        for (;;) {
+            if (pos >= end) return HQO_CORRUPT;
+            if (get_bit(words, pos++)) break;
+            q++;
+        }
+        if (q > (1u << 16)) return HQO_CORRUPT;
+        u[i] |= q << k;
+    }
+    for (uint64_t p = pos; p < end; p++)
+        if (get_bit(words, p)) return HQO_CORRUPT;
+    if ((pos + 31) / 32 != (uint64_t)nwords) return HQO_CORRUPT;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* One tile, end to end [V1 (i)-(iv), V2].
+ * w: n binary32 inputs (bf16 inputs are widened exactly by the caller).
+ * j: column tile (signs), t: tile index (dither).  Outputs the bf16 bits of
+ * Delta, k, the words, and optionally the pre-strip integer coordinates
+ * z[n] and coset bits c[n/d].  Returns the word count, -1 if cap_words is
+ * too small.  *status gets HQO_NONFINITE for a non-finite tile. */
+int hqo_encode_tile(const float *w, int n, int lattice, float bps, uint64_t seed,
+                    uint64_t j, uint64_t t, int dither, uint16_t *scale_out, uint8_t *k_out,
+                    uint32_t *words, int cap_words, int32_t *z_out, uint8_t *c_out, int *status)
+{
+    float v[HQO_MAX_TILE];
+    int32_t z[HQO_MAX_TILE];
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    int d = lattice, nv = n / lattice, nonfinite = 0;
+
+    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * w[i];
+    hqo_fwht_f32(v, n);
+    float S = hqo_sumsq(w, n);
+    uint16_t sb = hqo_tile_scale(S, hqo_rate_constant(lattice, bps), &nonfinite);
+    if (nonfinite) *status |= HQO_NONFINITE;
+
+    if (sb == 0) {
+        for (int i = 0; i < n; i++) z[i] = 0;
+        for (int q = 0; q < nv; q++) coset[q] = 0;
+    } else {
+        float inv = 1.0f / bf16_to_float(sb);
+        for (int q = 0; q < nv; q++) {
+            float x[8], pt[8], del[8];
+            int c;
+            if (dither) hqo_dither(lattice, seed, t, (uint32_t)q, del);
+            for (int m = 0; m < d; m++) {
+                x[m] = v[q * d + m] * inv;
+                if (dither) x[m] = x[m] + del[m];
+            }
+            hqo_nearest(lattice, x, &c, &z[q * d], pt);
+            coset[q] = (uint8_t)c;
+        }
+    }
+    for (int q = 0; q < nv; q++) hqo_symbols(lattice, &z[q * d], &u[q * d]);
+    int k = hqo_best_k(u, n);
+    *scale_out = sb;
+    *k_out = (uint8_t)k;
+    if (z_out) memcpy(z_out, z, sizeof(int32_t) * (size_t)n);
+    if (c_out) memcpy(c_out, coset, (size_t)nv);
+    return hqo_pack_tile(lattice, n, k, coset, u, words, cap_words);
+}
+
+/* Decode one tile into binary64 (before any output rounding):
+ * w_hat = s . H(Delta (p - delta)) / n with p the lattice point.
+ * Returns 0 or HQO_CORRUPT (output zeroed). */
+int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint16_t scale,
+                    int k, uint64_t seed, uint64_t j, uint64_t t, int dither, double *out)
+{
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    int32_t z[8];
+    double v[HQO_MAX_TILE];
+    int d = lattice, nv = n / lattice;
+    int st = hqo_unpack_tile(lattice, n, k, words, nwords, coset, u);
+    if (st) {
+        for (int i = 0; i < n; i++) out[i] = 0.0;
+        return st;
+    }
+    double delta_f = (double)bf16_to_float(scale);
+    for (int q = 0; q < nv; q++) {
+        double p[8];
+        float del[8];
+        hqo_unsymbols(lattice, &u[q * d], z);
+        if (lattice == 2) {
+            p[0] = (double)z[0] + 0.5 * coset[q];
+            p[1] = ((double)z[1] + 0.5 * coset[q]) * sqrt(3.0);
+        } else {
+            for (int m = 0; m < d; m++) p[m] = (double)z[m] + 0.5 * coset[q];
+        }
+        if (dither && scale != 0) {
+            hqo_dither(lattice, seed, t, (uint32_t)q, del);
+            for (int m = 0; m < d; m++) p[m] -= (double)del[m];
+        }
+        for (int m = 0; m < d; m++) v[q * d + m] = delta_f * p[m];
+    }
+    hqo_fwht_f64(v, n);
+    for (int i = 0; i < n; i++) out[i] = (double)hqo_sign(seed, j, (uint32_t)i) * v[i] / (double)n;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Whole matrices, tile by tile.  x is row-major rows x cols, dtype 0 =
+ * bf16 bit patterns (uint16), 1 = binary32.  Tile t = r (cols/n) + j covers
+ * x[r][j n .. j n + n).  Tiles [t0, t1) are encoded into fixed slots of
+ * slot_words words each: words for tile t start at slots + (t - t0) slot_words
+ * and their count goes to nwords[t - t0].  The caller forms the offsets
+ * (an exclusive prefix sum of nwords) and the payload (the slots
+ * concatenated); the prefix sum is the format's only cross-tile step. */
+int hqo_encode_tiles(const void *x, int dtype, int64_t rows, int64_t cols, int n, int lattice,
+                     float bps, uint64_t seed, int dither, int64_t t0, int64_t t1,
+                     uint32_t *slots, int slot_words, int32_t *nwords, uint16_t *scale,
+                     uint8_t *kk)
+{
+    float w[HQO_MAX_TILE];
+    int64_t tpr = cols / n;
+    int status = 0;
+    (void)rows;
+    for (int64_t t = t0; t < t1; t++) {
+        int64_t r = t / tpr, j = t % tpr;
+        int64_t base = r * cols + j * n;
+        for (int i = 0; i < n; i++) {
+            if (dtype == 0) w[i] = bf16_to_float(((const uint16_t *)x)[base + i]);
+            else w[i] = ((const float *)x)[base + i];
+        }
+        int nw = hqo_encode_tile(w, n, lattice, bps, seed, (uint64_t)j, (uint64_t)t, dither,
+                                 &scale[t - t0], &kk[t - t0], slots + (t - t0) * (int64_t)slot_words,
+                                 slot_words, NULL, NULL, &status);
+        if (nw < 0) return -1;
+        nwords[t - t0] = nw;
+    }
+    return status;
+}
+
+/* Decode tiles [t0, t1) of a stream given its offsets (off[t] .. off[t+1]
+ * are the words of tile t) into out (binary64, row-major rows x cols,
+ * only the decoded tiles are written).  Returns the OR of tile statuses. */
+int hqo_decode_tiles(const uint32_t *payload, const uint32_t *off, const uint16_t *scale,
+                     const uint8_t *kk, int64_t rows, int64_t cols, int n, int lattice,
+                     uint64_t seed, int dither, int64_t t0, int64_t t1, double *out)
+{
+    int64_t tpr = cols / n;
+    int status = 0;
+    (void)rows;
+    for (int64_t t = t0; t < t1; t++) {
+        int64_t r = t / tpr, j = t % tpr;
+        int nw = (off[t + 1] >= off[t]) ? (int)(off[t + 1] - off[t]) : -1;
+        if (nw < 0) {
+            for (int i = 0; i < n; i++) out[r * cols + j * n + i] = 0.0;
+            status |= HQO_CORRUPT;
+            continue;
+        }
+        status |= hqo_decode_tile(payload + off[t], nw, n, lattice, scale[t], kk[t], seed,
+                                  (uint64_t)j, (uint64_t)t, dither, out + r * cols + j * n);
+    }
+    return status;
+}
+
+/* GEMV reference: y_r = sum_c w_hat[r][c] x[c], in binary64, from the
+ * binary64 decode of rows [r0, r1). */
+int hqo_gemv_rows(const uint32_t *payload, const uint32_t *off, const uint16_t *scale,
+                  const uint8_t *kk, int64_t rows, int64_t cols, int n, int lattice, uint64_t seed,
+                  const double *x, int64_t r0, int64_t r1, double *y)
+{
+    int64_t tpr = cols / n;
+    int status = 0;
+    double *row = (double *)malloc(sizeof(double) * (size_t)cols);
+    if (!row) return -1;
+    (void)rows;
+    for (int64_t r = r0; r < r1; r++) {
+        for (int64_t j = 0; j < tpr; j++) {
+            int64_t t = r * tpr + j;
+            int nw = (off[t + 1] >= off[t]) ? (int)(off[t + 1] - off[t]) : -1;
+            if (nw < 0) {
+                for (int i = 0; i < n; i++) row[j * n + i] = 0.0;
+                status |= HQO_CORRUPT;
+                continue;
+            }
+            status |= hqo_decode_tile(payload + off[t], nw, n, lattice, scale[t], kk[t], seed,
+                                      (uint64_t)j, (uint64_t)t, 0, row + j * n);
+        }
+        double acc = 0.0;
+        for (int64_t c = 0; c < cols; c++) acc += row[c] * x[c];
+        y[r - r0] = acc;
+    }
+    free(row);
+    return status;
+}
+
+/* Nearest points of `count` vectors stored back to back (d floats each). */
+void hqo_nearest_batch(int lattice, const float *x, int64_t count, int32_t *c, int32_t *z,
+                       float *pt)
+{
+    int d = lattice;
+    for (int64_t q = 0; q < count; q++) {
+        int cc;
+        hqo_nearest(lattice, x + q * d, &cc, z + q * d, pt + q * d);
+        c[q] = cc;
+    }
+}
