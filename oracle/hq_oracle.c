@@ -163,12 +163,15 @@ static float bf16_to_float(uint16_t b)
 }
 
 /* Delta = bf16(c * sqrt(S)).  A non-finite S marks the tile non-finite;
- * a zero or subnormal Delta (and any non-finite tile) is stored as 0 and the
- * tile's lattice points are all zero. */
+ * a non-finite tile, a tile with S < 2^-96 (energy so small that squares of
+ * its entries underflow, which would let S understate the tile and the
+ * rotated coordinates outgrow the payload bound) and a zero or subnormal
+ * Delta are all stored as Delta = 0 with all lattice points zero. */
 uint16_t hqo_tile_scale(float S, float c, int *nonfinite)
 {
     *nonfinite = !isfinite(S);
     if (*nonfinite) return 0;
+    if (S < 0x1p-96f) return 0;
     float sigma = sqrtf(S);
     float d32 = c * sigma;
     uint16_t b = bf16_bits(d32);

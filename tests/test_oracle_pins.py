@@ -342,6 +342,13 @@ def test_zero_and_nonfinite_tiles():
     assert oracle.encode_tile(w, "E8", 4.0, 1)["status"] == oracle.NONFINITE
     st, out = oracle.decode_tile(z["words"], 256, "E8", 0, 0, 1)
     assert st == 0 and np.all(out == 0)
+    # energy below 2^-96: coded as zero without a status bit; just above: a real tile
+    tiny = np.zeros(256, np.float32)
+    tiny[3] = 2.0**-49
+    r = oracle.encode_tile(tiny, "E8", 4.0, 1)
+    assert r["scale"] == 0 and r["status"] == 0 and np.array_equal(r["words"], z["words"])
+    tiny[3] = 2.0**-47
+    assert oracle.encode_tile(tiny, "E8", 4.0, 1)["scale"] != 0
 
 
 def mse_closed_form(lat, delta, n):
