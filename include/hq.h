@@ -1,0 +1,185 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) HyperQuant per-tile codec.
+ *
+ * The method (sources cited by page title and section):
+ *   [V1] "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline for
+ *        Large Language and Diffusion Models", section "Abstract (arXiv)":
+ *        (i) per-tile randomized Hadamard transform, (ii) quantization to a
+ *        low-dimensional lattice E8, D4, A2 or Z, (iii) lossless
+ *        bit-stripping and Rice coding of the lattice indices, (iv) a KV-cache
+ *        bias correction keeping inner products unbiased.
+ *   [V2] "HyperQuant: A Near-Entropy-Optimal Lattice Quantization Pipeline
+ *        for Large Language and Diffusion Models", abstract: the rotation
+ *        whitens each tile, the strip removes the bits lattice membership
+ *        fixes, a Rice code carries the remainder, decoding is algebraic, and
+ *        the KV cache uses subtractive dither; a batch-1 decode path is
+ *        compared with a bf16 GEMV.
+ *
+ * Data model.  A matrix is row-major, `rows` x `cols`, `cols` a multiple of
+ * the tile length n.  Tile t = r * (cols / n) + j is the row segment
+ * x[r][j n .. j n + n).  For every tile the codec computes
+ *     v = H (s_j . w)           s_j: seeded random signs of column tile j,
+ *                               H: unnormalised Sylvester-Hadamard matrix
+ *     Delta = bf16(c(lattice, bps) * sqrt(sum w^2))
+ *     y = Q_lattice(v / Delta [+ dither])
+ * strips the bits membership fixes, zigzags the remaining integers and
+ * Rice-codes them with the tile's own parameter k.  Decoding returns
+ *     w_hat = s_j . H (Delta (y [- dither])) / n.
+ *
+ * Stream.  The caller owns every buffer (device memory, e.g. from
+ * torch.empty); the library never allocates, never synchronises, and runs
+ * every call asynchronously on the given CUDA stream (`stream` is a
+ * cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   payload     32-bit words; tile t occupies words [tile_off[t], tile_off[t+1])
+ *   tile_off    ntiles + 1 word offsets; tile_off[0] = 0,
+ *               tile_off[ntiles] = total payload words
+ *   tile_scale  ntiles bf16 bit patterns of Delta (0 = all-zero tile)
+ *   tile_k      ntiles Rice parameters, 0..15
+ * Tile layout, bits LSB-first in little-endian words: the n/d coset bits
+ * (E8 and A2 only), then k low bits of each of the n codes in coordinate
+ * order, then for each code q = u >> k zero bits and a one bit, then zero
+ * padding to a word.
+ *
+ * Errors.  Functions return HQ_OK or an HQ_ERR_* code synchronously for bad
+ * arguments or a failed launch; nothing is launched then.  Conditions found
+ * on the device are OR-ed into *d_status (a caller-owned device int32; pass
+ * NULL to skip): HQ_ST_NONFINITE (a tile held NaN/Inf or its sum of squares
+ * overflowed: it is encoded as an all-zero tile), HQ_ST_CAPACITY (payload
+ * too small: words past the capacity are not written), HQ_ST_CORRUPT (a
+ * decoded tile is not a canonical tile: its output is zero), HQ_ST_TIMEOUT
+ * (a bounded wait between thread blocks gave up: the call's output is
+ * invalid).
+ *
+ * The same seed must be given to encode and decode: signs and dither are
+ * regenerated from it, not stored.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* lattices; the value is the lattice dimension d */
+enum { HQ_Z = 1, HQ_A2 = 2, HQ_D4 = 4, HQ_E8 = 8 };
+
+/* element types of dense inputs / outputs */
+enum { HQ_BF16 = 0, HQ_F32 = 1 };
+
+/* synchronous return codes */
+enum {
+    HQ_OK = 0,
+    HQ_ERR_ARG = 1,          /* null pointer, bad size, tile, lattice, bps or dtype */
+    HQ_ERR_UNSUPPORTED = 2,  /* valid request outside what this build handles */
+    HQ_ERR_CAPACITY = 3,     /* payload capacity below the worst-case bound */
+    HQ_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+    HQ_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
+};
+
+/* device status bits OR-ed into *d_status */
+enum { HQ_ST_NONFINITE = 1, HQ_ST_CAPACITY = 2, HQ_ST_CORRUPT = 4, HQ_ST_TIMEOUT = 8 };
+
+/* A compressed matrix.  Host struct; all pointers are device memory owned by
+ * the caller.  Sizes: payload >= hq_max_payload_words(...) words for encode
+ * (the exact count is tile_off[ntiles] afterwards), tile_off ntiles + 1,
+ * tile_scale ntiles, tile_k ntiles. */
+typedef struct hq_stream {
+    uint32_t *payload;
+    uint64_t payload_capacity_words;
+    uint32_t *tile_off;
+    uint16_t *tile_scale;
+    uint8_t *tile_k;
+} hq_stream;
+
+/* Static description of a return code (never NULL). */
+const char *hq_error_string(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int hq_version(void);
+
+/* c(lattice, bps) = fp32(sqrt(2 pi e) 2^-bps V^(-1/d)), V the lattice cell
+ * volume (E8 1, D4 2, A2 sqrt3/2, Z 1): Delta = bf16(c sqrt(sum w^2)) puts
+ * the high-resolution entropy of the lattice indices at `bps` bits per
+ * coordinate for Gaussian tiles.  The pages name a per-tile scale for the
+ * target rate but not its rule; this is the reading ([V1] (ii), [V2]).
+ * Host only.  HQ_ERR_ARG for a bad lattice, bps outside (0, 8] or out == NULL. */
+int hq_rate_constant(int lattice, float bps, float *out);
+
+/* Worst-case words of one tile: n/d coset bits + n (1 + kb) bits rounded up,
+ * kb the bits of the largest zigzag symbol a tile can produce (the rotated
+ * coordinates obey |v_i| <= sqrt(n sum w^2)).  Host only. */
+int hq_tile_bound_words(int tile, int lattice, float bps, uint32_t *out);
+
+/* ntiles * hq_tile_bound_words: a payload this large never overflows.
+ * HQ_ERR_UNSUPPORTED if the bound reaches 2^32 words (offsets are 32-bit). */
+int hq_max_payload_words(int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                         uint64_t *out);
+
+/* Bytes of device workspace hq_encode / hq_kv_encode need for this shape
+ * (a chunk counter and one 64-bit prefix slot per chunk of tiles, used by
+ * the single-pass decoupled look-back scan that assigns tile offsets).
+ * Host only. */
+int hq_encode_workspace_bytes(int64_t rows, int64_t cols, int tile, uint64_t *out);
+
+/* Encode ([V1] (i)-(iii), [V2]).
+ *   x          device, rows x cols, HQ_BF16 or HQ_F32 (`dtype`), 16-byte aligned
+ *   rows, cols rows >= 0, cols >= 0, cols % tile == 0 (0 rows or cols: empty
+ *              stream, tile_off[0] = 0)
+ *   tile       n in {64, 128, 256, 512, 1024}
+ *   lattice    HQ_E8, HQ_D4, HQ_A2 or HQ_Z
+ *   bps        target bits per coordinate, 0 < bps <= 8
+ *   seed       signs of the rotation
+ *   out        stream to fill; payload_capacity_words >= hq_max_payload_words
+ *   workspace  device, >= hq_encode_workspace_bytes, 8-byte aligned; its
+ *              contents are overwritten (it is cleared on `stream` first)
+ * Tiles are encoded independently except for their offsets, which a single
+ * pass assigns with a decoupled look-back prefix scan over chunks of tiles. */
+int hq_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+              float bps, uint64_t seed, const hq_stream *out, void *workspace,
+              uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
+/* KV-cache encode ([V1] (iv), [V2] subtractive dither): as hq_encode, with a
+ * seeded dither uniform on the lattice's Voronoi cell added before the
+ * nearest-point step.  A KV slab is laid out as (heads * tokens) rows of
+ * head_dim columns, tile = head_dim, so each tile is one cached vector. */
+int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+                 float bps, uint64_t seed, const hq_stream *out, void *workspace,
+                 uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
+/* Decode ([V2] algebraic decoding): y = s . H (Delta y_lattice) / n per tile,
+ * rounded to `dtype` (bf16 round-to-nearest-even, or fp32).
+ *   in         stream written by hq_encode with the same shape, tile,
+ *              lattice, bps and seed
+ *   y          device, rows x cols, 16-byte aligned
+ * A tile whose words are not a canonical tile (bad offsets, k > 15, wrong
+ * symbol count, a set padding bit) is written as zeros and HQ_ST_CORRUPT is
+ * raised; no read leaves [tile_off[t], tile_off[t+1]) or the capacity. */
+int hq_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+              uint64_t seed, void *y, int dtype, void *stream, int32_t *d_status);
+
+/* KV-cache decode: as hq_decode, subtracting the same dither
+ * (w_hat = s . H (Delta (y - delta)) / n). */
+int hq_kv_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice,
+                 float bps, uint64_t seed, void *y, int dtype, void *stream, int32_t *d_status);
+
+/* Fused decode + GEMV at batch 1 ([V2] batch-1 decode path):
+ *   y[r] = sum_c w_hat[r][c] x[c], fp32 accumulation, without forming w_hat.
+ * Because H is symmetric, each tile contributes
+ *   (Delta / n) <y_lattice, H (s_j . x_j)>,
+ * so x is rotated once per column tile and the per-tile inverse rotation
+ * disappears.
+ *   w          stream of a rows x cols matrix (no dither)
+ *   x          device bf16, cols entries, 16-byte aligned
+ *   y          device fp32, rows entries
+ * cols * 4 bytes of rotated x must fit in shared memory (cols <= 40960). */
+int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice,
+                   float bps, uint64_t seed, const void *x, float *y, void *stream,
+                   int32_t *d_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

@@ -1,0 +1,283 @@
+// hq_api.cu -- host side of the C ABI declared in include/hq.h: argument
+// validation, sizing rules, hash keys and kernel dispatch.  No allocation,
+// no synchronisation; everything is enqueued on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "../../include/hq.h"
+#include "hq_internal.h"
+
+namespace hq {
+
+int sm_count()
+{
+    static int cached[64] = { 0 };
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+}  // namespace hq
+
+namespace {
+
+using namespace hq;
+
+bool valid_tile(int tile) { return tile == 64 || tile == 128 || tile == 256 || tile == 512 || tile == 1024; }
+bool valid_lattice(int d) { return d == HQ_Z || d == HQ_A2 || d == HQ_D4 || d == HQ_E8; }
+bool valid_bps(float b) { return std::isfinite(b) && b > 0.0f && b <= 8.0f; }
+bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+double cell_volume(int lattice)
+{
+    switch (lattice) {
+    case HQ_E8: return 1.0;
+    case HQ_D4: return 2.0;
+    case HQ_A2: return std::sqrt(3.0) / 2.0;
+    default: return 1.0;
+    }
+}
+
+float rate_constant(int lattice, float bps)
+{
+    const double c = std::sqrt(2.0 * M_PI * M_E) * std::pow(2.0, -(double)bps) *
+                     std::pow(cell_volume(lattice), -1.0 / (double)lattice);
+    return (float)c;
+}
+
+// Largest zigzag symbol a tile can produce, from |v_i| <= sqrt(n sum w^2):
+// |x_i| <= sqrt(n) / c (1 + 2^-7) covering the rounding of S, sqrt, c and
+// bf16(Delta); dither adds at most 1 per coordinate, each coset's rounding
+// moves a coordinate at most 1.5, so |z| <= X + 2.5 and u <= 2 |z|.
+uint32_t tile_bound_words(int tile, int lattice, float bps)
+{
+    const double c = (double)rate_constant(lattice, bps);
+    const double X = std::sqrt((double)tile) / c * (1.0 + 1.0 / 128.0) + 3.0;
+    const uint64_t umax = 2ull * (uint64_t)std::ceil(X);
+    int kb = 0;
+    while (kb < 63 && (umax >> kb) != 0) ++kb;
+    const int k = kb < 15 ? kb : 15;
+    const uint64_t coset = (lattice == HQ_E8 || lattice == HQ_A2) ? (uint64_t)(tile / lattice) : 0;
+    const uint64_t bits = coset + (uint64_t)tile * (1 + k) + (uint64_t)tile * (umax >> k);
+    return (uint32_t)((bits + 31) / 32);
+}
+
+A2Consts a2_consts() { return A2Consts{ (float)std::sqrt(3.0), (float)(1.0 / std::sqrt(3.0)) }; }
+
+int check_stream(const hq_stream *s, int64_t ntiles, bool need_payload)
+{
+    if (!s) return HQ_ERR_ARG;
+    if (!s->tile_off) return HQ_ERR_ARG;
+    if (ntiles > 0 && (!s->tile_scale || !s->tile_k || (need_payload && !s->payload))) return HQ_ERR_ARG;
+    return HQ_OK;
+}
+
+int common_shape(int64_t rows, int64_t cols, int tile, int lattice, float bps, int64_t *ntiles)
+{
+    if (rows < 0 || cols < 0 || !valid_tile(tile) || !valid_lattice(lattice) || !valid_bps(bps)) return HQ_ERR_ARG;
+    if (cols % tile) return HQ_ERR_ARG;
+    const int64_t tpr = cols / tile;
+    if (tpr && rows > (int64_t)(INT64_MAX / 2) / tpr) return HQ_ERR_UNSUPPORTED;
+    *ntiles = rows * tpr;
+    if (*ntiles >= (int64_t)1 << 40) return HQ_ERR_UNSUPPORTED;
+    return HQ_OK;
+}
+
+int64_t nchunks_for(int64_t ntiles, int tile)
+{
+    const int T = encode_chunk_tiles(tile);
+    return (ntiles + T - 1) / T;
+}
+
+int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                uint64_t seed, const hq_stream *out, void *workspace, uint64_t workspace_bytes,
+                void *stream, int32_t *d_status, bool dither)
+{
+    int64_t ntiles = 0;
+    int rc = common_shape(rows, cols, tile, lattice, bps, &ntiles);
+    if (rc) return rc;
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if ((rc = check_stream(out, ntiles, true))) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ntiles == 0) return cudaMemsetAsync(out->tile_off, 0, sizeof(uint32_t), s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
+    const uint32_t wmax = tile_bound_words(tile, lattice, bps);
+    const uint64_t need = (uint64_t)ntiles * wmax;
+    if (need >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
+    if (out->payload_capacity_words < need) return HQ_ERR_CAPACITY;
+    const int64_t nchunks = nchunks_for(ntiles, tile);
+    const uint64_t ws_need = 256 + 8 * (uint64_t)nchunks;
+    if (!workspace || !aligned(workspace, 8) || workspace_bytes < ws_need) return HQ_ERR_WORKSPACE;
+    if (nchunks >= (int64_t)1 << 31) return HQ_ERR_UNSUPPORTED;
+
+    if (cudaMemsetAsync(workspace, 0, ws_need, s) != cudaSuccess) return HQ_ERR_CUDA;
+    EncodeArgs a{};
+    a.x = x;
+    a.ntiles = ntiles;
+    a.tiles_per_row = cols / tile;
+    a.c = rate_constant(lattice, bps);
+    a.a2 = a2_consts();
+    a.sign_key = hash_key(seed, 1);
+    a.dither_key = hash_key(seed, 2);
+    a.payload = out->payload;
+    a.cap = out->payload_capacity_words;
+    a.off = out->tile_off;
+    a.scale = out->tile_scale;
+    a.kk = out->tile_k;
+    a.ticket = static_cast<uint32_t *>(workspace);
+    a.lb = reinterpret_cast<unsigned long long *>(static_cast<char *>(workspace) + 256);
+    a.status = d_status;
+    a.wmax = wmax;
+    a.nchunks = (uint32_t)nchunks;
+    return launch_encode(tile, lattice, dither, dtype, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+int decode_common(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                  uint64_t seed, DecodeArgs &a, int64_t *ntiles)
+{
+    int rc = common_shape(rows, cols, tile, lattice, bps, ntiles);
+    if (rc) return rc;
+    if ((rc = check_stream(in, *ntiles, true))) return rc;
+    a.payload = in->payload;
+    a.cap = in->payload_capacity_words;
+    a.off = in->tile_off;
+    a.scale = in->tile_scale;
+    a.kk = in->tile_k;
+    a.ntiles = *ntiles;
+    a.tiles_per_row = tile ? cols / tile : 0;
+    a.a2 = a2_consts();
+    a.sign_key = hash_key(seed, 1);
+    a.dither_key = hash_key(seed, 2);
+    a.wmax = tile_bound_words(tile, lattice, bps);
+    a.rows = rows;
+    return HQ_OK;
+}
+
+int decode_impl(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                uint64_t seed, void *y, int dtype, void *stream, int32_t *d_status, bool dither)
+{
+    DecodeArgs a{};
+    int64_t ntiles = 0;
+    int rc = decode_common(in, rows, cols, tile, lattice, bps, seed, a, &ntiles);
+    if (rc) return rc;
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (ntiles == 0) return HQ_OK;
+    if (!y || !aligned(y, 16)) return HQ_ERR_ARG;
+    a.y = y;
+    a.status = d_status;
+    return launch_decode(tile, lattice, dither, dtype, a, (cudaStream_t)stream) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hq_error_string(int code)
+{
+    switch (code) {
+    case HQ_OK: return "ok";
+    case HQ_ERR_ARG: return "invalid argument";
+    case HQ_ERR_UNSUPPORTED: return "unsupported size or configuration";
+    case HQ_ERR_CAPACITY: return "payload capacity below the worst-case bound";
+    case HQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case HQ_ERR_CUDA: return "CUDA call or kernel launch failed";
+    default: return "unknown error";
+    }
+}
+
+int hq_version(void) { return 100; }
+
+int hq_rate_constant(int lattice, float bps, float *out)
+{
+    if (!out || !valid_lattice(lattice) || !valid_bps(bps)) return HQ_ERR_ARG;
+    *out = rate_constant(lattice, bps);
+    return HQ_OK;
+}
+
+int hq_tile_bound_words(int tile, int lattice, float bps, uint32_t *out)
+{
+    if (!out || !valid_tile(tile) || !valid_lattice(lattice) || !valid_bps(bps)) return HQ_ERR_ARG;
+    *out = tile_bound_words(tile, lattice, bps);
+    return HQ_OK;
+}
+
+int hq_max_payload_words(int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t *out)
+{
+    int64_t ntiles = 0;
+    if (!out) return HQ_ERR_ARG;
+    int rc = common_shape(rows, cols, tile, lattice, bps, &ntiles);
+    if (rc) return rc;
+    const uint64_t w = (uint64_t)ntiles * tile_bound_words(tile, lattice, bps);
+    if (w >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
+    *out = w;
+    return HQ_OK;
+}
+
+int hq_encode_workspace_bytes(int64_t rows, int64_t cols, int tile, uint64_t *out)
+{
+    if (!out || rows < 0 || cols < 0 || !valid_tile(tile) || cols % tile) return HQ_ERR_ARG;
+    const int64_t ntiles = rows * (cols / tile);
+    *out = 256 + 8 * (uint64_t)nchunks_for(ntiles, tile);
+    return HQ_OK;
+}
+
+int hq_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+              uint64_t seed, const hq_stream *out, void *workspace, uint64_t workspace_bytes, void *stream,
+              int32_t *d_status)
+{
+    return encode_impl(x, dtype, rows, cols, tile, lattice, bps, seed, out, workspace, workspace_bytes, stream,
+                       d_status, false);
+}
+
+int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                 uint64_t seed, const hq_stream *out, void *workspace, uint64_t workspace_bytes, void *stream,
+                 int32_t *d_status)
+{
+    return encode_impl(x, dtype, rows, cols, tile, lattice, bps, seed, out, workspace, workspace_bytes, stream,
+                       d_status, true);
+}
+
+int hq_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t seed,
+              void *y, int dtype, void *stream, int32_t *d_status)
+{
+    return decode_impl(in, rows, cols, tile, lattice, bps, seed, y, dtype, stream, d_status, false);
+}
+
+int hq_kv_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                 uint64_t seed, void *y, int dtype, void *stream, int32_t *d_status)
+{
+    return decode_impl(in, rows, cols, tile, lattice, bps, seed, y, dtype, stream, d_status, true);
+}
+
+int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                   uint64_t seed, const void *x, float *y, void *stream, int32_t *d_status)
+{
+    DecodeArgs a{};
+    int64_t ntiles = 0;
+    int rc = decode_common(w, rows, cols, tile, lattice, bps, seed, a, &ntiles);
+    if (rc) return rc;
+    if (cols > 40960) return HQ_ERR_UNSUPPORTED;
+    if (rows > 0 && !y) return HQ_ERR_ARG;
+    if (ntiles == 0) {
+        if (rows > 0)
+            return cudaMemsetAsync(y, 0, sizeof(float) * (size_t)rows, (cudaStream_t)stream) == cudaSuccess
+                       ? HQ_OK : HQ_ERR_CUDA;
+        return HQ_OK;
+    }
+    if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
+    a.x = x;
+    a.gy = y;
+    a.status = d_status;
+    return launch_gemv(tile, lattice, a, cols, (cudaStream_t)stream) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // extern "C"

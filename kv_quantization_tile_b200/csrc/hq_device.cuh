@@ -1,0 +1,299 @@
+// hq_device.cuh -- device building blocks of the sm_100a HyperQuant codec.
+//
+// A tile of n coordinates is held by a group of LPT = n / EPL lanes of one
+// warp, EPL coordinates per lane, coordinate i = lane_in_group * EPL + r.
+// Index bits below log2(EPL) live in registers, the others across lanes, so
+// butterfly stages and pairwise reductions over index bit b run in
+// registers for b < log2(EPL) and as __shfl_xor over lanes otherwise.
+//
+// Every floating-point step that decides an integer (rotation, scale,
+// nearest point, dither) uses the _rn intrinsics so nothing is contracted
+// into an FMA and each operation rounds once to nearest-even, as the
+// method's definition of the codec does.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace hq {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+// SplitMix64 output function (Steele, Lea & Flood 2014).
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z)
+{
+    z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+    z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+    return z ^ (z >> 31);
+}
+
+// Per-call hash key of a tag: H(seed, tag, a, b) = mix64(mix64(key ^ a) ^ b).
+__host__ __forceinline__ uint64_t hash_key(uint64_t seed, uint64_t tag)
+{
+    return mix64(seed + kGamma * (tag + 1));
+}
+
+// ------------------------------------------------------------- groups
+template <int LPT>
+__device__ __forceinline__ unsigned group_mask(int lane)
+{
+    if constexpr (LPT == 32) return FULL;
+    else return ((1u << LPT) - 1u) << (lane & ~(LPT - 1));
+}
+
+template <int LPT>
+__device__ __forceinline__ uint32_t group_sum(unsigned mask, uint32_t v)
+{
+    return __reduce_add_sync(mask, v);
+}
+
+template <int LPT>
+__device__ __forceinline__ uint32_t group_max(unsigned mask, uint32_t v)
+{
+    return __reduce_max_sync(mask, v);
+}
+
+// exclusive prefix sum over the lanes of a group
+template <int LPT>
+__device__ __forceinline__ uint32_t group_excl_scan(unsigned mask, uint32_t v, int l)
+{
+    uint32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < LPT; d <<= 1) {
+        uint32_t o = __shfl_up_sync(mask, incl, d, LPT);
+        if (l >= d) incl += o;
+    }
+    return incl - v;
+}
+
+// ------------------------------------------------------------- rotation
+// Unnormalised Walsh-Hadamard transform, stages h = 1, 2, ..., n/2 in that
+// order; the lower index of each pair keeps the sum, the upper the
+// difference (lower - upper).  For lane stages the upper lane computes
+// other - own as fma(-1, own, other), exactly one rounding of the same
+// difference.
+template <int EPL, int LPT>
+__device__ __forceinline__ void fwht(float (&v)[EPL], unsigned mask, int l)
+{
+#pragma unroll
+    for (int h = 1; h < EPL; h <<= 1) {
+#pragma unroll
+        for (int a = 0; a < EPL; a++) {
+            if (!(a & h)) {
+                float p = v[a], q = v[a + h];
+                v[a] = __fadd_rn(p, q);
+                v[a + h] = __fsub_rn(p, q);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < LPT; m <<= 1) {
+        const float sg = (l & m) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int a = 0; a < EPL; a++) {
+            float o = __shfl_xor_sync(mask, v[a], m);
+            v[a] = __fmaf_rn(sg, v[a], o);
+        }
+    }
+}
+
+// Sum of squares by the pairwise tree over index bits (bit 0 first).
+template <int EPL, int LPT>
+__device__ __forceinline__ float sumsq(const float (&w)[EPL], unsigned mask)
+{
+    float a[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; i++) a[i] = __fmul_rn(w[i], w[i]);
+#pragma unroll
+    for (int h = 1; h < EPL; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < EPL; i++)
+            if (!(i & h) && (i % (2 * h)) == 0) a[i] = __fadd_rn(a[i], a[i + h]);
+    float s = a[0];
+#pragma unroll
+    for (int m = 1; m < LPT; m <<= 1) s = __fadd_rn(s, __shfl_xor_sync(mask, s, m));
+    return s;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Delta as bf16 bits: 0 for a non-finite S (flagged), S < 2^-96, or a zero /
+// subnormal result.
+__device__ __forceinline__ uint32_t tile_scale_bits(float S, float c, bool &nonfinite)
+{
+    nonfinite = (__float_as_uint(S) & 0x7f800000u) == 0x7f800000u;
+    if (nonfinite || S < 0x1p-96f) return 0;
+    float d32 = __fmul_rn(c, __fsqrt_rn(S));
+    uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(d32));
+    return (b & 0x7f80u) ? b : 0u;
+}
+
+// ------------------------------------------------------------- lattices
+// Conway & Sloane (1982) nearest points.  Ties: rint to even; D_n flips the
+// first coordinate of largest |x - rint x| towards x (up when exact); E8 and
+// A2 keep coset 0 when both squared distances are equal.
+template <int D>
+__device__ __forceinline__ void dn_round(const float (&x)[D], float (&f)[D])
+{
+    float e[D];
+    float sum = 0.0f;
+#pragma unroll
+    for (int i = 0; i < D; i++) {
+        f[i] = rintf(x[i]);
+        e[i] = __fsub_rn(x[i], f[i]);
+        sum = __fadd_rn(sum, f[i]);   // small integers: exact
+    }
+    if (__float2int_rn(sum) & 1) {
+        int b = 0;
+        float ab = fabsf(e[0]), eb = e[0];
+#pragma unroll
+        for (int i = 1; i < D; i++) {
+            float a = fabsf(e[i]);
+            if (a > ab) { ab = a; eb = e[i]; b = i; }
+        }
+        const float dir = (eb >= 0.0f) ? 1.0f : -1.0f;
+#pragma unroll
+        for (int i = 0; i < D; i++)
+            if (i == b) f[i] = __fadd_rn(f[i], dir);
+    }
+}
+
+struct A2Consts {
+    float s3;     // fp32(sqrt 3)
+    float inv_s3; // fp32(1 / sqrt 3)
+};
+
+// Nearest point of one D-dimensional vector: coset bit, integer coordinates
+// (pre-strip), and the point in binary32.
+template <int D>
+__device__ __forceinline__ void nearest(const float (&x)[D], int &c, int (&z)[D], float (&p)[D],
+                                        const A2Consts &a2)
+{
+    c = 0;
+    if constexpr (D == 1) {
+        p[0] = rintf(x[0]);
+        z[0] = __float2int_rn(p[0]);
+    } else if constexpr (D == 4) {
+        dn_round<4>(x, p);
+#pragma unroll
+        for (int i = 0; i < 4; i++) z[i] = __float2int_rn(p[i]);
+    } else if constexpr (D == 8) {
+        float a[8], b[8], xs[8];
+        dn_round<8>(x, a);
+#pragma unroll
+        for (int i = 0; i < 8; i++) xs[i] = __fsub_rn(x[i], 0.5f);
+        dn_round<8>(xs, b);
+        float d0 = 0.0f, d1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            float t = __fsub_rn(x[i], a[i]);
+            d0 = __fadd_rn(d0, __fmul_rn(t, t));
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            float t = __fsub_rn(x[i], __fadd_rn(b[i], 0.5f));
+            d1 = __fadd_rn(d1, __fmul_rn(t, t));
+        }
+        const bool one = !(d0 <= d1);
+        c = one ? 1 : 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            float f = one ? b[i] : a[i];
+            z[i] = __float2int_rn(f);
+            p[i] = one ? __fadd_rn(b[i], 0.5f) : a[i];
+        }
+    } else {  // A2: points (a + c/2, (b + c/2) sqrt3)
+        float y1 = __fmul_rn(x[1], a2.inv_s3);
+        float a0 = rintf(x[0]), b0 = rintf(y1);
+        float a1 = rintf(__fsub_rn(x[0], 0.5f)), b1 = rintf(__fsub_rn(y1, 0.5f));
+        float p00 = a0, p01 = __fmul_rn(b0, a2.s3);
+        float p10 = __fadd_rn(a1, 0.5f), p11 = __fmul_rn(__fadd_rn(b1, 0.5f), a2.s3);
+        float t0 = __fsub_rn(x[0], p00), t1 = __fsub_rn(x[1], p01);
+        float d0 = __fadd_rn(__fmul_rn(t0, t0), __fmul_rn(t1, t1));
+        float u0 = __fsub_rn(x[0], p10), u1 = __fsub_rn(x[1], p11);
+        float d1 = __fadd_rn(__fmul_rn(u0, u0), __fmul_rn(u1, u1));
+        const bool one = !(d0 <= d1);
+        c = one ? 1 : 0;
+        z[0] = __float2int_rn(one ? a1 : a0);
+        z[1] = __float2int_rn(one ? b1 : b0);
+        p[0] = one ? p10 : p00;
+        p[1] = one ? p11 : p01;
+    }
+}
+
+// ------------------------------------------------------------- dither
+// r_i uniform on the 24-bit grid of [0,1): one hash per coordinate pair,
+// bits 40..63 for the even and 16..39 for the odd coordinate.
+__device__ __forceinline__ void uniform_pair(uint64_t tile_key, uint32_t pair, float &r0, float &r1)
+{
+    uint64_t h = mix64(tile_key ^ (uint64_t)pair);
+    r0 = (float)(uint32_t)(h >> 40) * 0x1p-24f;
+    r1 = (float)(uint32_t)((h >> 16) & 0xFFFFFFu) * 0x1p-24f;
+}
+
+// Dither of vector q (coordinates q*D .. q*D+D-1) of a tile: delta = x0 -
+// Q(x0), x0 uniform on a box that tiles space under a sublattice.
+template <int D>
+__device__ __forceinline__ void dither(uint64_t tile_key, uint32_t q, float (&delta)[D],
+                                       const A2Consts &a2)
+{
+    float x0[D], p[D];
+    int z[D], c;
+#pragma unroll
+    for (int m = 0; m < D; m += 2) {
+        float r0, r1;
+        if constexpr (D == 1) {
+            uint32_t i = q;
+            float e, o;
+            uniform_pair(tile_key, i >> 1, e, o);
+            r0 = (i & 1) ? o : e;
+            r1 = 0.0f;
+        } else {
+            uniform_pair(tile_key, (q * D + m) >> 1, r0, r1);
+        }
+        if constexpr (D == 8 || D == 4) {
+            x0[m] = __fmul_rn(2.0f, r0);
+            x0[m + 1] = __fmul_rn(2.0f, r1);
+        } else if constexpr (D == 2) {
+            x0[0] = r0;
+            x0[1] = __fmul_rn(r1, a2.s3);
+        } else {
+            x0[0] = r0;
+        }
+    }
+    nearest<D>(x0, c, z, p, a2);
+#pragma unroll
+    for (int m = 0; m < D; m++) delta[m] = __fsub_rn(x0[m], p[m]);
+}
+
+// ------------------------------------------------------------- symbols
+__device__ __forceinline__ uint32_t zigzag(int z) { return ((uint32_t)z << 1) ^ (uint32_t)(z >> 31); }
+__device__ __forceinline__ int unzigzag(uint32_t u) { return (int)(u >> 1) ^ -(int)(u & 1u); }
+
+// ------------------------------------------------------------- bits
+// OR `len` (<= 64) bits of v into a shared-memory bit buffer at bit `pos`.
+// The shifted value spans at most three words.
+__device__ __forceinline__ void or_bits(uint32_t *buf, uint32_t pos, uint64_t v, int len)
+{
+    if (len <= 0 || v == 0) return;
+    const uint32_t w = pos >> 5, sh = pos & 31;
+    const uint32_t b0 = (uint32_t)(v << sh);
+    const uint32_t b1 = sh ? (uint32_t)(v >> (32 - sh)) : (uint32_t)(v >> 32);
+    const uint32_t b2 = sh ? (uint32_t)(v >> (64 - sh)) : 0u;
+    if (b0) atomicOr(&buf[w], b0);
+    if (len + (int)sh > 32 && b1) atomicOr(&buf[w + 1], b1);
+    if (len + (int)sh > 64 && b2) atomicOr(&buf[w + 2], b2);
+}
+
+// `len` (<= 32) bits at bit `pos` of a word buffer (buf[pos/32 + 1] must be
+// readable).
+__device__ __forceinline__ uint32_t get_bits(const uint32_t *buf, uint32_t pos, int len)
+{
+    uint32_t w = pos >> 5, sh = pos & 31;
+    uint64_t v = (uint64_t)buf[w] | ((uint64_t)buf[w + 1] << 32);
+    uint32_t r = (uint32_t)(v >> sh);
+    return len >= 32 ? r : (r & ((1u << len) - 1u));
+}
+
+}  // namespace hq

@@ -1,0 +1,70 @@
+// hq_internal.h -- argument blocks and launchers shared by the host API and
+// the kernel translation units (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "hq_device.cuh"
+
+namespace hq {
+
+constexpr int kStatusNonfinite = 1, kStatusCapacity = 2, kStatusCorrupt = 4, kStatusTimeout = 8;
+
+// Look-back slot: bits 62..63 flag (1 = chunk aggregate, 2 = inclusive
+// prefix), bits 0..61 the word count.
+constexpr uint64_t kFlagAggregate = 1ull << 62, kFlagInclusive = 2ull << 62;
+constexpr uint64_t kValueMask = (1ull << 62) - 1;
+constexpr uint32_t kSpinLimit = 1u << 22;   // polls before a wait gives up
+
+struct EncodeArgs {
+    const void *x;
+    int64_t ntiles;
+    int64_t tiles_per_row;
+    float c;
+    A2Consts a2;
+    uint64_t sign_key;    // hash key of tag 1 (signs)
+    uint64_t dither_key;  // hash key of tag 2 (dither)
+    uint32_t *payload;
+    uint64_t cap;
+    uint32_t *off;
+    uint16_t *scale;
+    uint8_t *kk;
+    uint32_t *ticket;
+    unsigned long long *lb;
+    int32_t *status;
+    uint32_t wmax;        // worst-case words of one tile
+    uint32_t nchunks;
+};
+
+struct DecodeArgs {
+    const uint32_t *payload;
+    uint64_t cap;
+    const uint32_t *off;
+    const uint16_t *scale;
+    const uint8_t *kk;
+    int64_t ntiles;
+    int64_t tiles_per_row;
+    A2Consts a2;
+    uint64_t sign_key;
+    uint64_t dither_key;
+    int32_t *status;
+    uint32_t wmax;
+    void *y;              // decode output
+    const void *x;        // gemv input (bf16)
+    float *gy;            // gemv output
+    int64_t rows;
+};
+
+// Launch helpers; return a cudaError_t.
+cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
+                          cudaStream_t s);
+cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const DecodeArgs &a,
+                          cudaStream_t s);
+cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
+
+// Tiles per encode chunk (one thread block) for a tile length.
+int encode_chunk_tiles(int tile);
+int sm_count();
+
+}  // namespace hq

@@ -1,0 +1,221 @@
+"""Thin ctypes binding of the C ABI in ``include/hq.h`` (``libhq.so``).
+
+Names and argument order follow the C functions; this module only marshals
+torch tensors to device pointers and the current CUDA stream to a
+``cudaStream_t``.  Every step of the codec runs in the library's kernels.
+There is no fallback: if the library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhq.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                      "`python -c 'import __graft_entry__ as g; g.build()'`")
+
+HQ_Z, HQ_A2, HQ_D4, HQ_E8 = 1, 2, 4, 8
+HQ_BF16, HQ_F32 = 0, 1
+HQ_OK, HQ_ERR_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_CAPACITY, HQ_ERR_WORKSPACE, HQ_ERR_CUDA = range(6)
+HQ_ST_NONFINITE, HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT = 1, 2, 4, 8
+LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
+
+EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
+           "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
+           "hq_decode", "hq_kv_decode", "hq_decode_gemv"]
+
+
+class hq_stream(ctypes.Structure):
+    _fields_ = [("payload", ctypes.c_void_p), ("payload_capacity_words", ctypes.c_uint64),
+                ("tile_off", ctypes.c_void_p), ("tile_scale", ctypes.c_void_p),
+                ("tile_k", ctypes.c_void_p)]
+
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_i64, _u64, _i32, _f32, _vp = ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+_SIGS = {
+    "hq_error_string": (ctypes.c_char_p, [_i32]),
+    "hq_version": (_i32, []),
+    "hq_rate_constant": (_i32, [_i32, _f32, ctypes.POINTER(_f32)]),
+    "hq_tile_bound_words": (_i32, [_i32, _i32, _f32, ctypes.POINTER(ctypes.c_uint32)]),
+    "hq_max_payload_words": (_i32, [_i64, _i64, _i32, _i32, _f32, ctypes.POINTER(_u64)]),
+    "hq_encode_workspace_bytes": (_i32, [_i64, _i64, _i32, ctypes.POINTER(_u64)]),
+    "hq_encode": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
+                         _vp, _u64, _vp, _vp]),
+    "hq_kv_encode": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
+                            _vp, _u64, _vp, _vp]),
+    "hq_decode": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i32,
+                         _vp, _vp]),
+    "hq_kv_decode": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i32,
+                            _vp, _vp]),
+    "hq_decode_gemv": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _vp,
+                              _vp, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype, _fn.argtypes = _res, _args
+
+
+class HQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {hq_error_string(code)} (code {code})")
+        self.code = code
+
+
+def library():
+    return _lib
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _check(code: int, where: str):
+    if code != HQ_OK:
+        raise HQError(code, where)
+
+
+def _lat(lattice) -> int:
+    return LATTICES[lattice] if isinstance(lattice, str) else int(lattice)
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    return t.data_ptr()
+
+
+def _stream_handle(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HQ_BF16
+    if t.dtype == torch.float32:
+        return HQ_F32
+    raise TypeError("bf16 or fp32 tensors only")
+
+
+# ----------------------------------------------------------------- sizing
+def hq_error_string(code: int) -> str:
+    return _lib.hq_error_string(code).decode()
+
+
+def hq_version() -> int:
+    return _lib.hq_version()
+
+
+def hq_rate_constant(lattice, bps: float) -> float:
+    out = _f32(0)
+    _check(_lib.hq_rate_constant(_lat(lattice), bps, ctypes.byref(out)), "hq_rate_constant")
+    return out.value
+
+
+def hq_tile_bound_words(tile: int, lattice, bps: float) -> int:
+    out = ctypes.c_uint32(0)
+    _check(_lib.hq_tile_bound_words(tile, _lat(lattice), bps, ctypes.byref(out)), "hq_tile_bound_words")
+    return out.value
+
+
+def hq_max_payload_words(rows: int, cols: int, tile: int, lattice, bps: float) -> int:
+    out = _u64(0)
+    _check(_lib.hq_max_payload_words(rows, cols, tile, _lat(lattice), bps, ctypes.byref(out)),
+           "hq_max_payload_words")
+    return out.value
+
+
+def hq_encode_workspace_bytes(rows: int, cols: int, tile: int) -> int:
+    out = _u64(0)
+    _check(_lib.hq_encode_workspace_bytes(rows, cols, tile, ctypes.byref(out)), "hq_encode_workspace_bytes")
+    return out.value
+
+
+# ----------------------------------------------------------------- streams
+@dataclass
+class Stream:
+    """Device buffers of one compressed matrix (all owned by torch)."""
+    payload: torch.Tensor      # int32 words (bit patterns of uint32)
+    tile_off: torch.Tensor     # int32, ntiles + 1 (uint32 offsets)
+    tile_scale: torch.Tensor   # int16, ntiles (bf16 bits of Delta)
+    tile_k: torch.Tensor       # uint8, ntiles
+
+    def struct(self) -> hq_stream:
+        return hq_stream(_ptr(self.payload), self.payload.numel(), _ptr(self.tile_off),
+                         _ptr(self.tile_scale) if self.tile_scale.numel() else 0,
+                         _ptr(self.tile_k) if self.tile_k.numel() else 0)
+
+    def words(self) -> int:
+        """Payload words actually used (reads tile_off[-1]; synchronises)."""
+        return int(self.tile_off[-1].item()) & 0xFFFFFFFF
+
+    def nbytes(self) -> int:
+        """Compressed bytes: used payload words plus the per-tile headers."""
+        return 4 * self.words() + 4 * self.tile_off.numel() + 2 * self.tile_scale.numel() + self.tile_k.numel()
+
+
+def alloc_stream(rows: int, cols: int, tile: int, lattice, bps: float, device="cuda",
+                 capacity_words: int | None = None) -> Stream:
+    ntiles = rows * (cols // tile)
+    cap = capacity_words if capacity_words is not None else hq_max_payload_words(rows, cols, tile, lattice, bps)
+    return Stream(payload=torch.empty(max(cap, 1), dtype=torch.int32, device=device),
+                  tile_off=torch.empty(ntiles + 1, dtype=torch.int32, device=device),
+                  tile_scale=torch.empty(ntiles, dtype=torch.int16, device=device),
+                  tile_k=torch.empty(ntiles, dtype=torch.uint8, device=device))
+
+
+def alloc_workspace(rows: int, cols: int, tile: int, device="cuda") -> torch.Tensor:
+    return torch.empty(hq_encode_workspace_bytes(rows, cols, tile), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------- codec
+def _encode(fn, x: torch.Tensor, tile: int, lattice, bps: float, seed: int, out: Stream,
+            workspace: torch.Tensor, status: torch.Tensor | None, stream):
+    assert x.is_contiguous() and x.dim() == 2
+    rows, cols = x.shape
+    s = out.struct()
+    code = fn(_ptr(x), _dtype_code(x), rows, cols, tile, _lat(lattice), bps, seed, ctypes.byref(s),
+              _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status))
+    _check(code, fn.__name__)
+    return out
+
+
+def hq_encode(x, tile, lattice, bps, seed, out: Stream, workspace, status=None, stream=None) -> Stream:
+    return _encode(_lib.hq_encode, x, tile, lattice, bps, seed, out, workspace, status, stream)
+
+
+def hq_kv_encode(x, tile, lattice, bps, seed, out: Stream, workspace, status=None, stream=None) -> Stream:
+    return _encode(_lib.hq_kv_encode, x, tile, lattice, bps, seed, out, workspace, status, stream)
+
+
+def _decode(fn, s: Stream, rows: int, cols: int, tile: int, lattice, bps: float, seed: int,
+            y: torch.Tensor, status, stream):
+    assert y.is_contiguous() and tuple(y.shape) == (rows, cols)
+    st = s.struct()
+    _check(fn(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(y), _dtype_code(y),
+              _stream_handle(stream), _ptr(status)), fn.__name__)
+    return y
+
+
+def hq_decode(s: Stream, rows, cols, tile, lattice, bps, seed, y, status=None, stream=None):
+    return _decode(_lib.hq_decode, s, rows, cols, tile, lattice, bps, seed, y, status, stream)
+
+
+def hq_kv_decode(s: Stream, rows, cols, tile, lattice, bps, seed, y, status=None, stream=None):
+    return _decode(_lib.hq_kv_decode, s, rows, cols, tile, lattice, bps, seed, y, status, stream)
+
+
+def hq_decode_gemv(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, status=None, stream=None):
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.numel() == cols
+    assert y.dtype == torch.float32 and y.is_contiguous() and y.numel() == rows
+    st = s.struct()
+    _check(_lib.hq_decode_gemv(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), _ptr(y),
+                               _stream_handle(stream), _ptr(status)), "hq_decode_gemv")
+    return y

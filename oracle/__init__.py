@@ -79,10 +79,10 @@ def lib() -> ctypes.CDLL:
                                           i32, vp]),
                 "hqo_encode_tiles": (i32, [vp, i32, i64, i64, i32, i32, f32, u64, i32, i64, i64,
                                            vp, i32, vp, vp, vp]),
-                "hqo_decode_tiles": (i32, [vp, vp, vp, vp, i64, i64, i32, i32, u64, i32, i64, i64,
-                                           vp]),
-                "hqo_gemv_rows": (i32, [vp, vp, vp, vp, i64, i64, i32, i32, u64, vp, i64, i64,
-                                        vp]),
+                "hqo_decode_tiles": (i32, [vp, u64, vp, vp, vp, i64, i64, i32, i32, u64, i32, i64,
+                                           i64, vp]),
+                "hqo_gemv_rows": (i32, [vp, u64, vp, vp, vp, i64, i64, i32, i32, u64, vp, i64,
+                                        i64, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -331,6 +331,7 @@ def decode(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int,
     ntiles = rows * (cols // tile)
     out = np.zeros((rows, cols), np.float64)
     pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
+    cap = pay.size
     if pay.size == 0:
         pay = np.zeros(1, np.uint32)
     off = np.ascontiguousarray(stream["off"], dtype=np.uint32)
@@ -339,7 +340,7 @@ def decode(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int,
     L = lib()
 
     def run(r):
-        return L.hqo_decode_tiles(_p(pay), _p(off), _p(sc) if sc.size else 0,
+        return L.hqo_decode_tiles(_p(pay), cap, _p(off), _p(sc) if sc.size else 0,
                                   _p(kk) if kk.size else 0, rows, cols, tile, d, seed,
                                   int(dither), r[0], r[1], _p(out))
 
@@ -366,7 +367,7 @@ def gemv(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, x,
     off = np.ascontiguousarray(stream["off"], dtype=np.uint32)
     sc = np.ascontiguousarray(stream["scale"], dtype=np.uint16)
     kk = np.ascontiguousarray(stream["k"], dtype=np.uint8)
-    st = lib().hqo_gemv_rows(_p(pay), _p(off), _p(sc), _p(kk), rows, cols, tile, d, seed,
+    st = lib().hqo_gemv_rows(_p(pay), pay.size, _p(off), _p(sc), _p(kk), rows, cols, tile, d, seed,
                              _p(xa), r0, r1, _p(y))
     if st < 0:
         raise MemoryError

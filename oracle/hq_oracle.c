@@ -483,6 +483,9 @@ int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint1
     double v[HQO_MAX_TILE];
     int d = lattice, nv = n / lattice;
     int st = hqo_unpack_tile(lattice, n, k, words, nwords, coset, u);
+    /* the encoder only writes Delta = 0 or a positive, normal, finite bf16 */
+    if (scale != 0 && ((scale & 0x8000u) || (scale & 0x7F80u) == 0 || (scale & 0x7F80u) == 0x7F80u))
+        st = HQO_CORRUPT;
     if (st) {
         for (int i = 0; i < n; i++) out[i] = 0.0;
         return st;
@@ -543,18 +546,20 @@ int hqo_encode_tiles(const void *x, int dtype, int64_t rows, int64_t cols, int n
 }
 
 /* Decode tiles [t0, t1) of a stream given its offsets (off[t] .. off[t+1]
- * are the words of tile t) into out (binary64, row-major rows x cols,
- * only the decoded tiles are written).  Returns the OR of tile statuses. */
-int hqo_decode_tiles(const uint32_t *payload, const uint32_t *off, const uint16_t *scale,
-                     const uint8_t *kk, int64_t rows, int64_t cols, int n, int lattice,
-                     uint64_t seed, int dither, int64_t t0, int64_t t1, double *out)
+ * are the words of tile t, all below cap) into out (binary64, row-major
+ * rows x cols, only the decoded tiles are written).  A tile whose offsets
+ * are out of order or past cap is corrupt.  Returns the OR of tile
+ * statuses. */
+int hqo_decode_tiles(const uint32_t *payload, uint64_t cap, const uint32_t *off,
+                     const uint16_t *scale, const uint8_t *kk, int64_t rows, int64_t cols, int n,
+                     int lattice, uint64_t seed, int dither, int64_t t0, int64_t t1, double *out)
 {
     int64_t tpr = cols / n;
     int status = 0;
     (void)rows;
     for (int64_t t = t0; t < t1; t++) {
         int64_t r = t / tpr, j = t % tpr;
-        int nw = (off[t + 1] >= off[t]) ? (int)(off[t + 1] - off[t]) : -1;
+        int nw = (off[t + 1] >= off[t] && off[t + 1] <= cap) ? (int)(off[t + 1] - off[t]) : -1;
         if (nw < 0) {
             for (int i = 0; i < n; i++) out[r * cols + j * n + i] = 0.0;
             status |= HQO_CORRUPT;
@@ -568,7 +573,7 @@ int hqo_decode_tiles(const uint32_t *payload, const uint32_t *off, const uint16_
 
 /* GEMV reference: y_r = sum_c w_hat[r][c] x[c], in binary64, from the
  * binary64 decode of rows [r0, r1). */
-int hqo_gemv_rows(const uint32_t *payload, const uint32_t *off, const uint16_t *scale,
+int hqo_gemv_rows(const uint32_t *payload, uint64_t cap, const uint32_t *off, const uint16_t *scale,
                   const uint8_t *kk, int64_t rows, int64_t cols, int n, int lattice, uint64_t seed,
                   const double *x, int64_t r0, int64_t r1, double *y)
 {
@@ -580,7 +585,7 @@ int hqo_gemv_rows(const uint32_t *payload, const uint32_t *off, const uint16_t *
     for (int64_t r = r0; r < r1; r++) {
         for (int64_t j = 0; j < tpr; j++) {
             int64_t t = r * tpr + j;
-            int nw = (off[t + 1] >= off[t]) ? (int)(off[t + 1] - off[t]) : -1;
+            int nw = (off[t + 1] >= off[t] && off[t + 1] <= cap) ? (int)(off[t + 1] - off[t]) : -1;
             if (nw < 0) {
                 for (int i = 0; i < n; i++) row[j * n + i] = 0.0;
                 status |= HQO_CORRUPT;
