@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 HyperQuant codec.
+
+A step is one pass of the codec over one Llama-3.1-8B-shaped decoder layer
+(seven bf16 matrices, 218,103,808 weights, N(0, 0.02^2) with 0.1 % outlier
+columns x20): E8 lattice at 4 bits per coordinate, tile 256 -- encode all
+seven, then decode all seven back to bf16.  `value` is bf16 GB/s of encode
+input plus decode output over the whole job (all ranks), with the inputs
+resident in HBM.  Each rank encodes its own layer (independent problems: weak
+scaling, no collective on the data path).
+
+Also reported: per-kernel roofline of the dominant kernel (algorithmic bytes
+/ CUDA-event time on the launching stream), the end-to-end figure through the
+C ABI from pinned host buffers, the batch-1 decode-GEMV and KV-cache paths,
+the CPU oracle timed on a bounded sample, and SM clocks sampled during the
+timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "E8 4-bps encode/decode GB/s of bf16 in/out and % of B200 HBM roofline"
+TILE, LAT, BPS, SEED = 256, "E8", 4.0, 42
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    """nvidia-smi samples (200 ms) of one GPU during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index, self.lines, self.proc = index, [], None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ oracle leg
+def cpu_baseline(seconds: float):
+    """The CPU oracle (as it stands) on a bounded sample of the gate matrix:
+    encode + decode of whole rows until `seconds` of wall time have passed,
+    one thread per core over disjoint row blocks."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from kv_quantization_tile_b200 import workloads
+
+    cores = len(os.sched_getaffinity(0))
+    gate = workloads.outlier_weight(14336, 4096, 1004, 1104, "cpu")
+    bits = gate.view(torch.int16).numpy().view(np.uint16)
+    oracle.build()
+    rows_per_block = 8
+    done_rows, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds and done_rows < bits.shape[0]:
+        blk = bits[done_rows: done_rows + rows_per_block * cores]
+        s = oracle.encode(blk, TILE, LAT, BPS, SEED, threads=cores)
+        oracle.decode(s, blk.shape[0], blk.shape[1], TILE, LAT, SEED, threads=cores)
+        done_rows += blk.shape[0]
+    el = time.perf_counter() - t0
+    elems = done_rows * bits.shape[1]
+    return {"value": round(4 * elems / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"encode+decode of the first {done_rows} rows x 4096 of the gate matrix "
+                      f"({elems} weights, E8 4 bps, tile 256) in {el:.1f} s on {cores} threads"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per = max(2.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(per / 4)
+    vals = [cpu_baseline(per) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "llama3.1-8b-layer E8 4bps tile256 encode+decode (bounded CPU sample)"},
+        "cpu_baseline": cb, "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                    "d2h_bytes_per_step": 0}}))
+
+
+# ------------------------------------------------------------------ GPU leg
+def traffic_record(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (its sha256 is recorded beside it)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "kv_quantization_tile_b200", "csrc", kernel_file)
+    try:
+        rec = json.load(open(path))
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        r = rec.get(kernel_file)
+        if r and r.get("source_sha256") == sha:
+            return r
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    mats = workloads.llama_layer(dev, names=args.only.split(",") if args.only else None)
+    n_elem = sum(m.numel() for _, m in mats)
+    ctx = []
+    for name, x in mats:
+        r, c = x.shape
+        ctx.append({"name": name, "x": x, "shape": (r, c), "s": hq.alloc_stream(r, c, TILE, LAT, BPS, dev),
+                    "ws": hq.alloc_workspace(r, c, TILE, dev),
+                    "y": torch.empty(r, c, dtype=torch.bfloat16, device=dev)})
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def encode(m):
+        hq.hq_encode(m["x"], TILE, LAT, BPS, SEED, m["s"], m["ws"], status)
+
+    def decode(m):
+        r, c = m["shape"]
+        hq.hq_decode(m["s"], r, c, TILE, LAT, BPS, SEED, m["y"], status)
+
+    def step(ev=None):
+        for i, m in enumerate(ctx):
+            if ev: ev["enc"][i][0].record(stream)
+            encode(m)
+            if ev: ev["enc"][i][1].record(stream)
+        for i, m in enumerate(ctx):
+            if ev: ev["dec"][i][0].record(stream)
+            decode(m)
+            if ev: ev["dec"][i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    comp_bytes = [m["s"].nbytes() for m in ctx]
+    payload_words = sum(m["s"].words() for m in ctx)
+
+    def E():
+        return torch.cuda.Event(enable_timing=True)
+
+    evs = [{"enc": [(E(), E()) for _ in ctx], "dec": [(E(), E()) for _ in ctx]} for _ in range(args.steps)]
+    clocks = Clocks(str(local))
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = E(), E()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local)
+
+    enc_ms = [sum(e[i][0].elapsed_time(e[i][1]) for e in (ev["enc"] for ev in evs)) / args.steps
+              for i in range(len(ctx))]
+    dec_ms = [sum(e[i][0].elapsed_time(e[i][1]) for e in (ev["dec"] for ev in evs)) / args.steps
+              for i in range(len(ctx))]
+    enc_bytes = [2 * m["x"].numel() + cb for m, cb in zip(ctx, comp_bytes)]
+    dec_bytes = enc_bytes
+    peak, peak_kind = peaks()
+    enc_gbs = sum(enc_bytes) / sum(enc_ms) / 1e6
+    dec_gbs = sum(dec_bytes) / sum(dec_ms) / 1e6
+    dominant = "encode" if sum(enc_ms) >= sum(dec_ms) else "decode"
+    dom_gbs = enc_gbs if dominant == "encode" else dec_gbs
+    kfile = "hq_encode.cu" if dominant == "encode" else "hq_decode.cu"
+    tr = traffic_record(kfile)
+    value = world * 4 * n_elem / (ms * 1e-3) / 1e9
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "llama3.1-8b-layer: 7 bf16 matrices (q,k,v,o 4096/1024x4096, gate/up 14336x4096, "
+                               "down 4096x14336), E8 4 bps tile 256, encode + decode",
+                   "elements_per_rank": n_elem, "tile": TILE, "lattice": LAT, "bps": BPS,
+                   "l2": "no flush: each step streams 436 MB in + 436 MB out per rank (> 126 MB L2)",
+                   "parallelism": f"replicas x{world} (independent layers, no data-path collective)"},
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(dom_gbs, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                     "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "traffic_launch": tr["launch"] if tr else None,
+                     "alg_bytes_launch": tr["alg_bytes"] if tr else None},
+        "ops": {"encode": {"ms_per_step": round(sum(enc_ms), 4), "alg_gbs": round(enc_gbs, 1),
+                           "bf16_gbs": round(2 * n_elem / sum(enc_ms) / 1e6, 1), "frac": round(enc_gbs / peak, 4)},
+                "decode": {"ms_per_step": round(sum(dec_ms), 4), "alg_gbs": round(dec_gbs, 1),
+                           "bf16_gbs": round(2 * n_elem / sum(dec_ms) / 1e6, 1), "frac": round(dec_gbs / peak, 4)},
+                "bits_per_weight_payload": round(32 * payload_words / n_elem, 4),
+                "bits_per_weight_total": round(8 * sum(comp_bytes) / n_elem, 4),
+                "per_matrix_ms": {m["name"]: [round(a, 4), round(b, 4)] for m, a, b in zip(ctx, enc_ms, dec_ms)}},
+        "gpu_launches": 2 * len(ctx) * args.steps,
+        "clocks": clk,
+    }
+
+    if not args.no_extras:
+        out["e2e"] = e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier)
+        if rank == 0:
+            out["paths"] = {"gemv": gemv_leg(dev, peak), "kv": kv_leg(dev, peak)}
+            out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier):
+    """Same step through the C ABI from pinned host memory: H2D of the seven
+    inputs, encode, decode, D2H of the seven decoded matrices, all timed."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq
+
+    host_in = [m["x"].cpu().pin_memory() for m in ctx]
+    host_out = [torch.empty(m["shape"], dtype=torch.bfloat16).pin_memory() for m in ctx]
+    dev_in = [torch.empty_like(m["x"]) for m in ctx]
+
+    def step():
+        for m, hi, di in zip(ctx, host_in, dev_in):
+            di.copy_(hi, non_blocking=True)
+            hq.hq_encode(di, TILE, LAT, BPS, SEED, m["s"], m["ws"], status)
+        for m, ho in zip(ctx, host_out):
+            r, c = m["shape"]
+            hq.hq_decode(m["s"], r, c, TILE, LAT, BPS, SEED, m["y"], status)
+            ho.copy_(m["y"], non_blocking=True)
+
+    steps = max(3, min(args.steps, 5))
+    step()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps)
+    nbytes = 2 * n_elem
+    return {"value": round(world * 4 * n_elem / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def time_launches(fn, flush, reps=20):
+    import torch
+    ts = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def gemv_leg(dev, peak):
+    """Batch-1 decode-GEMV on 14336x4096 and 4096x14336 E8 4-bps streams vs the
+    bf16 GEMV (cuBLAS) on the uncompressed matrices; L2 flushed before each."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    w1, w2, x1, x2 = workloads.gemv_case(dev)
+    flushbuf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, w, x in (("14336x4096", w1, x1), ("4096x14336", w2, x2)):
+        r, c = w.shape
+        s = hq.alloc_stream(r, c, TILE, LAT, BPS, dev)
+        ws = hq.alloc_workspace(r, c, TILE, dev)
+        hq.hq_encode(w, TILE, LAT, BPS, SEED, s, ws)
+        y = torch.empty(r, dtype=torch.float32, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            hq.hq_decode_gemv(s, r, c, TILE, LAT, BPS, SEED, x, y, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        ms = time_launches(lambda: hq.hq_decode_gemv(s, r, c, TILE, LAT, BPS, SEED, x, y, st),
+                           lambda: flush_l2(flushbuf))
+        xm = x.view(-1, 1)
+        ms_bf16 = time_launches(lambda: torch.matmul(w, xm), lambda: flush_l2(flushbuf))
+        nb = s.nbytes() + 2 * c + 4 * r
+        res[name] = {"us": round(ms * 1e3, 2), "alg_gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 4),
+                     "compressed_bytes": s.nbytes(), "bf16_gemv_us": round(ms_bf16 * 1e3, 2),
+                     "speedup_vs_bf16": round(ms_bf16 / ms, 3)}
+        del s, ws
+    return res
+
+
+def kv_leg(dev, peak):
+    """KV cache, one layer: K and V (8 x 32768 x 128 bf16) encoded and decoded
+    with subtractive dither, tile 128, E8 and D4 at 4 bps."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    k, v = workloads.kv_layer(dev)
+    res = {}
+    for lat in ("E8", "D4"):
+        ctx = []
+        for x in (k, v):
+            r, c = x.shape
+            ctx.append((x, hq.alloc_stream(r, c, 128, lat, 4.0, dev), hq.alloc_workspace(r, c, 128, dev),
+                        torch.empty_like(x)))
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def enc():
+            for x, s, ws, _ in ctx:
+                hq.hq_kv_encode(x, 128, lat, 4.0, SEED, s, ws, st)
+
+        def dec():
+            for x, s, _, y in ctx:
+                hq.hq_kv_decode(s, x.shape[0], 128, 128, lat, 4.0, SEED, y, st)
+
+        for _ in range(3):
+            enc(); dec()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        n = 2 * k.numel()
+        cb = sum(s.nbytes() for _, s, _, _ in ctx)
+        te = time_launches(enc, lambda: None, reps=10)
+        td = time_launches(dec, lambda: None, reps=10)
+        res[f"{lat}_4bps"] = {"encode_alg_gbs": round((2 * n + cb) / te / 1e6, 1),
+                              "decode_alg_gbs": round((2 * n + cb) / td / 1e6, 1),
+                              "encode_frac": round((2 * n + cb) / te / 1e6 / peak, 4),
+                              "decode_frac": round((2 * n + cb) / td / 1e6 / peak, 4),
+                              "bits_per_value_total": round(8 * cb / n, 4)}
+    return res
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
