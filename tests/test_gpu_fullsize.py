@@ -1,0 +1,129 @@
+"""Parity at the workloads' full sizes, in the launch configuration the
+benchmark times (needs a B200).
+
+The GPU encodes whole matrices; the oracle re-encodes sampled tiles one by
+one (tile words, scale and Rice parameter bit-exact; word count equal to the
+offset difference), offsets are checked for the invariants that hold at any
+size (start at 0, strictly increasing, end inside the capacity), and sampled
+decoded tiles are compared with the oracle's binary64 decode of its own
+words.  Decode-GEMV rows are compared with the oracle's GEMV of the same rows
+encoded by the oracle.
+"""
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from kv_quantization_tile_b200 import hq, workloads
+from gpu_util import DEV, gemv_tolerance, host_input
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_tiles(ntiles, m, seed, tile):
+    rng = np.random.default_rng(seed)
+    T = 8 if tile >= 256 else (16 if tile == 128 else 32)
+    fixed = {0, 1, T - 1, T, T + 1, ntiles - 2, ntiles - 1, ntiles // 2}
+    return sorted({int(t) for t in rng.choice(ntiles, size=min(m, ntiles), replace=False)} | fixed)
+
+
+def tile_input(x: torch.Tensor, tile: int, t: int) -> np.ndarray:
+    cols = x.shape[1]
+    r, j = divmod(t, cols // tile)
+    seg = x[r, j * tile:(j + 1) * tile]
+    return (host_input(seg.reshape(1, -1))[0].astype(np.uint32) << 16).view(np.float32)
+
+
+def check_matrix(x, tile, lat, bps, seed, dither, m=64, decode=True):
+    rows, cols = x.shape
+    ntiles = rows * (cols // tile)
+    s = hq.alloc_stream(rows, cols, tile, lat, bps, DEV)
+    ws = hq.alloc_workspace(rows, cols, tile, DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    (hq.hq_kv_encode if dither else hq.hq_encode)(x, tile, lat, bps, seed, s, ws, st)
+    off = s.tile_off.to(torch.int64) & 0xFFFFFFFF
+    d = off[1:] - off[:-1]
+    assert int(off[0]) == 0
+    assert bool((d > 0).all())
+    assert int(off[-1]) <= s.payload.numel()
+    assert int(st.item()) == 0
+    tiles = sample_tiles(ntiles, m, seed + tile, tile)
+    idx = torch.tensor(tiles, device=DEV)
+    o0 = off[idx].cpu().numpy()
+    o1 = off[idx + 1].cpu().numpy()
+    sc = s.tile_scale[idx].cpu().numpy().view(np.uint16)
+    kk = s.tile_k[idx].cpu().numpy()
+    widx = torch.from_numpy(np.concatenate([np.arange(a, b) for a, b in zip(o0, o1)])).to(DEV)
+    words = s.payload[widx].cpu().numpy().view(np.uint32)
+    if decode:
+        y = torch.empty(rows, cols, dtype=torch.bfloat16, device=DEV)
+        (hq.hq_kv_decode if dither else hq.hq_decode)(s, rows, cols, tile, lat, bps, seed, y, st)
+        assert int(st.item()) == 0
+    pos = 0
+    tpr = cols // tile
+    for t, a, b, sci, ki in zip(tiles, o0, o1, sc, kk):
+        r, j = divmod(t, tpr)
+        ref = oracle.encode_tile(tile_input(x, tile, t), lat, bps, seed, j=j, t=t, dither=dither)
+        nw = int(b - a)
+        assert nw == len(ref["words"]), (t, nw, len(ref["words"]))
+        assert np.array_equal(words[pos:pos + nw], ref["words"]), t
+        assert int(sci) == ref["scale"] and int(ki) == ref["k"], t
+        pos += nw
+        if decode:
+            stt, w64 = oracle.decode_tile(ref["words"], tile, lat, ref["scale"], ref["k"], seed, j, t, dither)
+            assert stt == 0
+            got = y[r, j * tile:(j + 1) * tile].float().cpu().numpy().astype(np.float64)
+            # 1e-5 x the tile's dequantized max-abs, plus one bf16 rounding
+            vh = (w64 * oracle.signs(seed, j, tile)) @ scipy.linalg.hadamard(tile)
+            tol = 1e-5 * np.abs(vh).max() + np.abs(w64) * 2.0**-8 + 1e-30
+            assert np.all(np.abs(got - w64) <= tol), t
+    return s
+
+
+@pytest.mark.parametrize("bps", [3.0, 4.0, 5.0])
+def test_llama_layer(bps):
+    for name, x in workloads.llama_layer(DEV):
+        check_matrix(x, 256, "E8", bps, 42, False, m=48)
+        del x
+    torch.cuda.empty_cache()
+
+
+def test_gemv_workload():
+    w1, w2, x1, x2 = workloads.gemv_case(DEV)
+    for w, xv in ((w1, x1), (w2, x2)):
+        rows, cols = w.shape
+        s = check_matrix(w, 256, "E8", 4.0, 42, False, m=32, decode=False)
+        y = torch.empty(rows, dtype=torch.float32, device=DEV)
+        st = torch.zeros(1, dtype=torch.int32, device=DEV)
+        hq.hq_decode_gemv(s, rows, cols, 256, "E8", 4.0, 42, xv, y, st)
+        assert int(st.item()) == 0
+        yg = y.cpu().numpy()
+        xh = xv.float().cpu().numpy().astype(np.float64)
+        rng = np.random.default_rng(rows)
+        for r in sorted(set(rng.choice(rows, 24, replace=False).tolist()) | {0, rows - 1}):
+            sub = host_input(w[r:r + 1])
+            ref = oracle.encode(sub, 256, "E8", 4.0, 42)
+            yr = oracle.gemv(ref, 1, cols, 256, "E8", 42, xh)[0]
+            tol = gemv_tolerance(ref, 1, cols, 256, "E8", 42, xh)[0]
+            assert abs(yg[r] - yr) <= tol, (r, yg[r], yr, tol)
+
+
+@pytest.mark.parametrize("lat", ["D4", "E8"])
+@pytest.mark.parametrize("bps", [2.0, 3.0, 4.0])
+def test_kv_layer(lat, bps):
+    k, v = workloads.kv_layer(DEV)
+    for x in (k, v):
+        check_matrix(x, 128, lat, bps, 42, True, m=48)
+
+
+def test_dit_stack():
+    """All 72 blocks: E8 4 bps on every matrix, D4/A2/Z 4 bps on the FFN."""
+    for b in range(72):
+        for name, x in workloads.dit_block(b, DEV):
+            check_matrix(x, 256, "E8", 4.0, 42, False, m=3, decode=(b % 12 == 0))
+            if name.startswith("ffn"):
+                for lat in ("D4", "A2", "Z"):
+                    check_matrix(x, 256, lat, 4.0, 42, False, m=2, decode=(b % 24 == 0))
+            del x
+        torch.cuda.empty_cache()
