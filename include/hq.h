@@ -178,6 +178,28 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    float bps, uint64_t seed, const void *x, float *y, void *stream,
                    int32_t *d_status);
 
+/* Encode without a caller-provided workspace.  No counterpart on the pages:
+ * this entry point exists for callers that cannot allocate device memory --
+ * engines that hand out memory only from their own pre-reserved pool and
+ * forbid cudaMalloc after start-up, plug-ins living inside another
+ * framework's allocator, or paths where cudaMalloc may not run because it
+ * can block or synchronise the device.
+ * Same arguments, output and device status as hq_encode, minus the
+ * workspace.  Its scratch is a fixed 512 KiB + 256 B array in each GPU's
+ * global memory, held by every GPU that loads the library until the process
+ * exits; a call may use at most 65536 encode chunks (that is,
+ * hq_encode_workspace_bytes(rows, cols, tile) <= 256 + 8 * 65536), larger
+ * shapes return HQ_ERR_UNSUPPORTED with nothing launched.  The call allocates
+ * nothing.  The first call on a device looks up that device's scratch
+ * address (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  Every call on a device shares the one
+ * array and clears the part it uses on `stream` before its kernel runs, so
+ * calls whose work overlaps on the GPU (different streams, no ordering)
+ * race on it and must be serialised by the caller. */
+int hq_encode_noalloc(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+                      float bps, uint64_t seed, const hq_stream *out, void *stream,
+                      int32_t *d_status);
+
 #ifdef __cplusplus
 }
 #endif

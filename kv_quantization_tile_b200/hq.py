@@ -27,7 +27,7 @@ LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 
 EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
-           "hq_decode", "hq_kv_decode", "hq_decode_gemv"]
+           "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc"]
 
 
 class hq_stream(ctypes.Structure):
@@ -55,6 +55,8 @@ _SIGS = {
                             _vp, _vp]),
     "hq_decode_gemv": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _vp,
                               _vp, _vp]),
+    "hq_encode_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
+                                 _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -219,3 +221,16 @@ def hq_decode_gemv(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, status
     _check(_lib.hq_decode_gemv(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), _ptr(y),
                                _stream_handle(stream), _ptr(status)), "hq_decode_gemv")
     return y
+
+
+def hq_encode_noalloc(x, tile, lattice, bps, seed, out: Stream, status=None, stream=None) -> Stream:
+    """hq_encode without a workspace, for callers that cannot allocate device
+    memory: the library keeps a fixed scratch array on each GPU instead (see
+    include/hq.h for its size limit and the rule that overlapping calls on
+    one GPU must be serialised)."""
+    assert x.is_contiguous() and x.dim() == 2
+    rows, cols = x.shape
+    s = out.struct()
+    _check(_lib.hq_encode_noalloc(_ptr(x), _dtype_code(x), rows, cols, tile, _lat(lattice), bps, seed,
+                                  ctypes.byref(s), _stream_handle(stream), _ptr(status)), "hq_encode_noalloc")
+    return out
