@@ -44,8 +44,8 @@
 #define HQO_CORRUPT 4
 
 /* ------------------------------------------------------------------ */
-/* Counter-based randomness [SM64]: the pages only say "random signs" and
- * "seeded dither"; the generator is this reading's choice. */
+/* Counter-based randomness [SM64]: the pages ask for random signs and a
+ * seeded dither without naming a generator; this one is our choice. */
 
 uint64_t hqo_mix64(uint64_t z)
 {
@@ -62,8 +62,9 @@ uint64_t hqo_hash(uint64_t seed, uint64_t tag, uint64_t a, uint64_t b)
     return hqo_mix64(h ^ b);
 }
 
-/* Random sign of coordinate i of column tile j [V1 (i), V2 "per-tile
- * Walsh-Hadamard rotation"]: bit (i mod 64) of H(seed, 1, j, i / 64), set
+/* Random sign of coordinate i of column tile j (the random signs of the
+ * per-tile Hadamard rotation, [V1] (i), [V2]): bit (i mod 64) of
+ * H(seed, 1, j, i / 64), set
  * bit = -1.  Signs depend on the column tile only, so every row of a
  * column tile shares them. */
 int hqo_sign(uint64_t seed, uint64_t j, uint32_t i)
@@ -109,8 +110,8 @@ void hqo_fwht_f64(double *v, int n)
 }
 
 /* ------------------------------------------------------------------ */
-/* Per-tile scale for the target rate (pages silent beyond "a per-tile
- * scale"; reading): the high-resolution entropy of a lattice quantizer of
+/* Per-tile scale for the target rate (the pages name such a scale but give
+ * no rule; reading): the high-resolution entropy of a lattice quantizer of
  * cell volume V and step D on i.i.d. N(0, s^2) coordinates is
  * log2(sqrt(2 pi e) s) - log2(D V^(1/d)) bits per dimension; setting it to
  * R gives D = s sqrt(2 pi e) 2^-R V^(-1/d).  With the unnormalised
@@ -286,8 +287,8 @@ void hqo_dither(int lattice, uint64_t seed, uint64_t t, uint32_t v, float *delta
 }
 
 /* ------------------------------------------------------------------ */
-/* Lossless strip and zigzag [V1 (iii), V2 "a lossless strip discards the
- * bits lattice membership already fixes"].  Reading: for D-type vectors
+/* Lossless strip and zigzag ([V1] (iii); [V2]: the strip drops what being a
+ * lattice point already determines).  Reading: for D-type vectors
  * (D4, and E8 after its coset bit is removed) the coordinate sum is even,
  * so the parity of the last coordinate is implied: it is stored halved
  * (floor).  A2 keeps the coset bit c and its two integers.  Z strips
@@ -321,7 +322,7 @@ void hqo_unsymbols(int lattice, const uint32_t *u, int32_t *z)
 }
 
 /* ------------------------------------------------------------------ */
-/* Rice code [V1 (iii), V2 "a Rice code carries the remainder"]:
+/* Rice code of what remains after the strip ([V1] (iii), [V2]):
  * code(u, k) = q = floor(u / 2^k) zero bits, one 1 bit, and the k low bits
  * of u; length q + 1 + k.  Per-tile k in [0, 15] minimising the tile's total
  * length, smallest k on ties (brute force over all 16 values). */
