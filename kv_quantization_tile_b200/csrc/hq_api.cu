@@ -71,6 +71,14 @@ uint32_t tile_bound_words(int tile, int lattice, float bps)
     return (uint32_t)((bits + 31) / 32);
 }
 
+// Where the Rice search starts: Delta puts every tile's coordinates at RMS
+// about 1/c, so the optimal k sits near log2(1/c) for all tiles of a call.
+int rice_hint(float c)
+{
+    const double k = std::floor(std::log2(1.0 / (double)c) + 0.5);
+    return k < 0 ? 0 : (k > 15 ? 15 : (int)k);
+}
+
 A2Consts a2_consts() { return A2Consts{ (float)std::sqrt(3.0), (float)(1.0 / std::sqrt(3.0)) }; }
 
 int check_stream(const hq_stream *s, int64_t ntiles, bool need_payload)
@@ -114,7 +122,9 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     const uint64_t need = (uint64_t)ntiles * wmax;
     if (need >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
     if (out->payload_capacity_words < need) return HQ_ERR_CAPACITY;
-    const int64_t nchunks = nchunks_for(ntiles, tile);
+    const int G = encode_tiles_per_group(tile, wmax);
+    const int64_t chunk_tiles = (int64_t)encode_chunk_tiles(tile) * G;
+    const int64_t nchunks = (ntiles + chunk_tiles - 1) / chunk_tiles;
     const uint64_t ws_need = 256 + 8 * (uint64_t)nchunks;
     if (!workspace || !aligned(workspace, 8) || workspace_bytes < ws_need) return HQ_ERR_WORKSPACE;
     if (nchunks >= (int64_t)1 << 31) return HQ_ERR_UNSUPPORTED;
@@ -138,6 +148,10 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     a.status = d_status;
     a.wmax = wmax;
     a.nchunks = (uint32_t)nchunks;
+    a.tiles_per_group = G;
+    const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
+    a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
+    a.k_hint = rice_hint(a.c);
     return launch_encode(tile, lattice, dither, dtype, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -159,6 +173,8 @@ int decode_common(const hq_stream *in, int64_t rows, int64_t cols, int tile, int
     a.dither_key = hash_key(seed, 2);
     a.wmax = tile_bound_words(tile, lattice, bps);
     a.rows = rows;
+    const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
+    a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
     return HQ_OK;
 }
 

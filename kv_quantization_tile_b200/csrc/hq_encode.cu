@@ -1,17 +1,22 @@
 // hq_encode.cu -- single-pass tile encoder for sm_100a.
 //
-// One thread block encodes one chunk of T consecutive tiles (a contiguous
-// span of the row-major input), one tile per group of LPT lanes:
-//   load (128-bit) -> random signs -> pairwise sum of squares -> register +
-//   shuffle Walsh-Hadamard transform -> Delta -> v / Delta [+ dither] ->
-//   nearest lattice point -> strip + zigzag -> per-tile Rice k (convex
-//   descent on the exact code length) -> per-lane code lengths.
+// Persistent blocks take chunks of T consecutive tiles (a contiguous span of
+// the row-major input) from an atomic ticket, so chunks are started in order.
+// Within a block, a group of LPT = N / EPL lanes owns G consecutive tiles of
+// the chunk and, per tile:
+//   loads it (128-bit, the next tile's load in flight), applies the random
+//   signs (per-block table), forms the pairwise sum of squares, runs the
+//   register + shuffle Walsh-Hadamard transform, derives Delta, quantizes
+//   v / Delta [+ dither] to the nearest lattice point, strips and zigzags,
+//   picks the Rice parameter (exact argmin: one pass evaluates k-1, k, k+1
+//   around the rate's typical k and walks further only if needed), and packs
+//   the tile into the group's shared-memory image.
 // The chunk's word count is then published for a decoupled look-back prefix
-// scan over chunks (chunk ids come from an atomic ticket, so every chunk a
-// block waits on belongs to a block that is already running); the tiles'
-// bits are OR-ed into a shared-memory image of the chunk and written out
-// with coalesced stores.  Every wait is bounded: a block that gives up
-// raises HQ_ST_TIMEOUT, publishes its own prefix and writes nothing.
+// scan over chunks; one warp polls 32 predecessor slots at a time.  Every
+// wait is bounded: a block that gives up raises HQ_ST_TIMEOUT, publishes its
+// own prefix so later chunks proceed, and writes nothing.  Finally each group
+// stores its image with coalesced stores and the block writes the chunk's
+// tile headers.
 //
 // Method: [V1] "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline
 // for Large Language and Diffusion Models", abstract (i)-(iv); [V2]
@@ -26,6 +31,8 @@ namespace hq {
 
 namespace {
 
+constexpr int kEncodeWarps = 8;
+
 __device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v)
 {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -38,26 +45,38 @@ __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long lon
     return v;
 }
 
-// Decoupled look-back (thread 0 of a block): publish this chunk's aggregate,
-// sum predecessors' aggregates until an inclusive prefix is found, publish
-// the inclusive prefix.  Returns the exclusive prefix; `timed_out` is set if
-// a predecessor published nothing within the poll limit.
-__device__ uint64_t chunk_lookback(unsigned long long *lb, uint32_t chunk, uint64_t agg,
-                                   bool &timed_out)
+// 1 << s for s in [0, 63], 0 for larger s (PTX clamps the shift amount)
+__device__ __forceinline__ uint32_t shl32(uint32_t v, uint32_t s)
+{
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(s));
+    return r;
+}
+
+// Decoupled look-back run by one whole warp: publish this chunk's aggregate,
+// then sum predecessors 32 at a time until an inclusive prefix is found.
+// Returns the exclusive prefix (same value in every lane).
+__device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, uint64_t agg, int lane,
+                                        bool &timed_out)
 {
     timed_out = false;
     if (chunk == 0) {
-        st_release(&lb[0], kFlagInclusive | agg);
+        if (lane == 0) st_release(&lb[0], kFlagInclusive | agg);
         return 0;
     }
-    st_release(&lb[chunk], kFlagAggregate | agg);
+    if (lane == 0) st_release(&lb[chunk], kFlagAggregate | agg);
     uint64_t excl = 0;
-    int64_t p = (int64_t)chunk - 1;
+    int64_t top = (int64_t)chunk - 1;  // newest predecessor not yet summed
     uint32_t polls = 0;
-    while (p >= 0) {
-        unsigned long long s = ld_acquire(&lb[p]);
+    while (top >= 0) {
+        const int64_t p = top - lane;
+        unsigned long long s = p >= 0 ? ld_acquire(&lb[p]) : (kFlagInclusive | 0ull);
         const uint64_t flag = s & ~kValueMask;
-        if (flag == 0) {
+        const unsigned incl = __ballot_sync(FULL, flag == kFlagInclusive);
+        const unsigned none = __ballot_sync(FULL, flag == 0);
+        // lanes up to and including the nearest inclusive prefix
+        const unsigned upto = incl ? ((incl & -incl) << 1) - 1u : FULL;
+        if (none & upto) {  // a needed predecessor has not published yet
             if (++polls > kSpinLimit) {
                 timed_out = true;
                 break;
@@ -65,32 +84,42 @@ __device__ uint64_t chunk_lookback(unsigned long long *lb, uint32_t chunk, uint6
             __nanosleep(64);
             continue;
         }
-        excl += s & kValueMask;
-        if (flag == kFlagInclusive) break;
-        --p;
+        uint64_t v = ((1u << lane) & upto) ? (s & kValueMask) : 0;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(FULL, v, m);
+        excl += v;
+        if (incl) break;
+        top -= 32;
     }
-    st_release(&lb[chunk], kFlagInclusive | ((excl + agg) & kValueMask));
+    if (lane == 0) st_release(&lb[chunk], kFlagInclusive | ((excl + agg) & kValueMask));
     return excl;
 }
 
 template <int EPL, bool F32IN>
-__device__ __forceinline__ void load_tile_part(const void *x, int64_t e0, float (&w)[EPL])
+struct RawTile {
+    uint4 q[F32IN ? EPL / 4 : EPL / 8];
+};
+
+template <int EPL, bool F32IN>
+__device__ __forceinline__ void load_raw(const void *x, int64_t e0, RawTile<EPL, F32IN> &r)
 {
-    if constexpr (F32IN) {
-        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + e0);
+    const uint4 *p = F32IN ? reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + e0)
+                           : reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) + e0);
 #pragma unroll
-        for (int i = 0; i < EPL / 4; i++) {
-            float4 f = __ldg(p + i);
-            w[4 * i] = f.x; w[4 * i + 1] = f.y; w[4 * i + 2] = f.z; w[4 * i + 3] = f.w;
-        }
-    } else {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) + e0);
+    for (int i = 0; i < (F32IN ? EPL / 4 : EPL / 8); i++) r.q[i] = __ldg(p + i);
+}
+
+template <int EPL, bool F32IN>
+__device__ __forceinline__ void unpack_raw(const RawTile<EPL, F32IN> &r, float (&w)[EPL])
+{
 #pragma unroll
-        for (int i = 0; i < EPL / 8; i++) {
-            uint4 q = __ldg(p + i);
-            const uint32_t qq[4] = { q.x, q.y, q.z, q.w };
+    for (int i = 0; i < (F32IN ? EPL / 4 : EPL / 8); i++) {
+        const uint32_t qq[4] = { r.q[i].x, r.q[i].y, r.q[i].z, r.q[i].w };
 #pragma unroll
-            for (int h = 0; h < 4; h++) {
+        for (int h = 0; h < 4; h++) {
+            if constexpr (F32IN) {
+                w[4 * i + h] = __uint_as_float(qq[h]);
+            } else {
                 w[8 * i + 2 * h] = __uint_as_float(qq[h] << 16);
                 w[8 * i + 2 * h + 1] = __uint_as_float(qq[h] & 0xffff0000u);
             }
@@ -100,218 +129,318 @@ __device__ __forceinline__ void load_tile_part(const void *x, int64_t e0, float 
 
 }  // namespace
 
-template <int N, int D, int EPL, bool DITHER, bool F32IN, int NWARPS>
-__global__ void __launch_bounds__(NWARPS * 32) encode_kernel(const EncodeArgs a)
+template <int N, int D, int EPL, bool DITHER, bool F32IN>
+__global__ void __launch_bounds__(kEncodeWarps * 32) encode_kernel(const EncodeArgs a)
 {
-    constexpr int LPT = N / EPL, TPW = 32 / LPT, T = NWARPS * TPW;
+    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kEncodeWarps * TPW;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;  // coset bits per tile
     constexpr int VPL = EPL / D;                          // vectors per lane
-    static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0, "layout");
+    constexpr int WPT = N / 64 > 0 ? N / 64 : 1;          // sign words per tile
+    static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
 
-    extern __shared__ uint32_t chunk_buf[];  // T * wmax words
-    __shared__ uint32_t s_tile_words[T];
-    __shared__ uint32_t s_tile_off[T];
-    __shared__ uint32_t s_chunk, s_total;
+    const int G = a.tiles_per_group;
+    const int T = GPB * G;  // tiles per chunk
+    extern __shared__ __align__(16) uint32_t smem[];
+    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);     // a.sign_words
+    uint32_t *stage = smem + 2 * a.sign_words;                                        // GPB * G * wmax
+    uint32_t *tile_w = stage + (size_t)GPB * G * a.wmax;                              // T: word offset in group
+    uint32_t *tile_hdr = tile_w + T;                                                  // T: scale | k << 16
+    uint32_t *grp_off = tile_hdr + T;                                                 // GPB + 1
+    __shared__ uint32_t s_chunk;
     __shared__ unsigned long long s_base;
     __shared__ int s_timeout;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane % LPT;
-    const int tl = warp * TPW + lane / LPT;  // tile within the chunk
+    const int gid = warp * TPW + lane / LPT;
     const unsigned mask = group_mask<LPT>(lane);
+    uint32_t *gstage = stage + (size_t)gid * G * a.wmax;
 
-    if (tid == 0) s_chunk = atomicAdd(a.ticket, 1u);
-    __syncthreads();
-    const uint32_t chunk = s_chunk;
-    const int64_t t = (int64_t)chunk * T + tl;
-    const bool active = t < a.ntiles;
-
-    // ---- load + signs
-    float w[EPL];
-    if (active) {
-        load_tile_part<EPL, F32IN>(a.x, t * N + (int64_t)l * EPL, w);
-    } else {
-#pragma unroll
-        for (int r = 0; r < EPL; r++) w[r] = 0.0f;
+    // per-block table of sign words for every column tile
+    for (int i = tid; i < a.sign_words; i += kEncodeWarps * 32) {
+        const uint64_t j = (uint64_t)(i / WPT), m = (uint64_t)(i % WPT);
+        sign_tab[i] = mix64(mix64(a.sign_key ^ j) ^ m);
     }
-    const uint64_t j = active ? (uint64_t)(t % a.tiles_per_row) : 0;
-    const uint32_t i0 = (uint32_t)l * EPL;
-    const uint32_t sbits = (uint32_t)(mix64(mix64(a.sign_key ^ j) ^ (uint64_t)(i0 >> 6)) >> (i0 & 63));
-    float v[EPL];
-#pragma unroll
-    for (int r = 0; r < EPL; r++) v[r] = __uint_as_float(__float_as_uint(w[r]) ^ (((sbits >> r) & 1u) << 31));
 
-    // ---- scale + rotation
-    const float S = sumsq<EPL, LPT>(w, mask);
-    fwht<EPL, LPT>(v, mask, l);
-    bool nonfinite;
-    const uint32_t sb = tile_scale_bits(S, a.c, nonfinite);
-    if (active && nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
+    for (;;) {
+        if (tid == 0) s_chunk = atomicAdd(a.ticket, 1u);
+        __syncthreads();  // also orders the sign table and the previous chunk's reads
+        const uint32_t chunk = s_chunk;
+        if (chunk >= a.nchunks) break;
+        const int64_t t_first = (int64_t)chunk * T + (int64_t)gid * G;  // this group's first tile
 
-    // ---- nearest point, strip, zigzag
-    uint32_t u[EPL];
-    uint32_t cbits = 0;
+        uint32_t goff = 0;  // words staged by this group so far
+        RawTile<EPL, F32IN> raw;
+        if (t_first < a.ntiles) load_raw<EPL, F32IN>(a.x, t_first * N + (int64_t)l * EPL, raw);
+        for (int gi = 0; gi < G; gi++) {
+            const int64_t t = t_first + gi;
+            const bool active = t < a.ntiles;
+            float w[EPL];
+            if (active) {
+                unpack_raw<EPL, F32IN>(raw, w);
+                if (gi + 1 < G && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
+            } else {
 #pragma unroll
-    for (int r = 0; r < EPL; r++) u[r] = 0;
-    if (sb != 0) {
-        const float inv = __frcp_rn(bf16_bits_to_float(sb));
-        const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
-#pragma unroll
-        for (int q = 0; q < VPL; q++) {
-            float x[D], p[D];
-            int z[D], c;
-#pragma unroll
-            for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
-            if constexpr (DITHER) {
-                float dl[D];
-                dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
-#pragma unroll
-                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+                for (int r = 0; r < EPL; r++) w[r] = 0.0f;
             }
-            nearest<D>(x, c, z, p, a.a2);
-            cbits |= (uint32_t)c << q;
+
+            // ---- signs
+            const uint64_t j = active ? (uint64_t)(t % a.tiles_per_row) : 0;
+            const uint32_t i0 = (uint32_t)l * EPL;
+            uint64_t sw;
+            if (a.sign_words) sw = sign_tab[j * WPT + (i0 >> 6)];
+            else sw = mix64(mix64(a.sign_key ^ j) ^ (uint64_t)(i0 >> 6));
+            const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
+            float v[EPL];
 #pragma unroll
-            for (int m = 0; m < D; m++) {
-                int s = z[m];
-                if constexpr (D == 8 || D == 4) {
-                    if (m == D - 1) s >>= 1;  // floor(z / 2): parity is implied by the even sum
+            for (int r = 0; r < EPL; r++)
+                v[r] = __uint_as_float(__float_as_uint(w[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
+
+            // ---- scale + rotation
+            const float S = sumsq<EPL, LPT>(w, mask);
+            fwht<EPL, LPT>(v, mask, l);
+            bool nonfinite;
+            const uint32_t sb = tile_scale_bits(S, a.c, nonfinite);
+            if (active && nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
+
+            // ---- nearest point, strip, zigzag
+            uint32_t u[EPL];
+            uint32_t cbits = 0;
+#pragma unroll
+            for (int r = 0; r < EPL; r++) u[r] = 0;
+            if (sb != 0) {
+                const float inv = __frcp_rn(bf16_bits_to_float(sb));
+                const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
+#pragma unroll
+                for (int q = 0; q < VPL; q++) {
+                    float x[D], p[D];
+                    int z[D], c;
+#pragma unroll
+                    for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
+                    if constexpr (DITHER) {
+                        float dl[D];
+                        dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
+#pragma unroll
+                        for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+                    }
+                    nearest<D>(x, c, z, p, a.a2);
+                    cbits |= (uint32_t)c << q;
+#pragma unroll
+                    for (int m = 0; m < D; m++) {
+                        int s = z[m];
+                        if constexpr (D == 8 || D == 4) {
+                            if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
+                        }
+                        u[q * D + m] = zigzag(s);
+                    }
                 }
-                u[q * D + m] = zigzag(s);
+            }
+
+            // ---- Rice parameter: smallest k minimising sum(u >> k) + N (1 + k).
+            // One pass gives the sums at k0-1, k0, k0+1 (k0 = the rate's typical k);
+            // the cost is convex in k, so k0 is optimal iff C(k0-1) > C(k0) <= C(k0+1).
+            int k = a.k_hint;
+            uint32_t part = 0;  // this lane's sum(u >> k) at the chosen k
+            {
+                const int km = k > 0 ? k - 1 : 0;
+                uint32_t s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+                for (int r = 0; r < EPL; r++) {
+                    const uint32_t aa = u[r] >> km;
+                    s0 += aa;
+                    s1 += aa >> 1;
+                    s2 += aa >> 2;
+                }
+                const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
+                               S2 = group_sum<LPT>(mask, s2);
+                // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
+                // sum(k) - sum(k + 1) > N
+                bool up = false, down = false;
+                if (k == 0) {
+                    if (S0 - S1 <= (uint32_t)N) {
+                        part = s0;                       // C(1) >= C(0)
+                    } else if (S1 - S2 <= (uint32_t)N) {
+                        k = 1;                           // C(1) < C(0), C(2) >= C(1)
+                        part = s1;
+                    } else {
+                        k = 2;
+                        part = s2;
+                        up = true;
+                    }
+                } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
+                    k = km;
+                    part = s0;
+                    down = true;
+                } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
+                    k = k + 1;
+                    part = s2;
+                    up = true;
+                } else {
+                    part = s1;
+                }
+                while (down && k > 0) {
+                    uint32_t sd = 0;
+#pragma unroll
+                    for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
+                    if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
+                    --k;
+                    part = sd;
+                }
+                while (up && k < 15) {
+                    uint32_t su = 0;
+#pragma unroll
+                    for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
+                    if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
+                    ++k;
+                    part = su;
+                }
+            }
+
+            // ---- lengths
+            const uint32_t ul = part + EPL;  // unary bits of this lane
+            const uint32_t uoff = group_excl_scan<LPT>(mask, ul, l);
+            const uint32_t utot = group_sum<LPT>(mask, ul);
+            const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)k + utot;
+            uint32_t W = active ? (bits + 31) >> 5 : 0;
+            const bool overflow = W > a.wmax;  // excluded by the bound; guards the image
+            if (overflow) {
+                W = a.wmax;
+                if (l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
+            }
+
+            // ---- pack into the group's image
+            uint32_t *tbuf = gstage + goff;
+            for (uint32_t i = l; i < W; i += LPT) tbuf[i] = 0u;
+            __syncwarp(mask);
+            if (active && !overflow) {
+                if constexpr (C > 0) or_bits(tbuf, (uint32_t)l * VPL, cbits, VPL);
+                if (k) {
+                    const uint32_t lowmask = (1u << k) - 1u;
+                    const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
+                    if (k <= 4) {  // 8 codes fit one 32-bit word
+#pragma unroll
+                        for (int r0 = 0; r0 < EPL; r0 += 8) {
+                            uint32_t acc = 0;
+#pragma unroll
+                            for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                            or_bits(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
+                        }
+                    } else {
+#pragma unroll
+                        for (int r0 = 0; r0 < EPL; r0 += 4) {
+                            uint64_t acc = 0;
+#pragma unroll
+                            for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                            or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
+                        }
+                    }
+                }
+                const uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
+                if (ul <= 64) {
+                    uint32_t lo = 0, hi = 0, rel = 0;
+#pragma unroll
+                    for (int r = 0; r < EPL; r++) {
+                        rel += u[r] >> k;
+                        lo |= shl32(1u, rel);
+                        hi |= shl32(1u, rel - 32u);
+                        ++rel;
+                    }
+                    or_bits(tbuf, upos, ((uint64_t)hi << 32) | lo, (int)ul);
+                } else {
+                    uint32_t rel = 0;
+#pragma unroll
+                    for (int r = 0; r < EPL; r++) {
+                        rel += u[r] >> k;
+                        const uint32_t pbit = upos + rel;
+                        atomicOr(&tbuf[pbit >> 5], 1u << (pbit & 31));
+                        ++rel;
+                    }
+                }
+            }
+            if (l == 0) {
+                tile_w[gid * G + gi] = goff;
+                tile_hdr[gid * G + gi] = sb | ((uint32_t)k << 16);
+            }
+            goff += W;
+        }
+        if (l == 0) grp_off[gid] = goff;
+        __syncthreads();
+
+        // ---- chunk prefix: group offsets, then the look-back (warp 0)
+        if (warp == 0) {
+            const uint32_t mine = lane < GPB ? grp_off[lane] : 0u;
+            uint32_t incl = mine;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t o = __shfl_up_sync(FULL, incl, d);
+                if (lane >= d) incl += o;
+            }
+            const uint32_t total = __shfl_sync(FULL, incl, 31);
+            bool to;
+            const uint64_t base = chunk_lookback_warp(a.lb, chunk, total, lane, to);
+            if (lane < GPB) grp_off[lane] = incl - mine;
+            if (lane == 0) {
+                grp_off[GPB] = total;
+                s_base = base;
+                s_timeout = to;
+                if (to && a.status) atomicOr(a.status, kStatusTimeout);
             }
         }
-    }
+        __syncthreads();
 
-    // ---- per-tile Rice parameter: smallest k in [0, 15] with
-    //      sum_i ceil(floor(u_i / 2^k) / 2) <= N (the code length is convex in k
-    //      and this is where its forward difference turns non-negative).
-    uint32_t lsum = 0;
-#pragma unroll
-    for (int r = 0; r < EPL; r++) lsum += u[r];
-    const uint32_t tot = group_sum<LPT>(mask, lsum);
-    const uint32_t mean = tot / N;
-    int k = mean ? 31 - __clz(mean) : 0;
-    k = k > 15 ? 15 : k;
-    auto halfsum = [&](int kk) {
-        uint32_t s = 0;
-#pragma unroll
-        for (int r = 0; r < EPL; r++) s += (u[r] + (1u << kk)) >> (kk + 1);
-        return group_sum<LPT>(mask, s);
-    };
-    if (k < 15 && halfsum(k) > (uint32_t)N) {
-        do {
-            ++k;
-        } while (k < 15 && halfsum(k) > (uint32_t)N);
-    } else {
-        while (k > 0 && halfsum(k - 1) <= (uint32_t)N) --k;
-    }
-
-    // ---- lengths
-    uint32_t ul = 0;
-#pragma unroll
-    for (int r = 0; r < EPL; r++) ul += (u[r] >> k) + 1u;
-    const uint32_t uoff = group_excl_scan<LPT>(mask, ul, l);
-    const uint32_t utot = group_sum<LPT>(mask, ul);
-    const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)k + utot;
-    uint32_t W = active ? (bits + 31) >> 5 : 0;
-    const bool overflow = W > a.wmax;  // excluded by the bound; guards the shared image
-    if (overflow) W = a.wmax;
-    if (l == 0) s_tile_words[tl] = W;
-    __syncthreads();
-
-    // ---- chunk prefix (in block) and across chunks (look-back)
-    if (tid == 0) {
-        uint32_t acc = 0;
-        for (int i = 0; i < T; i++) {
-            s_tile_off[i] = acc;
-            acc += s_tile_words[i];
-        }
-        s_total = acc;
-        bool to;
-        s_base = chunk_lookback(a.lb, chunk, acc, to);
-        s_timeout = to;
-        if (to && a.status) atomicOr(a.status, kStatusTimeout);
-    }
-    __syncthreads();
-
-    // ---- pack this tile into the chunk image
-    const uint32_t tb = s_tile_off[tl];
-    uint32_t *tbuf = chunk_buf + tb;
-    for (uint32_t i = l; i < W; i += LPT) tbuf[i] = 0u;
-    __syncwarp();
-    if (active && !overflow) {
-        if constexpr (C > 0) or_bits(tbuf, (uint32_t)l * VPL, cbits, VPL);
-        if (k) {
-            const uint32_t lowmask = (1u << k) - 1u;
-#pragma unroll
-            for (int r0 = 0; r0 < EPL; r0 += 4) {
-                uint64_t val = 0;
-#pragma unroll
-                for (int m = 0; m < 4; m++) val |= (uint64_t)(u[r0 + m] & lowmask) << (m * k);
-                or_bits(tbuf, (uint32_t)C + ((uint32_t)l * EPL + r0) * (uint32_t)k, val, 4 * k);
+        // ---- write the images and the tile headers
+        if (!s_timeout) {
+            const uint64_t base = s_base;
+            const uint32_t total = grp_off[GPB];
+            const bool fits = base + total <= a.cap;
+            if (!fits && tid == 0 && a.status) atomicOr(a.status, kStatusCapacity);
+            const uint64_t gbase = base + grp_off[gid];
+            if (fits) {
+                for (uint32_t i = l; i < goff; i += LPT) a.payload[gbase + i] = gstage[i];
             }
-        }
-        const uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
-        if (ul <= 64) {
-            uint64_t val = 0;
-            uint32_t rel = 0;
-#pragma unroll
-            for (int r = 0; r < EPL; r++) {
-                rel += u[r] >> k;
-                val |= 1ull << rel;
-                ++rel;
+            const int64_t t0 = (int64_t)chunk * T;
+            for (int i = tid; i < T; i += kEncodeWarps * 32) {
+                const int64_t t = t0 + i;
+                if (t < a.ntiles) {
+                    const int g = i / G;
+                    a.off[t] = (uint32_t)(base + grp_off[g] + tile_w[i]);
+                    a.scale[t] = (uint16_t)(tile_hdr[i] & 0xffffu);
+                    a.kk[t] = (uint8_t)(tile_hdr[i] >> 16);
+                }
             }
-            or_bits(tbuf, upos, val, (int)ul);
-        } else {
-            uint32_t rel = 0;
-#pragma unroll
-            for (int r = 0; r < EPL; r++) {
-                rel += u[r] >> k;
-                const uint32_t pbit = upos + rel;
-                atomicOr(&tbuf[pbit >> 5], 1u << (pbit & 31));
-                ++rel;
-            }
+            if (tid == 0 && chunk == a.nchunks - 1) a.off[a.ntiles] = (uint32_t)(base + total);
         }
     }
-    if (overflow && l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
-    __syncthreads();
-
-    // ---- write the chunk and the tile headers
-    const uint64_t base = s_base;
-    const uint32_t total = s_total;
-    if (s_timeout) return;
-    const bool fits = base + total <= a.cap;
-    if (!fits && tid == 0 && a.status) atomicOr(a.status, kStatusCapacity);
-    if (fits) {
-        for (uint32_t i = tid; i < total; i += NWARPS * 32) a.payload[base + i] = chunk_buf[i];
-    }
-    if (active && l == 0) {
-        a.off[t] = (uint32_t)(base + tb);
-        a.scale[t] = (uint16_t)sb;
-        a.kk[t] = (uint8_t)k;
-    }
-    if (tid == 0 && chunk == a.nchunks - 1) a.off[a.ntiles] = (uint32_t)(base + total);
 }
 
 // ------------------------------------------------------------------ launch
 namespace {
 
-constexpr int kEncodeWarps = 8;
+// coordinates per lane: 8 for n = 64, 16 for 128 and 256, 32 above
+template <int N>
+constexpr int epl_for() { return N == 64 ? 8 : (N <= 256 ? 16 : 32); }
 
 template <int N>
-constexpr int epl_for() { return N <= 256 ? 8 : N / 32; }
+constexpr int groups_per_block() { return kEncodeWarps * (32 / (N / epl_for<N>())); }
 
 template <int N, int D, bool DITHER, bool F32IN>
-cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s)
+cudaError_t launch_encode_t(const EncodeArgs &a0, cudaStream_t s)
 {
-    constexpr int EPL = epl_for<N>();
-    constexpr int T = kEncodeWarps * (32 / (N / EPL));
-    const size_t smem = (size_t)T * a.wmax * sizeof(uint32_t);
-    auto kern = encode_kernel<N, D, EPL, DITHER, F32IN, kEncodeWarps>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<a.nchunks, kEncodeWarps * 32, smem, s>>>(a);
+    constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
+    EncodeArgs a = a0;
+    const int T = GPB * a.tiles_per_group;
+    const size_t smem = (size_t)a.sign_words * 8 + (size_t)GPB * a.tiles_per_group * a.wmax * 4 +
+                        (size_t)T * 8 + (GPB + 1) * 4;
+    auto kern = encode_kernel<N, D, EPL, DITHER, F32IN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kEncodeWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int64_t blocks = (int64_t)sm_count() * per_sm;
+    if (blocks > a.nchunks) blocks = a.nchunks;
+    kern<<<(unsigned)blocks, kEncodeWarps * 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -333,13 +462,30 @@ cudaError_t launch_encode_n(int lattice, bool dither, int dtype, const EncodeArg
     }
 }
 
+int groups_for(int tile)
+{
+    switch (tile) {
+    case 64: return groups_per_block<64>();
+    case 128: return groups_per_block<128>();
+    case 256: return groups_per_block<256>();
+    case 512: return groups_per_block<512>();
+    default: return groups_per_block<1024>();
+    }
+}
+
 }  // namespace
 
-int encode_chunk_tiles(int tile)
+// Tiles per group per chunk: as many as keep the staged images within 48 KB
+// (at most 8), so a chunk spans up to 8 x (groups per block) tiles.
+int encode_tiles_per_group(int tile, uint32_t wmax)
 {
-    const int epl = tile <= 256 ? 8 : tile / 32;
-    return kEncodeWarps * (32 / (tile / epl));
+    const int gpb = groups_for(tile);
+    int g = (int)((48u * 1024u) / ((uint32_t)gpb * wmax * 4u));
+    return g < 1 ? 1 : (g > 8 ? 8 : g);
 }
+
+// Smallest chunk for a tile length (one tile per group): sizes the workspace.
+int encode_chunk_tiles(int tile) { return groups_for(tile); }
 
 cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
                           cudaStream_t s)

@@ -35,6 +35,9 @@ struct EncodeArgs {
     int32_t *status;
     uint32_t wmax;        // worst-case words of one tile
     uint32_t nchunks;
+    int tiles_per_group;  // G: consecutive tiles each lane group encodes per chunk
+    int sign_words;       // sign words cached per block (0: hash them per tile)
+    int k_hint;           // the rate's typical Rice parameter (search start)
 };
 
 struct DecodeArgs {
@@ -54,6 +57,7 @@ struct DecodeArgs {
     const void *x;        // gemv input (bf16)
     float *gy;            // gemv output
     int64_t rows;
+    int sign_words;       // sign words cached per block (0: hash them per tile)
 };
 
 // Launch helpers; return a cudaError_t.
@@ -63,8 +67,10 @@ cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const D
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
 
-// Tiles per encode chunk (one thread block) for a tile length.
+// Smallest encode chunk (tiles) for a tile length; sizes the workspace.
 int encode_chunk_tiles(int tile);
+// Tiles per lane group per chunk for a tile length and worst-case tile words.
+int encode_tiles_per_group(int tile, uint32_t wmax);
 int sm_count();
 
 }  // namespace hq

@@ -187,3 +187,29 @@ def test_corrupt_streams_are_contained():
             assert np.all(out[r, j * tile:(j + 1) * tile] == 0), name
             assert np.all(w64[r, j * tile:(j + 1) * tile] == 0), name
         assert_recon_close(out, w64, tile, 2, False)
+
+
+@pytest.mark.parametrize("lat", ["E8", "Z"])
+def test_long_unary_codes(lat):
+    """One rotated coordinate swept from small to huge over Gaussian noise:
+    its Rice code's unary part runs from a few bits to hundreds, covering
+    a lane whose codes fit a 64-bit window with one code of q >= 32 and
+    lanes that span more than 64 bits."""
+    n, seed, rows = 256, 12, 96
+    rng = np.random.default_rng(5)
+    s = oracle.signs(seed, 0, n).astype(np.float64)
+    H = np.array([[(-1) ** bin(r & i).count("1") for i in range(n)] for r in (0, 37, 200)], np.float64)
+    x = np.zeros((rows, n))
+    for r in range(rows):
+        amp = 0.2 * 1.06 ** r
+        x[r] = s * (H[r % 3] * amp + rng.standard_normal(n) * 0.05)
+    xd = torch.from_numpy(x).to(torch.float32).to(DEV)
+    for bps in (2.0, 5.0):
+        g, st = gpu_encode(xd, n, lat, bps, seed)
+        ref = oracle.encode(host_input(xd), n, lat, bps, seed)
+        assert st == 0
+        assert_streams_equal(fetch(g), ref)
+        out, gst = gpu_decode(device_stream(ref), rows, n, n, lat, bps, seed, dtype=torch.float32)
+        w64, _ = oracle.decode(ref, rows, n, n, lat, seed)
+        assert gst == 0
+        assert_recon_close(out, w64, n, seed, False)

@@ -73,7 +73,8 @@ def test_tile_bound_holds_on_adversarial_tiles(lat, tile):
 def test_sizing_functions():
     assert hq.hq_max_payload_words(10, 512, 256, "E8", 4.0) == 20 * hq.hq_tile_bound_words(256, "E8", 4.0)
     assert hq.hq_max_payload_words(0, 512, 256, "E8", 4.0) == 0
-    assert hq.hq_encode_workspace_bytes(100, 256, 256) >= 256 + 8 * math.ceil(100 / 8)
+    small, big = hq.hq_encode_workspace_bytes(100, 256, 256), hq.hq_encode_workspace_bytes(100000, 256, 256)
+    assert small >= 256 + 8 and big > small  # a counter area plus one slot per chunk
     with pytest.raises(hq.HQError) as e:
         hq.hq_max_payload_words(10, 500, 256, "E8", 4.0)
     assert e.value.code == hq.HQ_ERR_ARG
