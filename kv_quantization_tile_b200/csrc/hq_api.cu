@@ -96,7 +96,7 @@ int common_shape(int64_t rows, int64_t cols, int tile, int lattice, float bps, i
     const int64_t tpr = cols / tile;
     if (tpr && rows > (int64_t)(INT64_MAX / 2) / tpr) return HQ_ERR_UNSUPPORTED;
     *ntiles = rows * tpr;
-    if (*ntiles >= (int64_t)1 << 40) return HQ_ERR_UNSUPPORTED;
+    if (*ntiles >= (int64_t)1 << 32 || tpr >= (int64_t)1 << 32) return HQ_ERR_UNSUPPORTED;
     return HQ_OK;
 }
 
@@ -152,6 +152,7 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
     a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
     a.k_hint = rice_hint(a.c);
+    a.tpr_div = make_fastdiv((uint32_t)(cols / tile));
     return launch_encode(tile, lattice, dither, dtype, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -175,6 +176,7 @@ int decode_common(const hq_stream *in, int64_t rows, int64_t cols, int tile, int
     a.rows = rows;
     const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
     a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
+    a.tpr_div = make_fastdiv((uint32_t)(tile ? cols / tile : 1));
     return HQ_OK;
 }
 

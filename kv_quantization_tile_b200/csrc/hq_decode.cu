@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 #pragma unroll
         for (int r = 0; r < EPL; r++) v[r] = pt[r] * scale;
         fwht<EPL, LPT>(v, mask, l);
-        const uint64_t j = (uint64_t)(t % a.tiles_per_row);
+        const uint64_t j = (uint32_t)t - fast_div((uint32_t)t, a.tpr_div) * (uint32_t)a.tiles_per_row;
         const uint32_t sbits = sign_bits<N, EPL>(sign_tab, a.sign_words, a.sign_key, j, l);
 #pragma unroll
         for (int r = 0; r < EPL; r++) v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));

@@ -34,6 +34,30 @@ __host__ __forceinline__ uint64_t hash_key(uint64_t seed, uint64_t tag)
     return mix64(seed + kGamma * (tag + 1));
 }
 
+// ------------------------------------------------------------- division
+// Unsigned 32-bit division by a divisor fixed per call (Granlund & Montgomery,
+// "Division by invariant integers using multiplication", 1994): q = n / d.
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+
+__host__ inline FastDiv make_fastdiv(uint32_t d)
+{
+    FastDiv f{ d, 0, 0, 0 };
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;
+    f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+    f.s1 = l > 0 ? 1 : 0;
+    f.s2 = l > 0 ? l - 1 : 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv &f)
+{
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 // ------------------------------------------------------------- groups
 template <int LPT>
 __device__ __forceinline__ unsigned group_mask(int lane)
@@ -284,6 +308,15 @@ __device__ __forceinline__ void or_bits(uint32_t *buf, uint32_t pos, uint64_t v,
     if (b0) atomicOr(&buf[w], b0);
     if (len + (int)sh > 32 && b1) atomicOr(&buf[w + 1], b1);
     if (len + (int)sh > 64 && b2) atomicOr(&buf[w + 2], b2);
+}
+
+// OR `len` (<= 32) bits of v into a shared-memory bit buffer at bit `pos`
+// (at most two words).
+__device__ __forceinline__ void or_bits32(uint32_t *buf, uint32_t pos, uint32_t v, int len)
+{
+    const uint32_t w = pos >> 5, sh = pos & 31;
+    atomicOr(&buf[w], v << sh);
+    if (sh && (int)sh + len > 32) atomicOr(&buf[w + 1], v >> (32 - sh));
 }
 
 // `len` (<= 32) bits at bit `pos` of a word buffer (buf[pos/32 + 1] must be

@@ -45,6 +45,20 @@ __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long lon
     return v;
 }
 
+// Named barriers between the compute warps and the store warp (0 is
+// __syncthreads): image b ready / image b free again / ticket broadcast.
+constexpr int kBarReady0 = 1, kBarFree0 = 3, kBarTicket = 5;
+
+__device__ __forceinline__ void named_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void named_arrive(int id, int threads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // 1 << s for s in [0, 63], 0 for larger s (PTX clamps the shift amount)
 __device__ __forceinline__ uint32_t shl32(uint32_t v, uint32_t s)
 {
@@ -129,246 +143,279 @@ __device__ __forceinline__ void unpack_raw(const RawTile<EPL, F32IN> &r, float (
 
 }  // namespace
 
+// Resident blocks per SM the compiler must fit registers for: 4 (64 registers)
+// where the tile state fits, fewer for 32 coordinates per lane or dithered E8.
+constexpr int encode_min_blocks(int epl, int d, bool dither) { return epl >= 32 ? 2 : ((dither && d == 8) ? 3 : 4); }
+
 template <int N, int D, int EPL, bool DITHER, bool F32IN>
-__global__ void __launch_bounds__(kEncodeWarps * 32) encode_kernel(const EncodeArgs a)
+__global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, DITHER))
+    encode_kernel(const EncodeArgs a)
 {
-    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kEncodeWarps * TPW;
+    constexpr int NCW = kEncodeWarps - 1;  // compute warps; the last warp scans and stores
+    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = NCW * TPW;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;  // coset bits per tile
     constexpr int VPL = EPL / D;                          // vectors per lane
     constexpr int WPT = N / 64 > 0 ? N / 64 : 1;          // sign words per tile
     static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
+    constexpr int kAll = kEncodeWarps * 32, kCompute = NCW * 32;
 
     const int G = a.tiles_per_group;
     const int T = GPB * G;  // tiles per chunk
     extern __shared__ __align__(16) uint32_t smem[];
-    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);     // a.sign_words
-    uint32_t *stage = smem + 2 * a.sign_words;                                        // GPB * G * wmax
-    uint32_t *tile_w = stage + (size_t)GPB * G * a.wmax;                              // T: word offset in group
-    uint32_t *tile_hdr = tile_w + T;                                                  // T: scale | k << 16
-    uint32_t *grp_off = tile_hdr + T;                                                 // GPB + 1
-    __shared__ uint32_t s_chunk;
-    __shared__ unsigned long long s_base;
-    __shared__ int s_timeout;
+    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);      // a.sign_words
+    const uint32_t gstride = ((uint32_t)G * a.wmax + 3u) & ~3u;                        // words per group image
+    uint32_t *stage0 = smem + 2 * ((a.sign_words + 1) & ~1);                           // 2 x GPB x gstride
+    uint32_t *meta0 = stage0 + (size_t)2 * GPB * gstride;                              // 2 x (2T + GPB)
+    __shared__ uint32_t s_chunk[2];
+    __shared__ uint32_t s_goff[32];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int l = lane % LPT;
-    const int gid = warp * TPW + lane / LPT;
-    const unsigned mask = group_mask<LPT>(lane);
-    uint32_t *gstage = stage + (size_t)gid * G * a.wmax;
 
     // per-block table of sign words for every column tile
-    for (int i = tid; i < a.sign_words; i += kEncodeWarps * 32) {
+    for (int i = tid; i < a.sign_words; i += kAll) {
         const uint64_t j = (uint64_t)(i / WPT), m = (uint64_t)(i % WPT);
         sign_tab[i] = mix64(mix64(a.sign_key ^ j) ^ m);
     }
+    __syncthreads();
 
-    for (;;) {
-        if (tid == 0) s_chunk = atomicAdd(a.ticket, 1u);
-        __syncthreads();  // also orders the sign table and the previous chunk's reads
-        const uint32_t chunk = s_chunk;
-        if (chunk >= a.nchunks) break;
-        const int64_t t_first = (int64_t)chunk * T + (int64_t)gid * G;  // this group's first tile
-
-        uint32_t goff = 0;  // words staged by this group so far
-        RawTile<EPL, F32IN> raw;
-        if (t_first < a.ntiles) load_raw<EPL, F32IN>(a.x, t_first * N + (int64_t)l * EPL, raw);
-        for (int gi = 0; gi < G; gi++) {
-            const int64_t t = t_first + gi;
-            const bool active = t < a.ntiles;
-            float w[EPL];
-            if (active) {
-                unpack_raw<EPL, F32IN>(raw, w);
-                if (gi + 1 < G && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
-            } else {
-#pragma unroll
-                for (int r = 0; r < EPL; r++) w[r] = 0.0f;
+    if (warp < NCW) {
+        // ================= compute warps: encode chunks into alternating images
+        const int l = lane % LPT;
+        const int gid = warp * TPW + lane / LPT;
+        const unsigned mask = group_mask<LPT>(lane);
+        for (int it = 0;; it++) {
+            const int b = it & 1;
+            if (it >= 2) named_sync(kBarFree0 + b, kAll);  // the store warp is done with image b
+            if (tid == 0) s_chunk[b] = atomicAdd(a.ticket, 1u);
+            named_sync(kBarTicket, kCompute);
+            const uint32_t chunk = s_chunk[b];
+            if (chunk >= a.nchunks) {
+                named_arrive(kBarReady0 + b, kAll);  // tells the store warp to finish
+                // consume the store warp's last "image free" so every arrival is matched
+                if (it >= 1) named_sync(kBarFree0 + ((it - 1) & 1), kAll);
+                break;
             }
-
-            // ---- signs
-            const uint64_t j = active ? (uint64_t)(t % a.tiles_per_row) : 0;
-            const uint32_t i0 = (uint32_t)l * EPL;
-            uint64_t sw;
-            if (a.sign_words) sw = sign_tab[j * WPT + (i0 >> 6)];
-            else sw = mix64(mix64(a.sign_key ^ j) ^ (uint64_t)(i0 >> 6));
-            const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
-            float v[EPL];
-#pragma unroll
-            for (int r = 0; r < EPL; r++)
-                v[r] = __uint_as_float(__float_as_uint(w[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
-
-            // ---- scale + rotation
-            const float S = sumsq<EPL, LPT>(w, mask);
-            fwht<EPL, LPT>(v, mask, l);
-            bool nonfinite;
-            const uint32_t sb = tile_scale_bits(S, a.c, nonfinite);
-            if (active && nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
-
-            // ---- nearest point, strip, zigzag
-            uint32_t u[EPL];
-            uint32_t cbits = 0;
-#pragma unroll
-            for (int r = 0; r < EPL; r++) u[r] = 0;
-            if (sb != 0) {
-                const float inv = __frcp_rn(bf16_bits_to_float(sb));
-                const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
-#pragma unroll
-                for (int q = 0; q < VPL; q++) {
-                    float x[D], p[D];
-                    int z[D], c;
-#pragma unroll
-                    for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
-                    if constexpr (DITHER) {
-                        float dl[D];
-                        dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
-#pragma unroll
-                        for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
-                    }
-                    nearest<D>(x, c, z, p, a.a2);
-                    cbits |= (uint32_t)c << q;
-#pragma unroll
-                    for (int m = 0; m < D; m++) {
-                        int s = z[m];
-                        if constexpr (D == 8 || D == 4) {
-                            if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
-                        }
-                        u[q * D + m] = zigzag(s);
-                    }
-                }
-            }
-
-            // ---- Rice parameter: smallest k minimising sum(u >> k) + N (1 + k).
-            // One pass gives the sums at k0-1, k0, k0+1 (k0 = the rate's typical k);
-            // the cost is convex in k, so k0 is optimal iff C(k0-1) > C(k0) <= C(k0+1).
-            int k = a.k_hint;
-            uint32_t part = 0;  // this lane's sum(u >> k) at the chosen k
+            uint32_t *gstage = stage0 + ((size_t)b * GPB + gid) * gstride;
+            uint32_t *tile_w = meta0 + (size_t)b * (2 * T + GPB);  // T: word offset in group
+            uint32_t *tile_hdr = tile_w + T;                         // T: scale | k << 16
+            uint32_t *grp_w = tile_hdr + T;                          // GPB: words per group
+            const int64_t t_first = (int64_t)chunk * T + (int64_t)gid * G;  // this group's first tile
+            const uint32_t tpr = (uint32_t)a.tiles_per_row;
+            uint32_t jj = 0;  // column tile of the current tile (consecutive tiles: j + 1 mod tpr)
+            if (t_first < a.ntiles) jj = (uint32_t)t_first - fast_div((uint32_t)t_first, a.tpr_div) * tpr;
             {
-                const int km = k > 0 ? k - 1 : 0;
-                uint32_t s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-                for (int r = 0; r < EPL; r++) {
-                    const uint32_t aa = u[r] >> km;
-                    s0 += aa;
-                    s1 += aa >> 1;
-                    s2 += aa >> 2;
+                uint4 *zs = reinterpret_cast<uint4 *>(gstage);
+                for (uint32_t i = l; i < gstride / 4; i += LPT) zs[i] = make_uint4(0u, 0u, 0u, 0u);
+                __syncwarp(mask);
+            }
+
+            uint32_t goff = 0;  // words staged by this group so far
+            RawTile<EPL, F32IN> raw;
+            if (t_first < a.ntiles) load_raw<EPL, F32IN>(a.x, t_first * N + (int64_t)l * EPL, raw);
+            for (int gi = 0; gi < G; gi++) {
+                const int64_t t = t_first + gi;
+                const bool active = t < a.ntiles;
+                // ---- signs (v = s . w)
+                const uint64_t j = jj;
+                const uint32_t i0 = (uint32_t)l * EPL;
+                uint64_t sw;
+                if (a.sign_words) sw = sign_tab[j * WPT + (i0 >> 6)];
+                else sw = mix64(mix64(a.sign_key ^ j) ^ (uint64_t)(i0 >> 6));
+                const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
+                float v[EPL];
+                if (active) {
+                    unpack_raw<EPL, F32IN>(raw, v);
+    #pragma unroll
+                    for (int r = 0; r < EPL; r++)
+                        v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
+                    if (gi + 1 < G && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
+                } else {
+    #pragma unroll
+                    for (int r = 0; r < EPL; r++) v[r] = 0.0f;
                 }
-                const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
-                               S2 = group_sum<LPT>(mask, s2);
-                // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
-                // sum(k) - sum(k + 1) > N
-                bool up = false, down = false;
-                if (k == 0) {
-                    if (S0 - S1 <= (uint32_t)N) {
-                        part = s0;                       // C(1) >= C(0)
-                    } else if (S1 - S2 <= (uint32_t)N) {
-                        k = 1;                           // C(1) < C(0), C(2) >= C(1)
-                        part = s1;
-                    } else {
-                        k = 2;
+                if (++jj == tpr) jj = 0;
+
+                // ---- scale (sum of squares is sign-blind) + rotation
+                const float S = sumsq<EPL, LPT>(v, mask);
+                fwht<EPL, LPT>(v, mask, l);
+                bool nonfinite;
+                const uint32_t sb = tile_scale_bits(S, a.c, nonfinite);
+                if (active && nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
+
+                // ---- nearest point, strip, zigzag
+                uint32_t u[EPL];
+                uint32_t cbits = 0;
+    #pragma unroll
+                for (int r = 0; r < EPL; r++) u[r] = 0;
+                if (sb != 0) {
+                    const float inv = __frcp_rn(bf16_bits_to_float(sb));
+                    const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
+    #pragma unroll
+                    for (int q = 0; q < VPL; q++) {
+                        float x[D], p[D];
+                        int z[D], c;
+    #pragma unroll
+                        for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
+                        if constexpr (DITHER) {
+                            float dl[D];
+                            dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
+    #pragma unroll
+                            for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+                        }
+                        nearest<D>(x, c, z, p, a.a2);
+                        cbits |= (uint32_t)c << q;
+    #pragma unroll
+                        for (int m = 0; m < D; m++) {
+                            int s = z[m];
+                            if constexpr (D == 8 || D == 4) {
+                                if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
+                            }
+                            u[q * D + m] = zigzag(s);
+                        }
+                    }
+                }
+
+                // ---- Rice parameter: smallest k minimising sum(u >> k) + N (1 + k).
+                // One pass gives the sums at k0-1, k0, k0+1 (k0 = the rate's typical k);
+                // the cost is convex in k, so k0 is optimal iff C(k0-1) > C(k0) <= C(k0+1).
+                int k = a.k_hint;
+                uint32_t part = 0;  // this lane's sum(u >> k) at the chosen k
+                {
+                    const int km = k > 0 ? k - 1 : 0;
+                    uint32_t s0 = 0, s1 = 0, s2 = 0;
+    #pragma unroll
+                    for (int r = 0; r < EPL; r++) {
+                        const uint32_t aa = u[r] >> km;
+                        s0 += aa;
+                        s1 += aa >> 1;
+                        s2 += aa >> 2;
+                    }
+                    const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
+                                   S2 = group_sum<LPT>(mask, s2);
+                    // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
+                    // sum(k) - sum(k + 1) > N
+                    bool up = false, down = false;
+                    if (k == 0) {
+                        if (S0 - S1 <= (uint32_t)N) {
+                            part = s0;                       // C(1) >= C(0)
+                        } else if (S1 - S2 <= (uint32_t)N) {
+                            k = 1;                           // C(1) < C(0), C(2) >= C(1)
+                            part = s1;
+                        } else {
+                            k = 2;
+                            part = s2;
+                            up = true;
+                        }
+                    } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
+                        k = km;
+                        part = s0;
+                        down = true;
+                    } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
+                        k = k + 1;
                         part = s2;
                         up = true;
-                    }
-                } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
-                    k = km;
-                    part = s0;
-                    down = true;
-                } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
-                    k = k + 1;
-                    part = s2;
-                    up = true;
-                } else {
-                    part = s1;
-                }
-                while (down && k > 0) {
-                    uint32_t sd = 0;
-#pragma unroll
-                    for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
-                    if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
-                    --k;
-                    part = sd;
-                }
-                while (up && k < 15) {
-                    uint32_t su = 0;
-#pragma unroll
-                    for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
-                    if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
-                    ++k;
-                    part = su;
-                }
-            }
-
-            // ---- lengths
-            const uint32_t ul = part + EPL;  // unary bits of this lane
-            const uint32_t uoff = group_excl_scan<LPT>(mask, ul, l);
-            const uint32_t utot = group_sum<LPT>(mask, ul);
-            const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)k + utot;
-            uint32_t W = active ? (bits + 31) >> 5 : 0;
-            const bool overflow = W > a.wmax;  // excluded by the bound; guards the image
-            if (overflow) {
-                W = a.wmax;
-                if (l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
-            }
-
-            // ---- pack into the group's image
-            uint32_t *tbuf = gstage + goff;
-            for (uint32_t i = l; i < W; i += LPT) tbuf[i] = 0u;
-            __syncwarp(mask);
-            if (active && !overflow) {
-                if constexpr (C > 0) or_bits(tbuf, (uint32_t)l * VPL, cbits, VPL);
-                if (k) {
-                    const uint32_t lowmask = (1u << k) - 1u;
-                    const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
-                    if (k <= 4) {  // 8 codes fit one 32-bit word
-#pragma unroll
-                        for (int r0 = 0; r0 < EPL; r0 += 8) {
-                            uint32_t acc = 0;
-#pragma unroll
-                            for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                            or_bits(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
-                        }
                     } else {
-#pragma unroll
-                        for (int r0 = 0; r0 < EPL; r0 += 4) {
-                            uint64_t acc = 0;
-#pragma unroll
-                            for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                            or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
+                        part = s1;
+                    }
+                    while (down && k > 0) {
+                        uint32_t sd = 0;
+    #pragma unroll
+                        for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
+                        if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
+                        --k;
+                        part = sd;
+                    }
+                    while (up && k < 15) {
+                        uint32_t su = 0;
+    #pragma unroll
+                        for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
+                        if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
+                        ++k;
+                        part = su;
+                    }
+                }
+
+                // ---- lengths
+                const uint32_t ul = part + EPL;  // unary bits of this lane
+                const uint32_t uoff = group_excl_scan<LPT>(mask, ul, l);
+                const uint32_t utot = group_sum<LPT>(mask, ul);
+                const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)k + utot;
+                uint32_t W = active ? (bits + 31) >> 5 : 0;
+                const bool overflow = W > a.wmax;  // excluded by the bound; guards the image
+                if (overflow) W = a.wmax;
+
+                // ---- pack into the group's image (zeroed at chunk start)
+                uint32_t *tbuf = gstage + goff;
+                if (active && !overflow) {
+                    if constexpr (C > 0) or_bits32(tbuf, (uint32_t)l * VPL, cbits, VPL);
+                    if (k) {
+                        const uint32_t lowmask = (1u << k) - 1u;
+                        const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
+                        if (k <= 4) {  // 8 codes fit one 32-bit word
+    #pragma unroll
+                            for (int r0 = 0; r0 < EPL; r0 += 8) {
+                                uint32_t acc = 0;
+    #pragma unroll
+                                for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                                or_bits32(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
+                            }
+                        } else {
+    #pragma unroll
+                            for (int r0 = 0; r0 < EPL; r0 += 4) {
+                                uint64_t acc = 0;
+    #pragma unroll
+                                for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                                or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
+                            }
                         }
                     }
-                }
-                const uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
-                if (ul <= 64) {
-                    uint32_t lo = 0, hi = 0, rel = 0;
-#pragma unroll
-                    for (int r = 0; r < EPL; r++) {
-                        rel += u[r] >> k;
-                        lo |= shl32(1u, rel);
-                        hi |= shl32(1u, rel - 32u);
-                        ++rel;
+                    // unary parts: eight codes at a time into a 32-bit bitmap
+                    uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
+    #pragma unroll
+                    for (int r0 = 0; r0 < EPL; r0 += 8) {
+                        uint32_t bm = 0, rel = 0;
+    #pragma unroll
+                        for (int m = 0; m < 8; m++) {
+                            const uint32_t pbit = rel + (u[r0 + m] >> k);
+                            bm |= shl32(1u, pbit);
+                            rel = pbit + 1;
+                        }
+                        if (rel <= 32) {
+                            or_bits32(tbuf, upos, bm, (int)rel);
+                        } else {  // a long code: set the terminators one by one
+                            uint32_t pr = upos;
+    #pragma unroll
+                            for (int m = 0; m < 8; m++) {
+                                pr += u[r0 + m] >> k;
+                                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
+                                ++pr;
+                            }
+                        }
+                        upos += rel;
                     }
-                    or_bits(tbuf, upos, ((uint64_t)hi << 32) | lo, (int)ul);
-                } else {
-                    uint32_t rel = 0;
-#pragma unroll
-                    for (int r = 0; r < EPL; r++) {
-                        rel += u[r] >> k;
-                        const uint32_t pbit = upos + rel;
-                        atomicOr(&tbuf[pbit >> 5], 1u << (pbit & 31));
-                        ++rel;
-                    }
                 }
+                if (overflow && l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
+                if (l == 0) {
+                    tile_w[gid * G + gi] = goff;
+                    tile_hdr[gid * G + gi] = sb | ((uint32_t)k << 16);
+                }
+                goff += W;
             }
-            if (l == 0) {
-                tile_w[gid * G + gi] = goff;
-                tile_hdr[gid * G + gi] = sb | ((uint32_t)k << 16);
-            }
-            goff += W;
+            if (l == 0) grp_w[gid] = goff;
+            named_arrive(kBarReady0 + b, kAll);
         }
-        if (l == 0) grp_off[gid] = goff;
-        __syncthreads();
-
-        // ---- chunk prefix: group offsets, then the look-back (warp 0)
-        if (warp == 0) {
-            const uint32_t mine = lane < GPB ? grp_off[lane] : 0u;
+    } else {
+        // ================= store warp: chunk prefix, look-back, coalesced stores
+        for (int it = 0;; it++) {
+            const int b = it & 1;
+            named_sync(kBarReady0 + b, kAll);
+            const uint32_t chunk = s_chunk[b];
+            if (chunk >= a.nchunks) break;
+            const uint32_t *stage = stage0 + (size_t)b * GPB * gstride;
+            const uint32_t *tile_w = meta0 + (size_t)b * (2 * T + GPB);
+            const uint32_t *tile_hdr = tile_w + T;
+            const uint32_t *grp_w = tile_hdr + T;
+            const uint32_t mine = lane < GPB ? grp_w[lane] : 0u;
             uint32_t incl = mine;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
@@ -376,39 +423,37 @@ __global__ void __launch_bounds__(kEncodeWarps * 32) encode_kernel(const EncodeA
                 if (lane >= d) incl += o;
             }
             const uint32_t total = __shfl_sync(FULL, incl, 31);
+            const uint32_t gexcl = incl - mine;  // group `lane`'s word offset in the chunk
             bool to;
             const uint64_t base = chunk_lookback_warp(a.lb, chunk, total, lane, to);
-            if (lane < GPB) grp_off[lane] = incl - mine;
-            if (lane == 0) {
-                grp_off[GPB] = total;
-                s_base = base;
-                s_timeout = to;
-                if (to && a.status) atomicOr(a.status, kStatusTimeout);
-            }
-        }
-        __syncthreads();
-
-        // ---- write the images and the tile headers
-        if (!s_timeout) {
-            const uint64_t base = s_base;
-            const uint32_t total = grp_off[GPB];
-            const bool fits = base + total <= a.cap;
-            if (!fits && tid == 0 && a.status) atomicOr(a.status, kStatusCapacity);
-            const uint64_t gbase = base + grp_off[gid];
-            if (fits) {
-                for (uint32_t i = l; i < goff; i += LPT) a.payload[gbase + i] = gstage[i];
-            }
-            const int64_t t0 = (int64_t)chunk * T;
-            for (int i = tid; i < T; i += kEncodeWarps * 32) {
-                const int64_t t = t0 + i;
-                if (t < a.ntiles) {
-                    const int g = i / G;
-                    a.off[t] = (uint32_t)(base + grp_off[g] + tile_w[i]);
-                    a.scale[t] = (uint16_t)(tile_hdr[i] & 0xffffu);
-                    a.kk[t] = (uint8_t)(tile_hdr[i] >> 16);
+            if (to) {
+                if (lane == 0 && a.status) atomicOr(a.status, kStatusTimeout);
+            } else {
+                const bool fits = base + total <= a.cap;
+                if (!fits && lane == 0 && a.status) atomicOr(a.status, kStatusCapacity);
+                if (fits) {
+                    for (int g = 0; g < GPB; g++) {
+                        const uint32_t go = __shfl_sync(FULL, gexcl, g), gw = __shfl_sync(FULL, mine, g);
+                        const uint32_t *src = stage + (size_t)g * gstride;
+                        uint32_t *dst = a.payload + base + go;
+                        for (uint32_t i = lane; i < gw; i += 32) dst[i] = src[i];
+                    }
                 }
+                if (lane < GPB) s_goff[lane] = gexcl;
+                __syncwarp();
+                const int64_t t0 = (int64_t)chunk * T;
+                for (int i = lane; i < T; i += 32) {
+                    const int64_t t = t0 + i;
+                    if (t < a.ntiles) {
+                        a.off[t] = (uint32_t)(base + s_goff[i / G] + tile_w[i]);
+                        a.scale[t] = (uint16_t)(tile_hdr[i] & 0xffffu);
+                        a.kk[t] = (uint8_t)(tile_hdr[i] >> 16);
+                    }
+                }
+                if (lane == 0 && chunk == a.nchunks - 1) a.off[a.ntiles] = (uint32_t)(base + total);
+                __syncwarp();
             }
-            if (tid == 0 && chunk == a.nchunks - 1) a.off[a.ntiles] = (uint32_t)(base + total);
+            named_arrive(kBarFree0 + b, kAll);
         }
     }
 }
@@ -421,7 +466,7 @@ template <int N>
 constexpr int epl_for() { return N == 64 ? 8 : (N <= 256 ? 16 : 32); }
 
 template <int N>
-constexpr int groups_per_block() { return kEncodeWarps * (32 / (N / epl_for<N>())); }
+constexpr int groups_per_block() { return (kEncodeWarps - 1) * (32 / (N / epl_for<N>())); }
 
 template <int N, int D, bool DITHER, bool F32IN>
 cudaError_t launch_encode_t(const EncodeArgs &a0, cudaStream_t s)
@@ -429,8 +474,9 @@ cudaError_t launch_encode_t(const EncodeArgs &a0, cudaStream_t s)
     constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
     EncodeArgs a = a0;
     const int T = GPB * a.tiles_per_group;
-    const size_t smem = (size_t)a.sign_words * 8 + (size_t)GPB * a.tiles_per_group * a.wmax * 4 +
-                        (size_t)T * 8 + (GPB + 1) * 4;
+    const size_t gstride = ((size_t)a.tiles_per_group * a.wmax + 3) & ~(size_t)3;
+    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + 2 * (size_t)GPB * gstride * 4 +
+                        2 * ((size_t)T * 8 + (size_t)GPB * 4);
     auto kern = encode_kernel<N, D, EPL, DITHER, F32IN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -475,12 +521,12 @@ int groups_for(int tile)
 
 }  // namespace
 
-// Tiles per group per chunk: as many as keep the staged images within 48 KB
-// (at most 8), so a chunk spans up to 8 x (groups per block) tiles.
+// Tiles per group per chunk: as many as keep the two staged images within
+// 48 KB (at most 8), so a chunk spans up to 8 x (groups per block) tiles.
 int encode_tiles_per_group(int tile, uint32_t wmax)
 {
     const int gpb = groups_for(tile);
-    int g = (int)((48u * 1024u) / ((uint32_t)gpb * wmax * 4u));
+    int g = (int)((48u * 1024u) / (2u * (uint32_t)gpb * wmax * 4u));
     return g < 1 ? 1 : (g > 8 ? 8 : g);
 }
 

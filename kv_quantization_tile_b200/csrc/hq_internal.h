@@ -38,6 +38,7 @@ struct EncodeArgs {
     int tiles_per_group;  // G: consecutive tiles each lane group encodes per chunk
     int sign_words;       // sign words cached per block (0: hash them per tile)
     int k_hint;           // the rate's typical Rice parameter (search start)
+    FastDiv tpr_div;      // division by tiles_per_row
 };
 
 struct DecodeArgs {
@@ -58,6 +59,7 @@ struct DecodeArgs {
     float *gy;            // gemv output
     int64_t rows;
     int sign_words;       // sign words cached per block (0: hash them per tile)
+    FastDiv tpr_div;      // division by tiles_per_row
 };
 
 // Launch helpers; return a cudaError_t.
