@@ -178,6 +178,18 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    float bps, uint64_t seed, const void *x, float *y, void *stream,
                    int32_t *d_status);
 
+/* Testing hook for failure detection (no counterpart on the pages): hq_encode
+ * in which the chunk of tiles numbered `stalled_chunk` (in encode-chunk order)
+ * never publishes its word count to the cross-block prefix scan, so the
+ * next chunk's bounded wait runs out.  The call still returns: the waiting
+ * block raises HQ_ST_TIMEOUT after at most 0.5 s, publishes its own prefix
+ * so later chunks proceed, and the stream it leaves is invalid.  The device
+ * stays usable.  Not for production use. */
+int hq_test_encode_stalled(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+                           float bps, uint64_t seed, const hq_stream *out, void *workspace,
+                           uint64_t workspace_bytes, void *stream, int32_t *d_status,
+                           uint32_t stalled_chunk);
+
 /* Encode without a caller-provided workspace.  No counterpart on the pages:
  * this entry point exists for callers that cannot allocate device memory --
  * engines that hand out memory only from their own pre-reserved pool and

@@ -108,7 +108,7 @@ int64_t nchunks_for(int64_t ntiles, int tile)
 
 int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                 uint64_t seed, const hq_stream *out, void *workspace, uint64_t workspace_bytes,
-                void *stream, int32_t *d_status, bool dither)
+                void *stream, int32_t *d_status, bool dither, uint32_t stall_chunk = 0xffffffffu)
 {
     int64_t ntiles = 0;
     int rc = common_shape(rows, cols, tile, lattice, bps, &ntiles);
@@ -153,6 +153,7 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
     a.k_hint = rice_hint(a.c);
     a.tpr_div = make_fastdiv((uint32_t)(cols / tile));
+    a.stall_chunk = stall_chunk;
     return launch_encode(tile, lattice, dither, dtype, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -262,6 +263,14 @@ int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile,
 {
     return encode_impl(x, dtype, rows, cols, tile, lattice, bps, seed, out, workspace, workspace_bytes, stream,
                        d_status, true);
+}
+
+int hq_test_encode_stalled(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                           uint64_t seed, const hq_stream *out, void *workspace, uint64_t workspace_bytes,
+                           void *stream, int32_t *d_status, uint32_t stalled_chunk)
+{
+    return encode_impl(x, dtype, rows, cols, tile, lattice, bps, seed, out, workspace, workspace_bytes, stream,
+                       d_status, false, stalled_chunk);
 }
 
 int hq_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t seed,

@@ -70,18 +70,26 @@ __device__ __forceinline__ uint32_t shl32(uint32_t v, uint32_t s)
 // Decoupled look-back run by one whole warp: publish this chunk's aggregate,
 // then sum predecessors 32 at a time until an inclusive prefix is found.
 // Returns the exclusive prefix (same value in every lane).
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, uint64_t agg, int lane,
-                                        bool &timed_out)
+                                        bool publish, bool &timed_out)
 {
     timed_out = false;
     if (chunk == 0) {
-        if (lane == 0) st_release(&lb[0], kFlagInclusive | agg);
+        if (lane == 0 && publish) st_release(&lb[0], kFlagInclusive | agg);
         return 0;
     }
-    if (lane == 0) st_release(&lb[chunk], kFlagAggregate | agg);
+    if (lane == 0 && publish) st_release(&lb[chunk], kFlagAggregate | agg);
     uint64_t excl = 0;
     int64_t top = (int64_t)chunk - 1;  // newest predecessor not yet summed
     uint32_t polls = 0;
+    const uint64_t t0 = global_ns();
     while (top >= 0) {
         const int64_t p = top - lane;
         unsigned long long s = p >= 0 ? ld_acquire(&lb[p]) : (kFlagInclusive | 0ull);
@@ -91,7 +99,7 @@ __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, 
         // lanes up to and including the nearest inclusive prefix
         const unsigned upto = incl ? ((incl & -incl) << 1) - 1u : FULL;
         if (none & upto) {  // a needed predecessor has not published yet
-            if (++polls > kSpinLimit) {
+            if (++polls > kSpinLimit || global_ns() - t0 > kWaitLimitNs) {
                 timed_out = true;
                 break;
             }
@@ -105,7 +113,7 @@ __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, 
         if (incl) break;
         top -= 32;
     }
-    if (lane == 0) st_release(&lb[chunk], kFlagInclusive | ((excl + agg) & kValueMask));
+    if (lane == 0 && publish) st_release(&lb[chunk], kFlagInclusive | ((excl + agg) & kValueMask));
     return excl;
 }
 
@@ -425,7 +433,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
             const uint32_t total = __shfl_sync(FULL, incl, 31);
             const uint32_t gexcl = incl - mine;  // group `lane`'s word offset in the chunk
             bool to;
-            const uint64_t base = chunk_lookback_warp(a.lb, chunk, total, lane, to);
+            const uint64_t base = chunk_lookback_warp(a.lb, chunk, total, lane, chunk != a.stall_chunk, to);
             if (to) {
                 if (lane == 0 && a.status) atomicOr(a.status, kStatusTimeout);
             } else {

@@ -15,7 +15,8 @@ constexpr int kStatusNonfinite = 1, kStatusCapacity = 2, kStatusCorrupt = 4, kSt
 // prefix), bits 0..61 the word count.
 constexpr uint64_t kFlagAggregate = 1ull << 62, kFlagInclusive = 2ull << 62;
 constexpr uint64_t kValueMask = (1ull << 62) - 1;
-constexpr uint32_t kSpinLimit = 1u << 22;   // polls before a wait gives up
+constexpr uint32_t kSpinLimit = 1u << 24;          // polls before a wait gives up ...
+constexpr uint64_t kWaitLimitNs = 500ull * 1000000;  // ... or 0.5 s of waiting, whichever first
 
 struct EncodeArgs {
     const void *x;
@@ -39,6 +40,7 @@ struct EncodeArgs {
     int sign_words;       // sign words cached per block (0: hash them per tile)
     int k_hint;           // the rate's typical Rice parameter (search start)
     FastDiv tpr_div;      // division by tiles_per_row
+    uint32_t stall_chunk; // test hook: this chunk never publishes its prefix (0xffffffff: none)
 };
 
 struct DecodeArgs {

@@ -27,7 +27,7 @@ LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 
 EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
-           "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc"]
+           "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled"]
 
 
 class hq_stream(ctypes.Structure):
@@ -57,6 +57,8 @@ _SIGS = {
                               _vp, _vp]),
     "hq_encode_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
                                  _vp, _vp]),
+    "hq_test_encode_stalled": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
+                                      _vp, _u64, _vp, _vp, ctypes.c_uint32]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
