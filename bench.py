@@ -24,7 +24,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -39,7 +38,7 @@ TILE, LAT, BPS, SEED = 256, "E8", 4.0, 42
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
@@ -70,52 +69,66 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks
 class Clocks:
-    """nvidia-smi samples (200 ms) of one GPU during the timed region."""
+    """SM clock and clock-event reasons of one GPU, sampled every 10 ms during
+    the timed region through NVML (read-only queries); nvidia-smi if NVML is
+    unavailable."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, index: str):
-        self.index, self.lines, self.proc = index, [], None
+    def __init__(self, device):
+        self.device, self.samples, self.stop_flag, self.thread = device, [], False, None
+        self.max_mhz, self.handle, self.nvml = None, None, None
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+        self.nvml = pynvml
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+
+    def _loop(self):
+        pn = self.nvml
+        get_reasons = getattr(pn, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pn.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag:
+            try:
+                self.samples.append((pn.nvmlDeviceGetClockInfo(self.handle, pn.NVML_CLOCK_SM),
+                                     get_reasons(self.handle)))
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            threading.Thread(target=self._read, daemon=True).start()
+            self._open()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
         except Exception:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.thread = None
 
     def stop(self):
-        if self.proc:
-            time.sleep(0.25)
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = max(mx, float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.thread:
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "samples": 0, "reasons": [], "source": "none"}
+        reasons = set()
+        for _, bits in self.samples:
+            for name, const in self.REASONS.items():
+                mask = getattr(self.nvml, const, None) or getattr(self.nvml, const.replace("Event", "Throttle"), 0)
+                if bits & mask:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(reasons), "source": "nvml, 10 ms"}
 
 
 # ------------------------------------------------------------------ oracle leg
@@ -250,7 +263,7 @@ def run_ours(args):
         return torch.cuda.Event(enable_timing=True)
 
     evs = [{"enc": [(E(), E()) for _ in ctx], "dec": [(E(), E()) for _ in ctx]} for _ in range(args.steps)]
-    clocks = Clocks(str(local))
+    clocks = Clocks(dev)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
