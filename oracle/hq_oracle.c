@@ -189,8 +189,19 @@ uint16_t hqo_tile_scale(float S, float c, int *nonfinite)
  *   E8 : D8 u (D8 + 1/2);    z = y - c/2 (in D8).
  *   A2 : points (a + c/2, (b + c/2) sqrt3);  z = (a, b).
  * Tie rules (reading): rint ties to even; D_n flips the first coordinate of
- * largest |x - rint(x)|, towards x (upwards when x is an integer); E8 keeps
- * the integer coset when the two squared distances are equal; A2 likewise. */
+ * largest |x - rint(x)|, towards x (upwards when x is an integer); A2 keeps
+ * the integer coset when the two squared distances are equal.
+ *
+ * E8 (reading of [CS82]'s two-candidate decoder): with f = rint(x) and
+ * e = x - f, the D8 candidate is f with the first coordinate of largest |e|
+ * moved towards x when sum(f) is odd.  The D8 + 1/2 candidate starts from the
+ * nearest half-integers floor(x) + 1/2 (an integer x goes up): their
+ * distances to x are exactly 1/2 - |e_i|, so when sum(floor(x)) is odd the
+ * first coordinate of smallest |e| moves towards x (up when its fractional
+ * part is at least 1/2).  The squared distances then differ by
+ *   d0 - d1 = sum|e| - 2 + [sum f odd](1 - 2 max|e|) - [sum floor odd] 2 min|e|,
+ * evaluated in binary32 in that order (|e| summed for i = 0..7); d0 - d1 <= 0
+ * keeps the integer coset. */
 
 static void dn_round(const float *x, int d, int32_t *f)
 {
@@ -220,6 +231,42 @@ static float sqdist(const float *x, const float *p, int d)
     return s;
 }
 
+static void e8_nearest(const float *x, int *c, int32_t *z, float *pt)
+{
+    float e[8], ae[8];
+    int32_t f[8], g[8], sf = 0, sg = 0;
+    for (int i = 0; i < 8; i++) {
+        float r = rintf(x[i]);
+        f[i] = (int32_t)r;
+        g[i] = (int32_t)floorf(x[i]);
+        e[i] = x[i] - r;
+        ae[i] = fabsf(e[i]);
+        sf += f[i];
+        sg += g[i];
+    }
+    int bmax = 0, bmin = 0;
+    for (int i = 1; i < 8; i++) {
+        if (ae[i] > ae[bmax]) bmax = i;
+        if (ae[i] < ae[bmin]) bmin = i;
+    }
+    float s = 0.0f;
+    for (int i = 0; i < 8; i++) s = s + ae[i];
+    float dd = s - 2.0f;
+    if (sf & 1) dd = dd + (1.0f - 2.0f * ae[bmax]);
+    if (sg & 1) dd = dd - 2.0f * ae[bmin];
+    if (dd <= 0.0f) {
+        *c = 0;
+        for (int i = 0; i < 8; i++) z[i] = f[i];
+        if (sf & 1) z[bmax] += (e[bmax] >= 0.0f) ? 1 : -1;
+        for (int i = 0; i < 8; i++) pt[i] = (float)z[i];
+    } else {
+        *c = 1;
+        for (int i = 0; i < 8; i++) z[i] = g[i];
+        if (sg & 1) z[bmin] += (x[bmin] - (float)g[bmin] >= 0.5f) ? 1 : -1;
+        for (int i = 0; i < 8; i++) pt[i] = (float)z[i] + 0.5f;
+    }
+}
+
 void hqo_nearest(int lattice, const float *x, int *c, int32_t *z, float *pt)
 {
     *c = 0;
@@ -231,22 +278,7 @@ void hqo_nearest(int lattice, const float *x, int *c, int32_t *z, float *pt)
         dn_round(x, 4, z);
         for (int i = 0; i < 4; i++) pt[i] = (float)z[i];
     } else if (lattice == 8) {
-        int32_t a[8], b[8];
-        float xs[8], pa[8], pb[8];
-        dn_round(x, 8, a);
-        for (int i = 0; i < 8; i++) xs[i] = x[i] - 0.5f;
-        dn_round(xs, 8, b);
-        for (int i = 0; i < 8; i++) {
-            pa[i] = (float)a[i];
-            pb[i] = (float)b[i] + 0.5f;
-        }
-        float d0 = sqdist(x, pa, 8), d1 = sqdist(x, pb, 8);
-        if (d0 <= d1) {
-            for (int i = 0; i < 8; i++) { z[i] = a[i]; pt[i] = pa[i]; }
-        } else {
-            *c = 1;
-            for (int i = 0; i < 8; i++) { z[i] = b[i]; pt[i] = pb[i]; }
-        }
+        e8_nearest(x, c, z, pt);
     } else { /* A2 */
         const float S3 = (float)sqrt(3.0);
         const float T = (float)(1.0 / sqrt(3.0));
