@@ -203,29 +203,51 @@ __device__ __forceinline__ void nearest(const float (&x)[D], int &c, int (&z)[D]
 #pragma unroll
         for (int i = 0; i < 4; i++) z[i] = __float2int_rn(p[i]);
     } else if constexpr (D == 8) {
-        float a[8], b[8], xs[8];
-        dn_round<8>(x, a);
-#pragma unroll
-        for (int i = 0; i < 8; i++) xs[i] = __fsub_rn(x[i], 0.5f);
-        dn_round<8>(xs, b);
-        float d0 = 0.0f, d1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            float t = __fsub_rn(x[i], a[i]);
-            d0 = __fadd_rn(d0, __fmul_rn(t, t));
-        }
+        // Two candidates: D8 from f = rint(x) and D8 + 1/2 from floor(x) + 1/2,
+        // whose coordinates lie exactly 1/2 - |e_i| from x (e = x - f), so
+        //   d0 - d1 = sum|e| - 2 + [sum f odd](1 - 2 max|e|) - [sum floor odd] 2 min|e|
+        // (binary32, in this order); d0 - d1 <= 0 keeps the integer coset.
+        float f[8], g[8], e[8], ae[8];
+        float sf = 0.0f, sg = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            float t = __fsub_rn(x[i], __fadd_rn(b[i], 0.5f));
-            d1 = __fadd_rn(d1, __fmul_rn(t, t));
+            f[i] = rintf(x[i]);
+            g[i] = floorf(x[i]);
+            e[i] = __fsub_rn(x[i], f[i]);
+            ae[i] = fabsf(e[i]);
+            sf = __fadd_rn(sf, f[i]);  // small integers: exact
+            sg = __fadd_rn(sg, g[i]);
         }
-        const bool one = !(d0 <= d1);
+        const bool odd0 = __float2int_rn(sf) & 1, odd1 = __float2int_rn(sg) & 1;
+        float mx = ae[0], mn = ae[0], s = ae[0];
+#pragma unroll
+        for (int i = 1; i < 8; i++) {
+            mx = fmaxf(mx, ae[i]);
+            mn = fminf(mn, ae[i]);
+            s = __fadd_rn(s, ae[i]);
+        }
+        float dd = __fsub_rn(s, 2.0f);
+        if (odd0) dd = __fadd_rn(dd, __fsub_rn(1.0f, 2.0f * mx));
+        if (odd1) dd = __fsub_rn(dd, 2.0f * mn);
+        const bool one = !(dd <= 0.0f);
         c = one ? 1 : 0;
+        // the coordinate the parity fix moves: first index of max|e| (D8) or
+        // min|e| (D8 + 1/2); towards x
+        const bool fix = one ? odd1 : odd0;
+        const float target = one ? mn : mx;
+        int b = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; i--)
+            if (ae[i] == target) b = i;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            float f = one ? b[i] : a[i];
-            z[i] = __float2int_rn(f);
-            p[i] = one ? __fadd_rn(b[i], 0.5f) : a[i];
+            float base = one ? g[i] : f[i];
+            if (fix && i == b) {
+                const bool up = one ? (__fsub_rn(x[i], g[i]) >= 0.5f) : (e[i] >= 0.0f);
+                base = __fadd_rn(base, up ? 1.0f : -1.0f);
+            }
+            z[i] = __float2int_rn(base);
+            p[i] = one ? __fadd_rn(base, 0.5f) : base;
         }
     } else {  // A2: points (a + c/2, (b + c/2) sqrt3)
         float y1 = __fmul_rn(x[1], a2.inv_s3);
