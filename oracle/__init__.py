@@ -372,3 +372,24 @@ def gemv(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, x,
     if st < 0:
         raise MemoryError
     return y[: r1 - r0]
+
+
+def kv_attention(k_stream: dict, v_stream: dict, heads: int, tokens: int, head_dim: int, lattice,
+                 seed_k: int, seed_v: int, q, scale: float, threads: int = 1) -> np.ndarray:
+    """Batch-1 attention over a dithered compressed KV cache, in binary64:
+    K and V (rows = heads * tokens, one vector per row) are decoded with their
+    dither subtracted, then for each head o = softmax(scale K q) V.  The plain
+    definition of the consumer of the cache's inner products (the pages' KV
+    inner products stay unbiased per vector under subtractive dither)."""
+    rows = heads * tokens
+    K, st_k = decode(k_stream, rows, head_dim, head_dim, lattice, seed_k, dither=True, threads=threads)
+    V, st_v = decode(v_stream, rows, head_dim, head_dim, lattice, seed_v, dither=True, threads=threads)
+    if st_k or st_v:
+        raise ValueError("corrupt stream")
+    qa = np.asarray(q, dtype=np.float64).reshape(heads, head_dim)
+    out = np.zeros((heads, head_dim))
+    for h in range(heads):
+        s = scale * (K[h * tokens:(h + 1) * tokens] @ qa[h])
+        p = np.exp(s - s.max())
+        out[h] = (p / p.sum()) @ V[h * tokens:(h + 1) * tokens]
+    return out
