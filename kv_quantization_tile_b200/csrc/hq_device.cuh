@@ -318,6 +318,14 @@ __device__ __forceinline__ uint32_t zigzag(int z) { return ((uint32_t)z << 1) ^ 
 __device__ __forceinline__ int unzigzag(uint32_t u) { return (int)(u >> 1) ^ -(int)(u & 1u); }
 
 // ------------------------------------------------------------- bits
+// v << s with s >= 32 giving 0 (PTX clamps the shift amount)
+__device__ __forceinline__ uint32_t shl32(uint32_t v, uint32_t s)
+{
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(s));
+    return r;
+}
+
 // OR `len` (<= 64) bits of v into a shared-memory bit buffer at bit `pos`.
 // The shifted value spans at most three words.
 __device__ __forceinline__ void or_bits(uint32_t *buf, uint32_t pos, uint64_t v, int len)

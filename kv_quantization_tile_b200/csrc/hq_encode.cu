@@ -59,14 +59,6 @@ __device__ __forceinline__ void named_arrive(int id, int threads)
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// 1 << s for s in [0, 63], 0 for larger s (PTX clamps the shift amount)
-__device__ __forceinline__ uint32_t shl32(uint32_t v, uint32_t s)
-{
-    uint32_t r;
-    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(s));
-    return r;
-}
-
 // Decoupled look-back run by one whole warp: publish this chunk's aggregate,
 // then sum predecessors 32 at a time until an inclusive prefix is found.
 // Returns the exclusive prefix (same value in every lane).
