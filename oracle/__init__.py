@@ -375,10 +375,11 @@ def gemv(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, x,
 
 
 def kv_attention(k_stream: dict, v_stream: dict, heads: int, tokens: int, head_dim: int, lattice,
-                 seed_k: int, seed_v: int, q, scale: float, threads: int = 1) -> np.ndarray:
+                 seed_k: int, seed_v: int, q, scale: float, threads: int = 1, group: int = 1) -> np.ndarray:
     """Batch-1 attention over a dithered compressed KV cache, in binary64:
     K and V (rows = heads * tokens, one vector per row) are decoded with their
-    dither subtracted, then for each head o = softmax(scale K q) V.  The plain
+    dither subtracted, then for query head qh (group query heads per KV head,
+    qh // group its KV head h) o = softmax(scale K_h q) V_h.  The plain
     definition of the consumer of the cache's inner products (the pages' KV
     inner products stay unbiased per vector under subtractive dither)."""
     rows = heads * tokens
@@ -386,10 +387,11 @@ def kv_attention(k_stream: dict, v_stream: dict, heads: int, tokens: int, head_d
     V, st_v = decode(v_stream, rows, head_dim, head_dim, lattice, seed_v, dither=True, threads=threads)
     if st_k or st_v:
         raise ValueError("corrupt stream")
-    qa = np.asarray(q, dtype=np.float64).reshape(heads, head_dim)
-    out = np.zeros((heads, head_dim))
-    for h in range(heads):
-        s = scale * (K[h * tokens:(h + 1) * tokens] @ qa[h])
+    qa = np.asarray(q, dtype=np.float64).reshape(heads * group, head_dim)
+    out = np.zeros((heads * group, head_dim))
+    for qh in range(heads * group):
+        h = qh // group
+        s = scale * (K[h * tokens:(h + 1) * tokens] @ qa[qh])
         p = np.exp(s - s.max())
-        out[h] = (p / p.sum()) @ V[h * tokens:(h + 1) * tokens]
+        out[qh] = (p / p.sum()) @ V[h * tokens:(h + 1) * tokens]
     return out

@@ -498,3 +498,29 @@ def test_kv_attention_matches_exact_attention_at_high_rate():
     # swapping the value cache for the key cache changes the output (no mix-up of streams)
     other = oracle.kv_attention(ks, ks, heads, tokens, d, "E8", 7, 7, q, scale)
     assert np.max(np.abs(other - got)) > 0.05
+
+
+def test_kv_attention_grouped_queries_follow_their_kv_head():
+    """Grouped-query attention: query head qh reads KV head qh // group.  At
+    8 bps each query's output must match exact softmax attention over the raw
+    K, V of its own head, and not that of any other head."""
+    rng = np.random.default_rng(321)
+    heads, tokens, d, group = 3, 40, 64, 3
+    K = (rng.standard_normal((heads * tokens, d)) * np.array([1.0, 3.0, 0.5]).repeat(tokens)[:, None]).astype(np.float32)
+    V = (rng.standard_normal((heads * tokens, d)) + np.arange(heads).repeat(tokens)[:, None]).astype(np.float32)
+    q = rng.standard_normal((heads * group, d))
+    scale = 1 / math.sqrt(d)
+    ks = oracle.encode(K, d, "D4", 8.0, 1, dither=True)
+    vs = oracle.encode(V, d, "D4", 8.0, 2, dither=True)
+    got = oracle.kv_attention(ks, vs, heads, tokens, d, "D4", 1, 2, q, scale, group=group)
+    assert got.shape == (heads * group, d)
+
+    def exact(h, qv):
+        s = scale * (K[h * tokens:(h + 1) * tokens].astype(np.float64) @ qv)
+        p = np.exp(s - s.max())
+        return (p / p.sum()) @ V[h * tokens:(h + 1) * tokens]
+
+    for qh in range(heads * group):
+        errs = [np.max(np.abs(got[qh] - exact(h, q[qh]))) for h in range(heads)]
+        assert errs[qh // group] < 0.02, errs
+        assert all(e > 0.2 for h, e in enumerate(errs) if h != qh // group), errs
