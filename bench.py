@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -317,7 +318,8 @@ def run_ours(args):
     if not args.no_extras:
         out["e2e"] = e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier)
         if rank == 0:
-            out["paths"] = {"gemv": gemv_leg(dev, peak), "kv": kv_leg(dev, peak)}
+            out["paths"] = {"gemv": gemv_leg(dev, peak), "kv": kv_leg(dev, peak),
+                            "kv_attention": attention_leg(dev, peak)}
             out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out))
@@ -451,6 +453,65 @@ def kv_leg(dev, peak):
                               "decode_frac": round((2 * n + cb) / td / 1e6 / peak, 4),
                               "bits_per_value_total": round(8 * cb / n, 4)}
     return res
+
+
+def attention_leg(dev, peak, group=4):
+    """Batch-1 decode attention of one Llama-3.1-8B layer: 32 query heads over
+    the 8 x 32768 x 128 K and V caches (4 query heads per KV head), straight
+    from the E8 4-bps dithered streams, against (a) torch's bf16 SDPA on the
+    uncompressed cache and (b) decoding the streams to bf16 and then SDPA.
+    L2 flushed before each timed launch (the streams fit in L2)."""
+    import torch
+    import torch.nn.functional as F
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    k, v = workloads.kv_layer(dev)
+    heads, tokens, d = workloads.KV_HEADS, workloads.KV_TOKENS, workloads.KV_HEAD_DIM
+    streams = []
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    for x, seed in ((k, SEED), (v, SEED + 1)):
+        s = hq.alloc_stream(heads * tokens, d, d, LAT, BPS, dev)
+        hq.hq_kv_encode(x, d, LAT, BPS, seed, s, hq.alloc_workspace(heads * tokens, d, d, dev), st)
+        streams.append(s)
+    ks, vs = streams
+    g = torch.Generator(device=dev).manual_seed(5000)
+    q = torch.randn(heads * group, d, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(heads * group, d, dtype=torch.float32, device=dev)
+    ws = hq.alloc_attention_workspace(heads, tokens, d, group, dev)
+    scale = 1.0 / math.sqrt(d)
+
+    def ours():
+        hq.hq_kv_attention(ks, vs, heads, tokens, d, LAT, BPS, BPS, SEED, SEED + 1, q, scale, out, ws, group=group,
+                           status=st)
+
+    kb, vb = k.view(1, heads, tokens, d), v.view(1, heads, tokens, d)
+    q4 = q.view(1, heads * group, 1, d)
+
+    def sdpa(kk=kb, vv=vb):
+        return F.scaled_dot_product_attention(q4, kk, vv, scale=scale, enable_gqa=True)
+
+    kd, vd = torch.empty_like(k), torch.empty_like(v)
+
+    def decode_then_sdpa():
+        hq.hq_kv_decode(ks, heads * tokens, d, d, LAT, BPS, SEED, kd, st)
+        hq.hq_kv_decode(vs, heads * tokens, d, d, LAT, BPS, SEED + 1, vd, st)
+        sdpa(kd.view(1, heads, tokens, d), vd.view(1, heads, tokens, d))
+
+    flushbuf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        ours(); sdpa(); decode_then_sdpa()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    t = time_launches(ours, lambda: flush_l2(flushbuf))
+    t_sdpa = time_launches(sdpa, lambda: flush_l2(flushbuf))
+    t_dec = time_launches(decode_then_sdpa, lambda: flush_l2(flushbuf))
+    nb = ks.nbytes() + vs.nbytes() + 2 * q.numel() + 4 * out.numel()
+    return {"config": {"kv_heads": heads, "tokens": tokens, "head_dim": d, "query_heads": heads * group,
+                       "lattice": LAT, "bps": BPS},
+            "us": round(t * 1e3, 2), "alg_gbs": round(nb / t / 1e6, 1), "frac": round(nb / t / 1e6 / peak, 4),
+            "compressed_bytes": nb, "bf16_sdpa_us": round(t_sdpa * 1e3, 2),
+            "decode_then_sdpa_us": round(t_dec * 1e3, 2), "speedup_vs_bf16_sdpa": round(t_sdpa / t, 3)}
 
 
 def main():

@@ -178,6 +178,44 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    float bps, uint64_t seed, const void *x, float *y, void *stream,
                    int32_t *d_status);
 
+/* Bytes of device workspace hq_kv_attention needs: 256-byte-rounded
+ * counters (heads * ceil(group / queries per block) uint32) followed by
+ * heads * group * splits * (head_dim + 2) floats of per-split partial
+ * results.  `splits` depends only on (heads, tokens, group) and the GPU's SM
+ * count, so query this on the device the call will run on.  Host only.
+ * HQ_ERR_ARG for negative sizes, head_dim not 64/128/256, group < 1 or
+ * out == NULL. */
+int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim, int group,
+                                    uint64_t *out);
+
+/* Batch-1 attention over a dithered compressed KV cache ([V2] subtractive
+ * dither keeps each cached inner product unbiased; [V1] (iv) the KV codec
+ * serves attention).  For query head qh = h * group + g (grouped-query
+ * attention: `group` query heads share KV head h):
+ *   out[qh] = sum_t softmax_t(scale <q[qh], k_hat_t>) v_hat_t
+ * with k_hat_t, v_hat_t what hq_kv_decode returns for tile h * tokens + t of
+ * each stream, in fp32, without forming them: q is rotated once with the K
+ * signs, scores come from the K stream's lattice points, and values are
+ * accumulated in the rotated domain with one inverse rotation per query.
+ *   k, v        streams written by hq_kv_encode of a (heads * tokens) x
+ *               head_dim slab, tile = head_dim, with lattice, bps_k / bps_v
+ *               and seed_k / seed_v
+ *   heads       KV heads (<= 65535), tokens >= 0 cached vectors per head
+ *   head_dim    64, 128 or 256
+ *   group       query heads per KV head, >= 1
+ *   q           device bf16 [heads * group][head_dim], 16-byte aligned
+ *   scale       finite softmax scale (typically 1 / sqrt(head_dim))
+ *   out         device fp32 [heads * group][head_dim], 16-byte aligned
+ *   workspace   device, >= hq_kv_attention_workspace_bytes, 16-byte
+ *               aligned; its counters are cleared on `stream` first, so calls
+ *               sharing one workspace must be ordered
+ * tokens == 0 writes zeros.  A non-canonical tile counts as a zero vector and
+ * raises HQ_ST_CORRUPT.  Non-finite q or scores propagate to out. */
+int hq_kv_attention(const hq_stream *k, const hq_stream *v, int64_t heads, int64_t tokens,
+                    int head_dim, int group, int lattice, float bps_k, float bps_v, uint64_t seed_k,
+                    uint64_t seed_v, const void *q, float scale, float *out, void *workspace,
+                    uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
 /* Testing hook for failure detection (no counterpart on the pages): hq_encode
  * in which the chunk of tiles numbered `stalled_chunk` (in encode-chunk order)
  * never publishes its word count to the cross-block prefix scan, so the

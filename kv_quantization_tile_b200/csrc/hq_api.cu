@@ -196,6 +196,26 @@ int decode_impl(const hq_stream *in, int64_t rows, int64_t cols, int tile, int l
     return launch_decode(tile, lattice, dither, dtype, a, (cudaStream_t)stream) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
+bool valid_head_dim(int d) { return d == 64 || d == 128 || d == 256; }
+
+// Workspace of an attention call: counters, then the per-split partials.
+struct AttnWorkspace {
+    int splits, tokens_per_split;
+    uint64_t counter_bytes, total_bytes;
+};
+
+AttnWorkspace attention_workspace(int64_t heads, int64_t tokens, int head_dim, int group)
+{
+    AttnWorkspace w{};
+    attention_splits(heads, tokens, group, &w.splits, &w.tokens_per_split);
+    const int gb = attention_queries_per_block(group);
+    const uint64_t counters = (uint64_t)heads * (uint64_t)((group + gb - 1) / gb);
+    w.counter_bytes = (counters * 4 + 255) / 256 * 256;
+    w.total_bytes = w.counter_bytes + (uint64_t)heads * (uint64_t)group * (uint64_t)w.splits *
+                                          (uint64_t)(head_dim + 2) * 4;
+    return w;
+}
+
 }  // namespace
 
 extern "C" {
@@ -305,6 +325,52 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
     a.gy = y;
     a.status = d_status;
     return launch_gemv(tile, lattice, a, cols, (cudaStream_t)stream) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim, int group, uint64_t *out)
+{
+    if (!out || heads < 0 || tokens < 0 || !valid_head_dim(head_dim) || group < 1) return HQ_ERR_ARG;
+    if (heads > 65535 || tokens >= (int64_t)1 << 32 || group > 65535 * 8) return HQ_ERR_UNSUPPORTED;
+    *out = attention_workspace(heads, tokens, head_dim, group).total_bytes;
+    return HQ_OK;
+}
+
+int hq_kv_attention(const hq_stream *k, const hq_stream *v, int64_t heads, int64_t tokens, int head_dim,
+                    int group, int lattice, float bps_k, float bps_v, uint64_t seed_k, uint64_t seed_v,
+                    const void *q, float scale, float *out, void *workspace, uint64_t workspace_bytes,
+                    void *stream, int32_t *d_status)
+{
+    if (heads < 0 || tokens < 0 || !valid_head_dim(head_dim) || group < 1 || !std::isfinite(scale))
+        return HQ_ERR_ARG;
+    if (heads > 65535 || tokens >= (int64_t)1 << 32 || group > 65535 * 8) return HQ_ERR_UNSUPPORTED;
+    if (heads > 0 && tokens > (int64_t)(((uint64_t)1 << 32) - 1) / heads) return HQ_ERR_UNSUPPORTED;
+    AttnArgs a{};
+    int64_t nk = 0, nv = 0;
+    int rc = decode_common(k, heads * tokens, head_dim, head_dim, lattice, bps_k, seed_k, a.k, &nk);
+    if (rc) return rc;
+    if ((rc = decode_common(v, heads * tokens, head_dim, head_dim, lattice, bps_v, seed_v, a.v, &nv))) return rc;
+    if (heads == 0) return HQ_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!out || !aligned(out, 16)) return HQ_ERR_ARG;
+    if (tokens == 0)
+        return cudaMemsetAsync(out, 0, sizeof(float) * (size_t)(heads * group * head_dim), s) == cudaSuccess
+                   ? HQ_OK : HQ_ERR_CUDA;
+    if (!q || !aligned(q, 16)) return HQ_ERR_ARG;
+    const AttnWorkspace w = attention_workspace(heads, tokens, head_dim, group);
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < w.total_bytes) return HQ_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, w.counter_bytes, s) != cudaSuccess) return HQ_ERR_CUDA;
+    a.q = static_cast<const uint16_t *>(q);
+    a.out = out;
+    a.counter = static_cast<uint32_t *>(workspace);
+    a.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.counter_bytes);
+    a.heads = heads;
+    a.tokens = tokens;
+    a.group = group;
+    a.splits = w.splits;
+    a.tokens_per_split = w.tokens_per_split;
+    a.scale = scale;
+    a.status = d_status;
+    return launch_attention(head_dim, lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
 }  // extern "C"

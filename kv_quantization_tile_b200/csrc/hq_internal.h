@@ -64,12 +64,32 @@ struct DecodeArgs {
     FastDiv tpr_div;      // division by tiles_per_row
 };
 
+// Batch-1 attention over K and V codec streams (one tile per cached vector).
+struct AttnArgs {
+    DecodeArgs k, v;        // rows = heads * tokens, one tile of head_dim per row
+    const uint16_t *q;      // bf16 [heads * group][head_dim]
+    float *out;             // fp32 [heads * group][head_dim]
+    float *part;            // [heads * group][splits][head_dim + 2] partial results
+    uint32_t *counter;      // [heads][query chunks] finished splits, zero at launch
+    int64_t heads, tokens;
+    int group;              // query heads per KV head
+    int splits, tokens_per_split;
+    float scale;
+    int32_t *status;
+};
+
 // Launch helpers; return a cudaError_t.
 cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const DecodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
+cudaError_t launch_attention(int head_dim, int lattice, const AttnArgs &a, cudaStream_t s);
+
+// Query heads one attention block serves (1, 2, 4 or 8), and the token
+// splits of a call (every split non-empty).
+int attention_queries_per_block(int group);
+void attention_splits(int64_t heads, int64_t tokens, int group, int *splits, int *tokens_per_split);
 
 // Smallest encode chunk (tiles) for a tile length; sizes the workspace.
 int encode_chunk_tiles(int tile);

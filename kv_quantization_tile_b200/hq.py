@@ -27,7 +27,8 @@ LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 
 EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
-           "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled"]
+           "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
+           "hq_kv_attention_workspace_bytes", "hq_kv_attention"]
 
 
 class hq_stream(ctypes.Structure):
@@ -59,6 +60,9 @@ _SIGS = {
                                  _vp, _vp]),
     "hq_test_encode_stalled": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
                                       _vp, _u64, _vp, _vp, ctypes.c_uint32]),
+    "hq_kv_attention_workspace_bytes": (_i32, [_i64, _i64, _i32, _i32, ctypes.POINTER(_u64)]),
+    "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
+                               _i32, _f32, _f32, _u64, _u64, _vp, _f32, _vp, _vp, _u64, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -223,6 +227,34 @@ def hq_decode_gemv(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, status
     _check(_lib.hq_decode_gemv(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), _ptr(y),
                                _stream_handle(stream), _ptr(status)), "hq_decode_gemv")
     return y
+
+
+def hq_kv_attention_workspace_bytes(heads: int, tokens: int, head_dim: int, group: int = 1) -> int:
+    out = _u64(0)
+    _check(_lib.hq_kv_attention_workspace_bytes(heads, tokens, head_dim, group, ctypes.byref(out)),
+           "hq_kv_attention_workspace_bytes")
+    return out.value
+
+
+def alloc_attention_workspace(heads: int, tokens: int, head_dim: int, group: int = 1,
+                              device="cuda") -> torch.Tensor:
+    return torch.empty(hq_kv_attention_workspace_bytes(heads, tokens, head_dim, group), dtype=torch.uint8,
+                       device=device)
+
+
+def hq_kv_attention(k: Stream, v: Stream, heads: int, tokens: int, head_dim: int, lattice, bps_k: float,
+                    bps_v: float, seed_k: int, seed_v: int, q, scale: float, out, workspace, group: int = 1,
+                    status=None, stream=None):
+    """Batch-1 attention of q (bf16 [heads * group, head_dim]) over the KV
+    streams written by hq_kv_encode; out is fp32 [heads * group, head_dim]."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.numel() == heads * group * head_dim
+    assert out.dtype == torch.float32 and out.is_contiguous() and out.numel() == heads * group * head_dim
+    ks, vs = k.struct(), v.struct()
+    _check(_lib.hq_kv_attention(ctypes.byref(ks), ctypes.byref(vs), heads, tokens, head_dim, group,
+                                _lat(lattice), bps_k, bps_v, seed_k, seed_v, _ptr(q), scale, _ptr(out),
+                                _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status)),
+           "hq_kv_attention")
+    return out
 
 
 def hq_encode_noalloc(x, tile, lattice, bps, seed, out: Stream, status=None, stream=None) -> Stream:

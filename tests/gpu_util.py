@@ -115,3 +115,73 @@ def gemv_tolerance(ref: dict, rows, cols, tile, lat, seed, x: np.ndarray) -> np.
     B = (vh * xl1[None]).sum(axis=1) / tile
     K = 2 * math.log2(tile) + 16 + cols // tile
     return 2.0**-24 * K * B + 1e-30
+
+
+def attention_tolerance(ks: dict, vs: dict, heads, tokens, d, lat, seed_k, seed_v, q: np.ndarray,
+                        scale: float, group: int = 1) -> np.ndarray:
+    """Per output element, an fp32 error bound of the GPU attention against
+    the binary64 oracle, derived from the kernel's arithmetic (u = 2^-24,
+    g(m) = m u / (1 - m u)):
+      score s_t = scale (Delta_t / n) <y_t - delta_t, H(s_K . q)>, with
+        |ds_t| <= |scale| / n (g(n+2) sum_i |z_ti||q~_i| + g(log2 n) ||q||_1 ||z_t||_1) + 3 u |s_t|
+        (z_t = Delta_t (y_t - delta_t) the rotated vector, q~ its query);
+      softmax weights then carry a relative error of at most
+        eta = max_t |ds_t| + u (2 max_t |s_t - m| + 16)   (exp, shifts, merge),
+        moving a convex combination by <= 2 e/(1-e) max_t |v_hat_ti|, e = expm1(eta);
+      the rotated accumulation sum_t w_t z_t (any order, at most
+        tokens + 48 + log2 n roundings deep), the division by the weight sum
+        and the final transform add (2 g(M) + g(log2 n + 1)) (1/n) sum_i sum_t w_t |z_ti|."""
+    u = 2.0**-24
+
+    def g(m):
+        return m * u / (1 - m * u)
+
+    rows = heads * tokens
+    K, _ = oracle.decode(ks, rows, d, d, lat, seed_k, dither=True, threads=8)
+    V, _ = oracle.decode(vs, rows, d, d, lat, seed_v, dither=True, threads=8)
+    H = scipy.linalg.hadamard(d).astype(np.float64)
+    sk = oracle.signs(seed_k, 0, d).astype(np.float64)
+    sv = oracle.signs(seed_v, 0, d).astype(np.float64)
+    ZK = np.abs((K * sk) @ H)
+    ZV = np.abs((V * sv) @ H)
+    L = math.log2(d)
+    M = tokens + 48 + L
+    qa = np.asarray(q, np.float64).reshape(heads * group, d)
+    tol = np.zeros((heads * group, d))
+    for qh in range(heads * group):
+        h = qh // group
+        sl = slice(h * tokens, (h + 1) * tokens)
+        qv = qa[qh]
+        qt = np.abs(H @ (sk * qv))
+        s = scale * (K[sl] @ qv)
+        ds = abs(scale) / d * (g(d + 2) * (ZK[sl] @ qt) + g(L) * np.abs(qv).sum() * ZK[sl].sum(axis=1)) \
+            + 3 * u * np.abs(s)
+        m = s.max()
+        eta = ds.max() + u * (2 * np.abs(s - m).max() + 16)
+        e = math.expm1(eta)
+        p = np.exp(s - m)
+        w = p / p.sum()
+        err_w = 2 * e / (1 - e) * np.abs(V[sl]).max(axis=0)
+        A = (w @ ZV[sl]).sum() / d
+        tol[qh] = err_w + (2 * g(M) + g(L + 1)) * A * (1 + 2 * e)
+    return tol + 2.0**-100
+
+
+def gpu_attention(ks: hq.Stream, vs: hq.Stream, heads, tokens, d, lat, bps_k, bps_v, seed_k, seed_v,
+                  q: torch.Tensor, scale: float, group: int = 1):
+    """Run hq_kv_attention; returns (out as float64 numpy, device status)."""
+    out = torch.full((heads * group, d), float("nan"), dtype=torch.float32, device=DEV)
+    ws = hq.alloc_attention_workspace(heads, tokens, d, group, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    hq.hq_kv_attention(ks, vs, heads, tokens, d, lat, bps_k, bps_v, seed_k, seed_v, q, scale, out, ws,
+                       group=group, status=status)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64), int(status.item())
+
+
+def assert_attention_close(out: np.ndarray, ref: np.ndarray, tol: np.ndarray):
+    err = np.abs(out - ref)
+    if not np.all(err <= tol):
+        i = np.unravel_index(np.argmax(err / tol), err.shape)
+        raise AssertionError(f"attention off at {i}: {out[i]} vs {ref[i]} (tol {tol[i]}, "
+                             f"{int((err > tol).sum())} elements out)")

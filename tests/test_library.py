@@ -113,3 +113,45 @@ def test_encode_and_decode_reject_bad_arguments_before_any_launch():
     assert lib.hq_decode(ctypes.byref(s), 4, 256, 256, 8, 4.0, 0, 16, 5, None, None) == ARG
     assert lib.hq_decode_gemv(ctypes.byref(s), 4, 1 << 16, 256, 8, 4.0, 0, 16, 16, None, None) == \
         hq.HQ_ERR_UNSUPPORTED
+
+
+def test_kv_attention_sizing_and_validation():
+    for heads, tokens, d, group in [(8, 32768, 128, 4), (1, 40000, 64, 1), (3, 333, 256, 11), (2, 1, 64, 2)]:
+        w = hq.hq_kv_attention_workspace_bytes(heads, tokens, d, group)
+        gb = 1 if group <= 1 else 2 if group <= 2 else 4 if group <= 4 else 8
+        counters = heads * -(-group // gb) * 4
+        cbytes = -(-counters // 256) * 256
+        per_split = heads * group * (d + 2) * 4
+        assert (w - cbytes) % per_split == 0
+        splits = (w - cbytes) // per_split
+        assert -(-tokens // (4096 // gb)) <= splits <= tokens
+    ARG = hq.HQ_ERR_ARG
+    lib = hq.library()
+    out = ctypes.c_uint64(0)
+    assert lib.hq_kv_attention_workspace_bytes(8, 100, 96, 1, ctypes.byref(out)) == ARG
+    assert lib.hq_kv_attention_workspace_bytes(8, 100, 128, 0, ctypes.byref(out)) == ARG
+    assert lib.hq_kv_attention_workspace_bytes(-1, 100, 128, 1, ctypes.byref(out)) == ARG
+    assert lib.hq_kv_attention_workspace_bytes(70000, 100, 128, 1, ctypes.byref(out)) == hq.HQ_ERR_UNSUPPORTED
+    s = hq.hq_stream(16, 1 << 20, 16, 16, 16)
+    S = ctypes.byref(s)
+
+    def call(k=S, v=S, heads=2, tokens=10, d=128, group=1, lat=8, bk=4.0, bv=4.0, q=16, scale=0.1, o=16,
+             ws=16, wsb=1 << 20):
+        return lib.hq_kv_attention(k, v, heads, tokens, d, group, lat, bk, bv, 1, 2, q, scale, o, ws, wsb, None,
+                                   None)
+
+    assert call(k=None) == ARG
+    assert call(v=None) == ARG
+    assert call(d=100) == ARG
+    assert call(group=0) == ARG
+    assert call(lat=3) == ARG
+    assert call(bv=9.0) == ARG
+    assert call(scale=float("inf")) == ARG
+    assert call(q=0) == ARG
+    assert call(q=18) == ARG
+    assert call(o=0) == ARG
+    assert call(o=20) == ARG
+    assert call(ws=0) == hq.HQ_ERR_WORKSPACE
+    assert call(wsb=64) == hq.HQ_ERR_WORKSPACE
+    assert call(heads=70000) == hq.HQ_ERR_UNSUPPORTED
+    assert call(heads=0) == hq.HQ_OK  # nothing to do, nothing launched
