@@ -73,13 +73,14 @@ int hqo_sign(uint64_t seed, uint64_t j, uint32_t i)
     return ((h >> (i & 63)) & 1) ? -1 : 1;
 }
 
-/* Uniform r_i in [0,1) with 24 bits, for coordinate i of tile t (dither).
- * One hash serves coordinates 2m and 2m+1: bits 40..63 and 16..39. */
+/* Uniform r_i in [0,1) on the 16-bit grid, for coordinate i of tile t
+ * (dither).  One hash serves coordinates 4m .. 4m+3: coordinate 4m + k takes
+ * bits 16k .. 16k+15 of H(seed, 2, t, m). */
 float hqo_uniform(uint64_t seed, uint64_t t, uint32_t i)
 {
-    uint64_t h = hqo_hash(seed, 2, t, i >> 1);
-    uint32_t r = (i & 1) ? (uint32_t)((h >> 16) & 0xFFFFFFu) : (uint32_t)(h >> 40);
-    return (float)r * 0x1p-24f;
+    uint64_t h = hqo_hash(seed, 2, t, i >> 2);
+    uint32_t r = (uint32_t)((h >> (16 * (i & 3))) & 0xFFFFu);
+    return (float)r * 0x1p-16f;
 }
 
 /* ------------------------------------------------------------------ */
@@ -298,24 +299,25 @@ void hqo_nearest(int lattice, const float *x, int *c, int32_t *z, float *pt)
 }
 
 /* ------------------------------------------------------------------ */
-/* Subtractive dither for the KV cache [V2]: delta uniform on the Voronoi
- * cell, drawn as a uniform point x0 of a box that tiles space under a
- * sublattice of the lattice (2Z^d for E8 and D4, Z for Z, Z x sqrt3 Z for
- * A2), reduced by the lattice: delta = x0 - Q(x0).  Vector v of tile t. */
+/* Subtractive dither for the KV cache [V2].  The pages ask for subtractive
+ * dither under an idealised sampler without fixing its law.  Reading: delta
+ * is uniform on a box that is a fundamental domain of a sublattice L' of the
+ * lattice L -- L' = D_d for E8 and D4 (box [-1/2,1/2)^(d-1) x [-1,1)),
+ * Z x sqrt3 Z for A2 ([-1/2,1/2) x sqrt3 [-1/2,1/2)), Z for Z ([-1/2,1/2)).
+ * Then delta mod L is uniform, so the error Q(x + delta) - delta - x is
+ * uniform on the Voronoi cell and independent of x (the subtractive-dither
+ * property) with no nearest-point step in drawing delta.  On the 16-bit
+ * grid of the uniforms every value is exact in binary32 except the A2
+ * second coordinate, rounded once.  Vector v of tile t. */
 void hqo_dither(int lattice, uint64_t seed, uint64_t t, uint32_t v, float *delta)
 {
     int d = lattice;
-    float x0[8] = { 0 }, pt[8];
-    int32_t z[8];
-    int c;
     for (int m = 0; m < d; m++) {
         float r = hqo_uniform(seed, t, v * (uint32_t)d + (uint32_t)m);
-        if (lattice == 8 || lattice == 4) x0[m] = 2.0f * r;
-        else if (lattice == 1) x0[m] = r;
-        else x0[m] = (m == 0) ? r : r * (float)sqrt(3.0);
+        if ((lattice == 8 || lattice == 4) && m == d - 1) delta[m] = 2.0f * r - 1.0f;
+        else if (lattice == 2 && m == 1) delta[m] = (r - 0.5f) * (float)sqrt(3.0);
+        else delta[m] = r - 0.5f;
     }
-    hqo_nearest(lattice, x0, &c, z, pt);
-    for (int m = 0; m < d; m++) delta[m] = x0[m] - pt[m];
 }
 
 /* ------------------------------------------------------------------ */

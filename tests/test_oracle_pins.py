@@ -40,8 +40,11 @@ def test_signs_and_uniforms_are_balanced():
     r = np.array([oracle.uniform(3, t, i) for t in range(40) for i in range(128)])
     assert r.min() >= 0.0 and r.max() < 1.0
     assert abs(r.mean() - 0.5) < 4 * math.sqrt(1 / 12 / r.size)
-    # 24-bit grid: r * 2^24 is an integer
-    assert np.all(np.floor(r * 2**24) == r * 2**24)
+    # 16-bit grid: r * 2^16 is an integer, and all four 16-bit fields of a hash are used
+    assert np.all(np.floor(r * 2**16) == r * 2**16)
+    for k in range(4):
+        rk = r.reshape(40, 32, 4)[:, :, k].ravel()
+        assert abs(rk.mean() - 0.5) < 4 * math.sqrt(1 / 12 / rk.size)
 
 
 # ------------------------------------------------------------ Hadamard
@@ -392,17 +395,57 @@ def test_symbols_in_stream_equal_lattice_coordinates():
 
 
 # ------------------------------------------------------------ dither
+BOX_HALF_WIDTH = {"E8": [0.5] * 7 + [1.0], "D4": [0.5] * 3 + [1.0], "A2": [0.5, math.sqrt(3) / 2], "Z": [0.5]}
+
+
 @pytest.mark.parametrize("lat", ["D4", "E8", "Z", "A2"])
-def test_dither_is_uniform_on_the_cell(lat):
-    """delta lies in the Voronoi cell: Q(delta) = 0 and E|delta|^2/d = G V^(2/d)."""
+def test_dither_is_uniform_on_a_sublattice_box(lat):
+    """delta is uniform on the centred box of a sublattice's fundamental
+    domain: D_d for E8 and D4, Z x sqrt3 Z for A2, Z itself; coordinate m
+    spans [-w_m, w_m) with mean 0 and variance w_m^2 / 3."""
     d = FACTS["dimension"][lat]
-    D = np.array([oracle.dither(lat, 13, t, v) for t in range(400) for v in range(128 // d)])
+    w = np.array(BOX_HALF_WIDTH[lat])
+    D = np.array([oracle.dither(lat, 13, t, v) for t in range(500) for v in range(128 // d)]).astype(np.float64)
+    assert np.all(D >= -w) and np.all(D < w)
+    assert np.all(np.abs(D.mean(axis=0)) < 4 * w / math.sqrt(3 * D.shape[0]))
+    assert np.all(np.abs(D.var(axis=0) / (w ** 2 / 3) - 1) < 0.06)
+    # the box's volume is a whole number of lattice cells: 2 V for E8 and A2 (their sublattices
+    # D8 and Z x sqrt3 Z have index 2), V for D4 and Z (the box is a fundamental domain of the lattice)
+    cells = np.prod(2 * w) / FACTS["cell_volume"][lat]
+    assert abs(cells - (2 if lat in ("E8", "A2") else 1)) < 1e-12
+
+
+@pytest.mark.parametrize("lat", ["D4", "E8", "Z", "A2"])
+def test_dither_reduced_by_the_lattice_is_uniform_on_the_cell(lat):
+    """delta - Q(delta) lies in the Voronoi cell with the cell's second moment
+    G V^(2/d) and mean 0: delta mod the lattice is uniform, which is what
+    subtractive dither needs."""
+    d = FACTS["dimension"][lat]
+    D = np.array([oracle.dither(lat, 21, t, v) for t in range(500) for v in range(128 // d)])
     _, _, P = oracle.nearest_batch(lat, D)
-    assert np.mean(np.all(P == 0, axis=1)) > 0.999
-    m2 = np.mean(np.sum(D.astype(np.float64) ** 2, axis=1)) / d
+    R = D.astype(np.float64) - P
+    _, _, P2 = oracle.nearest_batch(lat, R.astype(np.float32))
+    assert np.mean(np.all(P2 == 0, axis=1)) > 0.999
+    m2 = np.mean(np.sum(R ** 2, axis=1)) / d
     ref = FACTS["G"][lat] * FACTS["cell_volume"][lat] ** (2 / d)
     assert abs(m2 / ref - 1) < 0.05
-    assert np.all(np.abs(D.mean(axis=0)) < 0.05)
+    assert np.all(np.abs(R.mean(axis=0)) < 0.05)
+
+
+def test_sixteen_bit_dither_grid_bias_is_below_two_to_minus_sixteen():
+    """Exact, by enumeration of the grid: with delta = r - 1/2 over all 2^16
+    grid values r, the mean error rint(x + delta) - delta - x of the scalar
+    lattice is within 2^-16 of 0 for any x (a sample of x, ties included)."""
+    r = np.arange(2**16, dtype=np.float64) * 2.0**-16
+    delta = r - 0.5
+    for x in [0.0, 0.25, 0.5, 1e-6, 0.3333, -1.75, 123.456789, 2.0**-17, 0.5 + 2.0**-17]:
+        y = x + delta
+        q = np.where(y - np.floor(y) == 0.5, np.floor(y) + (np.floor(y) % 2 == 1), np.round(y))
+        bias = np.mean(q - delta - x)
+        assert abs(bias) <= 2.0**-16, (x, bias)
+    # the oracle's scalar dither lies on that grid
+    D = np.array([oracle.dither("Z", 5, t, v)[0] for t in range(50) for v in range(128)], np.float64)
+    assert np.all((D + 0.5) * 2**16 == np.floor((D + 0.5) * 2**16))
 
 
 def kv_rows(vec, rows):
