@@ -35,20 +35,6 @@ namespace {
 constexpr int kAttnWarps = 8, kAttnThreads = kAttnWarps * 32;
 constexpr int kFactorChunk = 256;  // splits merged per pass of the combine
 
-template <int N, int D, int EPL>
-__device__ __forceinline__ void dither_sub(const DecodeArgs &a, int64_t t, int l, float (&pt)[EPL])
-{
-    constexpr int VPL = EPL / D;
-    const uint64_t tkey = mix64(a.dither_key ^ (uint64_t)t);
-#pragma unroll
-    for (int q = 0; q < VPL; q++) {
-        float dl[D];
-        dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
-#pragma unroll
-        for (int m = 0; m < D; m++) pt[q * D + m] = __fsub_rn(pt[q * D + m], dl[m]);
-    }
-}
-
 // Block-wide max or sum of GB values per thread (one per query); every
 // thread gets the results.  `red` holds kAttnWarps * GB floats.
 template <int GB, bool MAX>
@@ -153,7 +139,7 @@ __global__ void __launch_bounds__(kAttnThreads) kv_attention_kernel(const AttnAr
         float pt[EPL];
         uint32_t sbits;
         const bool bad = parse_tile<N, D, EPL>(a.k, tg, wbuf, mask, l, pt, sbits);
-        if (!bad && sbits) dither_sub<N, D, EPL>(a.k, tg, l, pt);
+        if (!bad && sbits) sub_dither<D, EPL>(mix64(a.k.dither_key ^ (uint64_t)tg), l, pt, a.k.a2);
         float dot[GB];
 #pragma unroll
         for (int g = 0; g < GB; g++) {
@@ -214,7 +200,7 @@ __global__ void __launch_bounds__(kAttnThreads) kv_attention_kernel(const AttnAr
         float pt[EPL];
         uint32_t sbits;
         const bool bad = parse_tile<N, D, EPL>(a.v, tg, wbuf, mask, l, pt, sbits);
-        if (!bad && sbits) dither_sub<N, D, EPL>(a.v, tg, l, pt);
+        if (!bad && sbits) sub_dither<D, EPL>(mix64(a.v.dither_key ^ (uint64_t)tg), l, pt, a.v.a2);
         const float delta = bf16_bits_to_float(sbits);
 #pragma unroll
         for (int g = 0; g < GB; g++) {

@@ -44,16 +44,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
         uint32_t sb;
         const bool bad = parse_tile<N, D, EPL>(a, t, wbuf, mask, l, pt, sb);
         if constexpr (DITHER) {
-            if (!bad && sb) {
-                const uint64_t tkey = mix64(a.dither_key ^ (uint64_t)t);
-#pragma unroll
-                for (int q = 0; q < VPL; q++) {
-                    float dl[D];
-                    dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
-#pragma unroll
-                    for (int m = 0; m < D; m++) pt[q * D + m] = __fsub_rn(pt[q * D + m], dl[m]);
-                }
-            }
+            if (!bad && sb) sub_dither<D, EPL>(mix64(a.dither_key ^ (uint64_t)t), l, pt, a.a2);
         }
         const float scale = bf16_bits_to_float(sb) * (1.0f / N);  // exact: a power-of-two step
         float v[EPL];

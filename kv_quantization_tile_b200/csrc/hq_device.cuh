@@ -269,48 +269,68 @@ __device__ __forceinline__ void nearest(const float (&x)[D], int &c, int (&z)[D]
 }
 
 // ------------------------------------------------------------- dither
-// r_i uniform on the 24-bit grid of [0,1): one hash per coordinate pair,
-// bits 40..63 for the even and 16..39 for the odd coordinate.
-__device__ __forceinline__ void uniform_pair(uint64_t tile_key, uint32_t pair, float &r0, float &r1)
+// Four uniforms on the 16-bit grid of [0,1) for coordinates 4g .. 4g+3 of a
+// tile: coordinate 4g + k takes bits 16k .. 16k+15 of mix64(tile_key ^ g).
+__device__ __forceinline__ void uniform4(uint64_t tile_key, uint32_t g, float (&r)[4])
 {
-    uint64_t h = mix64(tile_key ^ (uint64_t)pair);
-    r0 = (float)(uint32_t)(h >> 40) * 0x1p-24f;
-    r1 = (float)(uint32_t)((h >> 16) & 0xFFFFFFu) * 0x1p-24f;
+    const uint64_t h = mix64(tile_key ^ (uint64_t)g);
+    const uint32_t lo = (uint32_t)h, hi = (uint32_t)(h >> 32);
+    r[0] = (float)(lo & 0xffffu) * 0x1p-16f;
+    r[1] = (float)(lo >> 16) * 0x1p-16f;
+    r[2] = (float)(hi & 0xffffu) * 0x1p-16f;
+    r[3] = (float)(hi >> 16) * 0x1p-16f;
 }
 
-// Dither of vector q (coordinates q*D .. q*D+D-1) of a tile: delta = x0 -
-// Q(x0), x0 uniform on a box that tiles space under a sublattice.
+// Dither coordinate m of a D-vector from its uniform r: a centred box that
+// is a fundamental domain of a sublattice (D_d for E8 and D4: [-1/2,1/2)^(d-1)
+// x [-1,1); Z x sqrt3 Z for A2; Z for Z).  Exact except the A2 second
+// coordinate (one rounding).
 template <int D>
-__device__ __forceinline__ void dither(uint64_t tile_key, uint32_t q, float (&delta)[D],
-                                       const A2Consts &a2)
+__device__ __forceinline__ float box_dither(float r, int m, const A2Consts &a2)
 {
-    float x0[D], p[D];
-    int z[D], c;
-#pragma unroll
-    for (int m = 0; m < D; m += 2) {
-        float r0, r1;
-        if constexpr (D == 1) {
-            uint32_t i = q;
-            float e, o;
-            uniform_pair(tile_key, i >> 1, e, o);
-            r0 = (i & 1) ? o : e;
-            r1 = 0.0f;
-        } else {
-            uniform_pair(tile_key, (q * D + m) >> 1, r0, r1);
-        }
-        if constexpr (D == 8 || D == 4) {
-            x0[m] = __fmul_rn(2.0f, r0);
-            x0[m + 1] = __fmul_rn(2.0f, r1);
-        } else if constexpr (D == 2) {
-            x0[0] = r0;
-            x0[1] = __fmul_rn(r1, a2.s3);
-        } else {
-            x0[0] = r0;
-        }
+    if constexpr (D == 8 || D == 4) {
+        return m == D - 1 ? __fmaf_rn(2.0f, r, -1.0f) : __fsub_rn(r, 0.5f);
+    } else if constexpr (D == 2) {
+        return m == 1 ? __fmul_rn(__fsub_rn(r, 0.5f), a2.s3) : __fsub_rn(r, 0.5f);
+    } else {
+        return __fsub_rn(r, 0.5f);
     }
-    nearest<D>(x0, c, z, p, a2);
+}
+
+// Dither of vector q of lane l (coordinates l*EPL + q*D ...).  For D < 4 one
+// hash serves 4/D consecutive vectors: r4 carries it from the vector that
+// starts a group of four coordinates to the next ones (call with q in order).
+template <int D, int EPL>
+__device__ __forceinline__ void dither_vec(uint64_t tile_key, int l, int q, float (&r4)[4], float (&delta)[D],
+                                           const A2Consts &a2)
+{
+    const uint32_t g0 = (uint32_t)l * (EPL / 4) + (uint32_t)(q * D) / 4;
+    if constexpr (D >= 4) {
 #pragma unroll
-    for (int m = 0; m < D; m++) delta[m] = __fsub_rn(x0[m], p[m]);
+        for (int b = 0; b < D / 4; b++) {
+            uniform4(tile_key, g0 + b, r4);
+#pragma unroll
+            for (int k = 0; k < 4; k++) delta[4 * b + k] = box_dither<D>(r4[k], 4 * b + k, a2);
+        }
+    } else {
+        if (((q * D) & 3) == 0) uniform4(tile_key, g0, r4);
+#pragma unroll
+        for (int m = 0; m < D; m++) delta[m] = box_dither<D>(r4[((q * D) & 3) + m], m, a2);
+    }
+}
+
+// Subtract the dither from lane l's EPL lattice coordinates.
+template <int D, int EPL>
+__device__ __forceinline__ void sub_dither(uint64_t tile_key, int l, float (&pt)[EPL], const A2Consts &a2)
+{
+    float r4[4];
+#pragma unroll
+    for (int q = 0; q < EPL / D; q++) {
+        float dl[D];
+        dither_vec<D, EPL>(tile_key, l, q, r4, dl, a2);
+#pragma unroll
+        for (int m = 0; m < D; m++) pt[q * D + m] = __fsub_rn(pt[q * D + m], dl[m]);
+    }
 }
 
 // ------------------------------------------------------------- symbols

@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
                 if (sb != 0) {
                     const float inv = __frcp_rn(bf16_bits_to_float(sb));
                     const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
+                    float r4[4];
     #pragma unroll
                     for (int q = 0; q < VPL; q++) {
                         float x[D], p[D];
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
                         for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
                         if constexpr (DITHER) {
                             float dl[D];
-                            dither<D>(tkey, (uint32_t)(l * VPL + q), dl, a.a2);
+                            dither_vec<D, EPL>(tkey, l, q, r4, dl, a.a2);
     #pragma unroll
                             for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
                         }
