@@ -141,8 +141,10 @@ int hq_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, in
               uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
 /* KV-cache encode ([V1] (iv), [V2] subtractive dither): as hq_encode, with a
- * seeded dither uniform on the lattice's Voronoi cell added before the
- * nearest-point step.  A KV slab is laid out as (heads * tokens) rows of
+ * seeded dither added before the nearest-point step: uniform (16-bit grid)
+ * on a centred box that is a fundamental domain of a sublattice (D_d for E8
+ * and D4, Z x sqrt3 Z for A2, Z for Z), so the decoded error is uniform on
+ * the Voronoi cell and independent of the input.  A KV slab is laid out as (heads * tokens) rows of
  * head_dim columns, tile = head_dim, so each tile is one cached vector. */
 int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
                  float bps, uint64_t seed, const hq_stream *out, void *workspace,
@@ -181,10 +183,12 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
 /* Bytes of device workspace hq_kv_attention needs: 256-byte-rounded
  * counters (heads * ceil(group / queries per block) uint32) followed by
  * heads * group * splits * (head_dim + 2) floats of per-split partial
- * results.  `splits` depends only on (heads, tokens, group) and the GPU's SM
- * count, so query this on the device the call will run on.  Host only.
- * HQ_ERR_ARG for negative sizes, head_dim not 64/128/256, group < 1 or
- * out == NULL. */
+ * results, for the largest number of token splits a call of this shape can
+ * choose (a call picks its splits from the kernel's occupancy and never
+ * exceeds this).  Depends on (heads, tokens, head_dim, group) and the SM
+ * count of the current device, so query it on the device the call will run
+ * on.  Host only.  HQ_ERR_ARG for negative sizes, head_dim not 64/128/256,
+ * group < 1 or out == NULL. */
 int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim, int group,
                                     uint64_t *out);
 

@@ -207,7 +207,7 @@ struct AttnWorkspace {
 AttnWorkspace attention_workspace(int64_t heads, int64_t tokens, int head_dim, int group)
 {
     AttnWorkspace w{};
-    attention_splits(heads, tokens, group, &w.splits, &w.tokens_per_split);
+    attention_splits(heads, tokens, group, 8, &w.splits, &w.tokens_per_split);  // the largest split count
     const int gb = attention_queries_per_block(group);
     const uint64_t counters = (uint64_t)heads * (uint64_t)((group + gb - 1) / gb);
     w.counter_bytes = (counters * 4 + 255) / 256 * 256;
@@ -366,8 +366,6 @@ int hq_kv_attention(const hq_stream *k, const hq_stream *v, int64_t heads, int64
     a.heads = heads;
     a.tokens = tokens;
     a.group = group;
-    a.splits = w.splits;
-    a.tokens_per_split = w.tokens_per_split;
     a.scale = scale;
     a.status = d_status;
     return launch_attention(head_dim, lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;

@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kAttnWarps = 8, kAttnThreads = kAttnWarps * 32;
 constexpr int kFactorChunk = 256;  // splits merged per pass of the combine
+constexpr int kAttnWaves = 1;      // waves of resident blocks the token splits aim to fill
 
 // Block-wide max or sum of GB values per thread (one per query); every
 // thread gets the results.  `red` holds kAttnWarps * GB floats.
@@ -65,10 +66,15 @@ __device__ __forceinline__ void block_reduce(float (&v)[GB], float *red)
 
 // Shared memory: K and V sign words | rotated queries (GB x n, float4 chunk c
 // of lane l at (g * EPL/4 + c) * LPT + l) | region U, first the per-group
-// staged tiles and the scores (GB x tokens_per_split), later reused for the
+// staged tiles, the scores (GB x tokens_per_split) and each warp's value
+// staging rows (TPW x n) and weights (TPW x GB), later reused for the
 // cross-warp partial outputs and the combine.
+// Resident blocks per SM the register allocation targets: four, fewer where
+// the GB x n/32 column accumulators of head_dim 256 would spill.
+constexpr int attn_min_blocks(int n, int gb) { return n * gb >= 2048 ? 2 : (n == 256 && n * gb >= 1024 ? 3 : 4); }
+
 template <int N, int D, int EPL, int GB>
-__global__ void __launch_bounds__(kAttnThreads) kv_attention_kernel(const AttnArgs a)
+__global__ void __launch_bounds__(kAttnThreads, attn_min_blocks(N, GB)) kv_attention_kernel(const AttnArgs a)
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kAttnWarps * TPW, C4 = EPL / 4;
     constexpr int WPT = N / 64;
@@ -189,43 +195,69 @@ __global__ void __launch_bounds__(kAttnThreads) kv_attention_kernel(const AttnAr
             s_stat[GB + g] = ls[g];
         }
 
-    // ---- values: acc_g = sum_t p_gt Delta_t (y_t - delta_t), rotated domain
-    float acc[GB][EPL];
+    // ---- values: acc_g = sum_t p_gt Delta_t (y_t - delta_t), rotated domain.
+    // The groups of a warp parse one token each into the warp's staging rows
+    // (lane l's chunk c at slot c ^ swz(l), conflict-free 128-bit stores) with
+    // the token's weights p_gt Delta_t; then every lane accumulates columns
+    // lane + 32 c of all staged tokens for all GB queries.
+    constexpr int CPL = N / 32;           // columns per lane
+    constexpr int U4 = EPL / 4;
+    float *stage = scores + ((GB * tps + 3) & ~3);
+    float *zw = stage + warp * TPW * N;                            // [TPW][n]
+    float *ww = stage + kAttnWarps * TPW * N + warp * TPW * GB;    // [TPW][GB]
+    int pos[CPL];  // staging position of column lane + 32 c
+#pragma unroll
+    for (int c = 0; c < CPL; c++) {
+        const int i = lane + 32 * c, li = i / EPL, cc = (i % EPL) / 4;
+        pos[c] = li * EPL + 4 * (cc ^ ((li * U4 >> 3) & (U4 - 1))) + (i & 3);
+    }
+    float acc[GB][CPL];
 #pragma unroll
     for (int g = 0; g < GB; g++)
 #pragma unroll
-        for (int r = 0; r < EPL; r++) acc[g][r] = 0.0f;
-    for (int i = gid; i < nt; i += GPB) {
-        const int64_t tg = (int64_t)h * a.tokens + t0 + i;
-        float pt[EPL];
-        uint32_t sbits;
-        const bool bad = parse_tile<N, D, EPL>(a.v, tg, wbuf, mask, l, pt, sbits);
-        if (!bad && sbits) sub_dither<D, EPL>(mix64(a.v.dither_key ^ (uint64_t)tg), l, pt, a.v.a2);
-        const float delta = bf16_bits_to_float(sbits);
+        for (int c = 0; c < CPL; c++) acc[g][c] = 0.0f;
+    const int grp = lane / LPT;
+    for (int base = warp * TPW; base < nt; base += GPB) {
+        const int i = base + grp;
+        if (i < nt) {
+            const int64_t tg = (int64_t)h * a.tokens + t0 + i;
+            float pt[EPL];
+            uint32_t sbits;
+            const bool bad = parse_tile<N, D, EPL>(a.v, tg, wbuf, mask, l, pt, sbits);
+            if (!bad && sbits) sub_dither<D, EPL>(mix64(a.v.dither_key ^ (uint64_t)tg), l, pt, a.v.a2);
+            float4 *row = reinterpret_cast<float4 *>(zw + grp * N + l * EPL);
+            const int sw = (l * U4 >> 3) & (U4 - 1);
 #pragma unroll
-        for (int g = 0; g < GB; g++) {
-            const float w = scores[g * tps + i] * delta;
+            for (int c = 0; c < U4; c++) row[c ^ sw] = make_float4(pt[4 * c], pt[4 * c + 1], pt[4 * c + 2], pt[4 * c + 3]);
+            if (l < GB) ww[grp * GB + l] = scores[l * tps + i] * bf16_bits_to_float(sbits);
+            if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
+        } else {  // past the split's end: weight 0 on a zero row
+            float4 *row = reinterpret_cast<float4 *>(zw + grp * N + l * EPL);
 #pragma unroll
-            for (int r = 0; r < EPL; r++) acc[g][r] = fmaf(w, pt[r], acc[g][r]);
+            for (int c = 0; c < U4; c++) row[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (l < GB) ww[grp * GB + l] = 0.0f;
         }
-        if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < TPW; s++) {
+            float w[GB];
+#pragma unroll
+            for (int g = 0; g < GB; g++) w[g] = ww[s * GB + g];
+#pragma unroll
+            for (int c = 0; c < CPL; c++) {
+                const float z = zw[s * N + pos[c]];
+#pragma unroll
+                for (int g = 0; g < GB; g++) acc[g][c] = fmaf(w[g], z, acc[g][c]);
+            }
+        }
+        __syncwarp();
     }
-    // groups of a warp hold the same coordinates: fold them, then the warps
-#pragma unroll
-    for (int m = LPT; m < 32; m <<= 1)
-#pragma unroll
-        for (int g = 0; g < GB; g++)
-#pragma unroll
-            for (int r = 0; r < EPL; r++) acc[g][r] += __shfl_xor_sync(FULL, acc[g][r], m);
     __syncthreads();  // U (staged tiles, weights) is free from here on
     float *red = U;   // [warps][GB][n]
-    if (lane < LPT)
 #pragma unroll
-        for (int g = 0; g < GB; g++)
+    for (int g = 0; g < GB; g++)
 #pragma unroll
-            for (int c = 0; c < C4; c++)
-                *reinterpret_cast<float4 *>(red + (warp * GB + g) * N + l * EPL + 4 * c) =
-                    make_float4(acc[g][4 * c], acc[g][4 * c + 1], acc[g][4 * c + 2], acc[g][4 * c + 3]);
+        for (int c = 0; c < CPL; c++) red[(warp * GB + g) * N + lane + 32 * c] = acc[g][c];
     __syncthreads();
     for (int e = tid; e < G * N; e += kAttnThreads) {
         const int g = e / N, i = e % N;
@@ -328,16 +360,16 @@ __global__ void __launch_bounds__(kAttnThreads) kv_attention_kernel(const AttnAr
 // ------------------------------------------------------------------ launch
 namespace {
 
-// Coordinates per lane: fewer when many queries share the block, so the
-// GB x EPL accumulators stay in registers.
+// Coordinates per lane of a parsed tile.
 template <int N, int GB>
-constexpr int attn_epl() { return N == 64 ? 8 : (GB * (N / 8) >= 128 ? 8 : 16); }
+constexpr int attn_epl() { return N == 64 ? 8 : 16; }
 
 template <int N, int GB>
 size_t attn_smem(uint32_t wmax, int tps)
 {
     constexpr int EPL = attn_epl<N, GB>(), GPB = kAttnWarps * (32 / (N / EPL));
-    const size_t staged = (size_t)GPB * group_words(wmax) * 4 + (size_t)GB * tps * 4;
+    const size_t staged = (size_t)GPB * group_words(wmax) * 4 + (size_t)((GB * tps + 3) & ~3) * 4 +
+                          (size_t)kAttnWarps * (32 / (N / EPL)) * (N + GB) * 4;
     const size_t red = (size_t)kAttnWarps * GB * N * 4;
     const size_t merge = (size_t)GB * (kFactorChunk + N) * 4;
     size_t u = staged > red ? staged : red;
@@ -345,15 +377,22 @@ size_t attn_smem(uint32_t wmax, int tps)
     return 2 * (N / 64) * 8 + (size_t)GB * N * 4 + u;
 }
 
+// Splits from the kernel's occupancy at the largest split, then the launch.
 template <int N, int D, int GB>
-cudaError_t launch_attention_t(const AttnArgs &a, int zchunks, cudaStream_t s)
+cudaError_t launch_attention_t(AttnArgs a, int zchunks, cudaStream_t s)
 {
     constexpr int EPL = attn_epl<N, GB>();
     const uint32_t wmax = a.k.wmax > a.v.wmax ? a.k.wmax : a.v.wmax;
-    const size_t smem = attn_smem<N, GB>(wmax, a.tokens_per_split);
     auto kern = kv_attention_kernel<N, D, EPL, GB>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem_max = attn_smem<N, GB>(wmax, 4096 / GB);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
     if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kAttnThreads, smem_max);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    attention_splits(a.heads, a.tokens, a.group, per_sm, &a.splits, &a.tokens_per_split);
+    const size_t smem = attn_smem<N, GB>(wmax, a.tokens_per_split);
     kern<<<dim3((unsigned)a.splits, (unsigned)a.heads, (unsigned)zchunks), kAttnThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
@@ -384,18 +423,22 @@ cudaError_t launch_attention_n(int lattice, int gb, const AttnArgs &a, int zchun
 
 int attention_queries_per_block(int group) { return group <= 1 ? 1 : group <= 2 ? 2 : group <= 4 ? 4 : 8; }
 
-// Token splits: about four blocks per SM over the whole grid, at least 128
-// tokens per split where the sequence allows, and at most 4096 / GB tokens
-// per split so the GB rows of scores fit in 16 KB of shared memory.  Every
-// split is non-empty.
-void attention_splits(int64_t heads, int64_t tokens, int group, int *splits, int *tokens_per_split)
+// Token splits: enough to fill kAttnWaves waves of resident blocks
+// (blocks_per_sm per SM) over the heads x query-chunk blocks, but no fewer
+// than 128 tokens per split where the sequence allows and no more than
+// 4096 / GB tokens per split (the GB rows of scores stay within 16 KB of
+// shared memory).  Every split is non-empty.  The count never grows when
+// blocks_per_sm shrinks, so blocks_per_sm = 8 (the most 256-thread blocks an
+// SM holds) bounds the workspace of any launch.
+void attention_splits(int64_t heads, int64_t tokens, int group, int blocks_per_sm, int *splits,
+                      int *tokens_per_split)
 {
     const int gb = attention_queries_per_block(group);
     const int64_t zc = (group + gb - 1) / gb;
     const int64_t tmax = 4096 / gb;
     const int64_t smin = (tokens + tmax - 1) / tmax;
     const int64_t blocks = heads * zc > 0 ? heads * zc : 1;
-    int64_t s = (4 * (int64_t)sm_count() + blocks - 1) / blocks;
+    int64_t s = (int64_t)kAttnWaves * sm_count() * (blocks_per_sm > 0 ? blocks_per_sm : 1) / blocks;
     const int64_t s128 = (tokens + 127) / 128;
     if (s > s128) s = s128;
     if (s < smin) s = smin;
@@ -406,7 +449,7 @@ void attention_splits(int64_t heads, int64_t tokens, int group, int *splits, int
     *tokens_per_split = (int)tps;
 }
 
-cudaError_t launch_attention(int head_dim, int lattice, const AttnArgs &a, cudaStream_t s)
+cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s)
 {
     const int gb = attention_queries_per_block(a.group);
     const int zchunks = (a.group + gb - 1) / gb;

@@ -84,12 +84,15 @@ cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const E
 cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const DecodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
-cudaError_t launch_attention(int head_dim, int lattice, const AttnArgs &a, cudaStream_t s);
+// Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
+cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 
 // Query heads one attention block serves (1, 2, 4 or 8), and the token
-// splits of a call (every split non-empty).
+// splits for `blocks_per_sm` resident blocks (every split non-empty; never
+// more splits for fewer resident blocks).
 int attention_queries_per_block(int group);
-void attention_splits(int64_t heads, int64_t tokens, int group, int *splits, int *tokens_per_split);
+void attention_splits(int64_t heads, int64_t tokens, int group, int blocks_per_sm, int *splits,
+                      int *tokens_per_split);
 
 // Smallest encode chunk (tiles) for a tile length; sizes the workspace.
 int encode_chunk_tiles(int tile);
