@@ -45,6 +45,9 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
+    p.add_argument("--leg", default=None, choices=["gemv", "kv", "kv_attention"],
+                   help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
+    p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
     return p.parse_args()
 
 
@@ -514,9 +517,22 @@ def attention_leg(dev, peak, group=4):
             "decode_then_sdpa_us": round(t_dec * 1e3, 2), "speedup_vs_bf16_sdpa": round(t_sdpa / t, 3)}
 
 
+def run_leg(args):
+    peak, _ = peaks()
+    if args.leg == "gemv":
+        res = gemv_leg("cuda", peak)
+    elif args.leg == "kv":
+        res = kv_leg("cuda", peak)
+    else:
+        res = attention_leg("cuda", peak, group=args.group)
+    print(json.dumps({"leg": args.leg, **res}))
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.leg:
+        run_leg(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
