@@ -186,16 +186,26 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ GPU leg
+KERNEL_HEADERS = ("hq_device.cuh", "hq_parse.cuh", "hq_internal.h")
+
+
+def kernel_source_sha(kernel_file: str) -> str:
+    """sha256 over a kernel's .cu file and the shared device headers."""
+    h = hashlib.sha256()
+    for f in (kernel_file,) + KERNEL_HEADERS:
+        h.update(open(os.path.join(ROOT, "kv_quantization_tile_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
 def traffic_record(kernel_file: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (its sha256 is recorded beside it)."""
+    on the current kernel source (kernel file + shared headers, sha256
+    recorded beside it)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "kv_quantization_tile_b200", "csrc", kernel_file)
     try:
         rec = json.load(open(path))
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
         r = rec.get(kernel_file)
-        if r and r.get("source_sha256") == sha:
+        if r and r.get("source_sha256") == kernel_source_sha(kernel_file):
             return r
     except Exception:
         pass
