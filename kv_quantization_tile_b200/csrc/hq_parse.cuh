@@ -5,12 +5,13 @@
 //   * The tile's words are staged in shared memory (plus zero guard words).
 //   * Coset bits and the fixed-width low parts are read at computed offsets.
 //   * Unary parts: one pass popcounts the unary words (a lane per word) and
-//     records the running count of terminators per word; each lane then
-//     selects the terminator of rank l*EPL - 1 (the end of the previous lane's
-//     codes), which gives its start bit, and parses its EPL codes
-//     sequentially from a bit-reversed 64-bit window with one count-leading-
-//     zeros per code.  A lane whose codes span more than 64 bits parses from
-//     shared memory word by word instead.
+//     scans the counts across the group; the lane holding the word in which
+//     terminator m*EPL - 1 lies writes lane m's start bit (the bit after that
+//     terminator), so no lane searches.  Each lane then parses its EPL codes
+//     from a bit-reversed 64-bit window with one count-leading-zeros and two
+//     funnel shifts per code, once it has checked that no zero run of its
+//     span reaches 32 bits; otherwise (and for spans over 64 bits) it parses
+//     from shared memory word by word.
 // Every read stays inside the tile's own words.  A tile that is not canonical
 // (offsets out of order or past the capacity, k > 15, a scale that is not 0
 // or a positive normal bf16, a terminator count other than n, a word count
@@ -22,19 +23,25 @@
 namespace hq {
 
 // words of shared memory per group: staged tile words + 4 guard words, then
-// the running terminator count of each unary word
-__host__ __device__ constexpr uint32_t group_words(uint32_t wmax) { return 2 * wmax + 4; }
+// the start bit of each lane (up to 32 lanes)
+__host__ __device__ constexpr uint32_t group_words(uint32_t wmax) { return wmax + 4 + 32; }
 
-// position of the r-th (0-based) set bit of v (v has more than r set bits)
+// position of the r-th (0-based) set bit of v (v has more than r set bits):
+// a branch-free binary search on popcounts of halves
 __device__ __forceinline__ uint32_t select_bit(uint32_t v, uint32_t r)
 {
-    uint32_t c = __popc(v & 0xffffu);
-    uint32_t base = 0;
-    if (r >= c) { r -= c; v >>= 16; base = 16; }
-    c = __popc(v & 0xffu);
-    if (r >= c) { r -= c; v >>= 8; base += 8; }
-    for (uint32_t i = 0; i < r; i++) v &= v - 1;
-    return base + (__ffs(v) - 1);
+    uint32_t pos = 0, c;
+    c = __popc(v & 0xffffu);
+    if (r >= c) { r -= c; pos = 16; }
+    c = __popc((v >> pos) & 0xffu);
+    if (r >= c) { r -= c; pos += 8; }
+    c = __popc((v >> pos) & 0xfu);
+    if (r >= c) { r -= c; pos += 4; }
+    c = __popc((v >> pos) & 0x3u);
+    if (r >= c) { r -= c; pos += 2; }
+    c = (v >> pos) & 1u;
+    if (r >= c) pos += 1;
+    return pos;
 }
 
 // Parse tile t into lattice point coordinates pt (binary32).  Returns true
@@ -46,7 +53,7 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     constexpr int LPT = N / EPL;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
     constexpr int VPL = EPL / D;
-    uint32_t *cnt = wbuf + a.wmax + 4;
+    uint32_t *starts = wbuf + a.wmax + 4;
 
     const uint32_t o0 = a.off[t], o1 = a.off[t + 1];
     const int k = a.kk[t];
@@ -60,14 +67,17 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     if (!bad && U0 + (uint32_t)N > 32u * W0) bad = true;
     const uint32_t W = bad ? 0u : W0;
 
+    __syncwarp(mask);  // the group is done with the previous tile's words
     for (uint32_t i = l; i < W; i += LPT) wbuf[i] = __ldg(a.payload + o0 + i);
     if (l < 4) wbuf[W + l] = 0u;
     __syncwarp(mask);
 
-    // ---- unary terminators: running count per unary word
+    // ---- unary terminators: count per word, scanned across the group; the
+    // word holding terminator m*EPL - 1 yields lane m's start
     const uint32_t wu0 = U0 >> 5;
     const uint32_t nwu = W > wu0 ? W - wu0 : 0;  // unary words (the first shared with the low parts)
     uint32_t found = 0;
+    bool last_empty = false;
     for (uint32_t wb = 0; wb < nwu; wb += LPT) {
         const uint32_t wi = wb + l;
         uint32_t v = wi < nwu ? wbuf[wu0 + wi] : 0u;
@@ -79,13 +89,17 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
             const uint32_t o = __shfl_up_sync(mask, incl, d, LPT);
             if (l >= d) incl += o;
         }
-        if (wi < nwu) cnt[wi] = found + incl;
+        if (wi < nwu) {
+            const uint32_t before = found + incl - c, after = found + incl;
+            if (wi == nwu - 1 && c == 0) last_empty = true;  // padding after the last terminator
+            for (uint32_t m = (before + EPL) / EPL; m < (uint32_t)LPT && m * EPL <= after; m++)
+                starts[m] = (wu0 + wi) * 32u + select_bit(v, m * EPL - 1u - before) + 1u - U0;
+        }
         found += __shfl_sync(mask, incl, LPT - 1, LPT);
     }
-    if (!bad && found != (uint32_t)N) bad = true;
+    const bool pad_word = __any_sync(mask, last_empty);
+    if (!bad && (found != (uint32_t)N || pad_word)) bad = true;
     __syncwarp(mask);
-    // canonical word count: the last word holds the last terminator
-    if (!bad && cnt[nwu - 1] == (nwu > 1 ? cnt[nwu - 2] : 0u)) bad = true;
 
 #pragma unroll
     for (int r = 0; r < EPL; r++) pt[r] = 0.0f;
@@ -94,19 +108,7 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
         return true;
     }
 
-    // ---- this lane's first unary bit (relative to U0): after terminator l*EPL - 1
-    uint32_t start = 0;
-    if (l > 0) {
-        const uint32_t R = (uint32_t)l * EPL - 1;
-        uint32_t wi = (uint32_t)(((uint64_t)R * nwu) / (uint32_t)N);  // estimate, then step
-        if (wi >= nwu) wi = nwu - 1;
-        while (wi > 0 && cnt[wi - 1] > R) --wi;
-        while (cnt[wi] <= R) ++wi;
-        const uint32_t before = wi ? cnt[wi - 1] : 0u;
-        uint32_t v = wbuf[wu0 + wi];
-        if (wi == 0) v &= 0xffffffffu << (U0 & 31);
-        start = (wu0 + wi) * 32u + select_bit(v, R - before) + 1u - U0;
-    }
+    const uint32_t start = l > 0 ? starts[l] : 0u;
     // the next lane's start bounds this lane's codes
     uint32_t end = __shfl_down_sync(mask, start, 1, LPT);
     if (l == LPT - 1) {
@@ -143,24 +145,24 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     uint32_t q[EPL];
     const uint32_t span = end - start;
     const uint32_t p0 = U0 + start;
-    if (span <= 64) {
-        const uint32_t w0 = p0 >> 5, sh = p0 & 31;
-        const uint32_t b0 = wbuf[w0], b1 = wbuf[w0 + 1], b2 = wbuf[w0 + 2];
-        uint32_t rh = __brev(__funnelshift_r(b0, b1, sh));  // next stream bit at the MSB
-        uint32_t rl = __brev(__funnelshift_r(b1, b2, sh));
+    // the lane's span in a bit-reversed 64-bit window (next bit at the MSB);
+    // bits past the span are set so they cannot lengthen a zero run
+    const uint32_t w0 = p0 >> 5, sh = p0 & 31;
+    const uint32_t b0 = wbuf[w0], b1 = wbuf[w0 + 1], b2 = wbuf[w0 + 2];
+    uint32_t rh = __brev(__funnelshift_r(b0, b1, sh));
+    uint32_t rl = __brev(__funnelshift_r(b1, b2, sh));
+    if (span < 64) {
+        rl |= span >= 32 ? (0xffffffffu >> (span - 32)) : 0xffffffffu;
+        rh |= span < 32 ? (0xffffffffu >> span) : 0u;
+    }
+    // every zero run shorter than 32 bits: each terminator sits in rh
+    if (span <= 64 && rh != 0 && rl != 0 && (__ffs(rh) - 1u) + __clz(rl) < 32u) {
 #pragma unroll
         for (int r = 0; r < EPL; r++) {
-            uint32_t z = __clz(rh);
-            if (z < 32) {
-                const uint32_t s = z + 1;
-                rh = __funnelshift_lc(rl, rh, s);
-                rl = shl32(rl, s);
-            } else {  // q >= 32: the terminator sits in the low word
-                z = 32 + __clz(rl);
-                rh = shl32(rl, z - 31);
-                rl = 0;
-            }
+            const uint32_t z = __clz(rh);
             q[r] = z;
+            rh = __funnelshift_lc(rl, rh, z + 1);  // a shift of 32 moves rl into rh
+            rl = shl32(rl, z + 1);
         }
     } else {
         uint32_t p = p0;
