@@ -374,6 +374,17 @@ def gemv(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, x,
     return y[: r1 - r0]
 
 
+def gemm(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X, threads: int = 1) -> np.ndarray:
+    """Batched decode + matrix product in binary64: Y = X W_hat^T with W_hat the
+    stream's binary64 decode (rows x cols) and X (batch x cols) -- the plain
+    definition of a layer applied to a batch of activations through the
+    compressed weights ([V2] decode path beside bf16 matrix products)."""
+    W, st = decode(stream, rows, cols, tile, lattice, seed, threads=threads)
+    if st:
+        raise ValueError("corrupt stream")
+    return np.asarray(X, dtype=np.float64).reshape(-1, cols) @ W.T
+
+
 def kv_attention(k_stream: dict, v_stream: dict, heads: int, tokens: int, head_dim: int, lattice,
                  seed_k: int, seed_v: int, q, scale: float, threads: int = 1, group: int = 1) -> np.ndarray:
     """Batch-1 attention over a dithered compressed KV cache, in binary64:

@@ -567,3 +567,19 @@ def test_kv_attention_grouped_queries_follow_their_kv_head():
         errs = [np.max(np.abs(got[qh] - exact(h, q[qh]))) for h in range(heads)]
         assert errs[qh // group] < 0.02, errs
         assert all(e > 0.2 for h, e in enumerate(errs) if h != qh // group), errs
+
+
+def test_gemm_is_decode_then_matmul_and_matches_gemv_per_row():
+    """The batched product equals the decoded matrix times each activation row,
+    and each of its rows equals the (separately pinned) batch-1 GEMV."""
+    rng = np.random.default_rng(77)
+    rows, cols = 10, 512
+    X = bf16_bits_of(rng.standard_normal((rows, cols)) * 0.02)
+    s = oracle.encode(X, 256, "E8", 4.0, 9)
+    W, _ = oracle.decode(s, rows, cols, 256, "E8", 9)
+    A = rng.standard_normal((3, cols))
+    Y = oracle.gemm(s, rows, cols, 256, "E8", 9, A)
+    assert Y.shape == (3, rows)
+    assert np.allclose(Y, A @ W.T, rtol=1e-13, atol=1e-13)
+    for b in range(3):
+        assert np.allclose(Y[b], oracle.gemv(s, rows, cols, 256, "E8", 9, A[b]), rtol=1e-12, atol=1e-12)
