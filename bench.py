@@ -45,7 +45,7 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
-    p.add_argument("--leg", default=None, choices=["gemv", "kv", "kv_attention"],
+    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "kv", "kv_attention"],
                    help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
     p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
     return p.parse_args()
@@ -331,7 +331,7 @@ def run_ours(args):
     if not args.no_extras:
         out["e2e"] = e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier)
         if rank == 0:
-            out["paths"] = {"gemv": gemv_leg(dev, peak), "kv": kv_leg(dev, peak),
+            out["paths"] = {"gemv": gemv_leg(dev, peak), "gemm": gemm_leg(dev, peak), "kv": kv_leg(dev, peak),
                             "kv_attention": attention_leg(dev, peak)}
             out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
@@ -468,6 +468,53 @@ def kv_leg(dev, peak):
     return res
 
 
+def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
+    """Batched decode + matrix product on the tensor cores for the Llama gate
+    projection (14336 x 4096, E8 4 bps): Y = X W_hat^T for X of `batch` bf16
+    rows, against cuBLAS bf16 (torch.matmul) on the uncompressed weights and
+    against decoding to bf16 first.  L2 flushed before each timed launch."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    w1, _, _, _ = workloads.gemv_case(dev)
+    r, c = w1.shape
+    s = hq.alloc_stream(r, c, TILE, LAT, BPS, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    hq.hq_encode(w1, TILE, LAT, BPS, SEED, s, hq.alloc_workspace(r, c, TILE, dev), st)
+    flushbuf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    wd = torch.empty_like(w1)
+    res = {"matrix": f"{r}x{c}", "compressed_bytes": s.nbytes()}
+    for batch in batches:
+        g = torch.Generator(device=dev).manual_seed(6000 + batch)
+        x = torch.randn(batch, c, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(batch, r, dtype=torch.float32, device=dev)
+        ws = hq.alloc_gemm_workspace(r, c, batch, dev)
+
+        def ours():
+            hq.hq_decode_gemm(s, r, c, TILE, LAT, BPS, SEED, x, y, ws, st)
+
+        def dense():
+            torch.matmul(x, w1.t())
+
+        def decode_then_dense():
+            hq.hq_decode(s, r, c, TILE, LAT, BPS, SEED, wd, st)
+            torch.matmul(x, wd.t())
+
+        for _ in range(3):
+            ours(); dense(); decode_then_dense()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        t = time_launches(ours, lambda: flush_l2(flushbuf))
+        td = time_launches(dense, lambda: flush_l2(flushbuf))
+        tdd = time_launches(decode_then_dense, lambda: flush_l2(flushbuf))
+        flops = 2.0 * batch * r * c
+        res[f"batch{batch}"] = {"us": round(t * 1e3, 2), "tflops": round(flops / t / 1e9, 2),
+                                "weights_per_us": round(r * c / t / 1e3, 1),
+                                "bf16_cublas_us": round(td * 1e3, 2), "decode_then_cublas_us": round(tdd * 1e3, 2)}
+    return res
+
+
 def attention_leg(dev, peak, group=4):
     """Batch-1 decode attention of one Llama-3.1-8B layer: 32 query heads over
     the 8 x 32768 x 128 K and V caches (4 query heads per KV head), straight
@@ -531,6 +578,8 @@ def run_leg(args):
     peak, _ = peaks()
     if args.leg == "gemv":
         res = gemv_leg("cuda", peak)
+    elif args.leg == "gemm":
+        res = gemm_leg("cuda", peak)
     elif args.leg == "kv":
         res = kv_leg("cuda", peak)
     else:

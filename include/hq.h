@@ -180,6 +180,34 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    float bps, uint64_t seed, const void *x, float *y, void *stream,
                    int32_t *d_status);
 
+/* Bytes of device workspace hq_decode_gemm needs for this shape: the
+ * rotated activations (bf16, batch rounded up to the block's batch rows x
+ * cols), then, when column tiles are split across blocks, fp32 partial
+ * results (splits x padded batch x rows).  Depends on the SM count of the
+ * current device.  Host only.  HQ_ERR_ARG for negative sizes, a cols that is
+ * not a multiple of 256 or out == NULL. */
+int hq_decode_gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, uint64_t *out);
+
+/* Batched decode + matrix product on the tensor cores ([V2] decode path
+ * beside bf16 matrix products; [V1] MMA decode paths):
+ *   y[b][r] = sum_c x[b][c] w_hat[r][c]   (Y = X W_hat^T)
+ * computed as (1/n) sum_j <H(s_j . x_bj), Delta_rj y_rj>: the weights stay in
+ * the rotated domain and are parsed straight into bf16 tensor-core operands
+ * (Delta y rounded once to bf16, as a bf16 decode would); the activations are
+ * rotated once per call and rounded to bf16; products accumulate in fp32
+ * (tcgen05.mma, tensor memory).
+ *   w          stream of a rows x cols matrix (no dither), tile 256
+ *              (HQ_ERR_UNSUPPORTED for other tiles)
+ *   x          device bf16 [batch][cols], 16-byte aligned
+ *   batch      >= 0 activation rows
+ *   y          device fp32 [batch][rows]
+ *   workspace  device, >= hq_decode_gemm_workspace_bytes, 16-byte aligned
+ * Corrupt tiles count as zero rows of W and raise HQ_ST_CORRUPT; a bounded
+ * wait on the tensor cores that gives up raises HQ_ST_TIMEOUT. */
+int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                   uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                   uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
 /* Bytes of device workspace hq_kv_attention needs: 256-byte-rounded
  * counters (heads * ceil(group / queries per block) uint32) followed by
  * heads * group * splits * (head_dim + 2) floats of per-split partial

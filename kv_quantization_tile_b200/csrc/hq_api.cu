@@ -327,6 +327,54 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
     return launch_gemv(tile, lattice, a, cols, (cudaStream_t)stream) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
+int hq_decode_gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, uint64_t *out)
+{
+    if (!out || rows < 0 || cols < 0 || batch < 0 || cols % 256) return HQ_ERR_ARG;
+    if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
+    GemmPlan p{};
+    gemm_plan(rows, cols, batch, &p);
+    *out = (p.xt_bytes + 255) / 256 * 256 + p.part_bytes;
+    return HQ_OK;
+}
+
+int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t seed,
+                   const void *x, int64_t batch, float *y, void *workspace, uint64_t workspace_bytes, void *stream,
+                   int32_t *d_status)
+{
+    GemmArgs a{};
+    int64_t ntiles = 0;
+    int rc = decode_common(w, rows, cols, tile, lattice, bps, seed, a.w, &ntiles);
+    if (rc) return rc;
+    if (tile != 256) return HQ_ERR_UNSUPPORTED;
+    if (batch < 0) return HQ_ERR_ARG;
+    if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
+    if (batch == 0 || rows == 0) return HQ_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!y || !aligned(y, 4)) return HQ_ERR_ARG;
+    if (cols == 0)
+        return cudaMemsetAsync(y, 0, sizeof(float) * (size_t)(batch * rows), s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
+    GemmPlan p{};
+    gemm_plan(rows, cols, batch, &p);
+    const uint64_t xt_span = (p.xt_bytes + 255) / 256 * 256;
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < xt_span + p.part_bytes) return HQ_ERR_WORKSPACE;
+    a.x = static_cast<const uint16_t *>(x);
+    a.xt = static_cast<uint16_t *>(workspace);
+    a.y = y;
+    a.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + xt_span);
+    a.rows = rows;
+    a.cols = cols;
+    a.tiles_per_row = cols / 256;
+    a.batch = (int)batch;
+    a.batch_pad = p.batch_pad;
+    a.nb = p.nb;
+    a.ksplit = p.ksplit;
+    a.tiles_per_split = p.tiles_per_split;
+    a.sign_key = hash_key(seed, 1);
+    a.status = d_status;
+    return launch_gemm(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
 int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim, int group, uint64_t *out)
 {
     if (!out || heads < 0 || tokens < 0 || !valid_head_dim(head_dim) || group < 1) return HQ_ERR_ARG;

@@ -78,12 +78,33 @@ struct AttnArgs {
     int32_t *status;
 };
 
+// Batched decode + matrix product (tile 256): Y = X W_hat^T.
+struct GemmArgs {
+    DecodeArgs w;               // weight stream, rows x cols
+    const uint16_t *x;          // bf16 [batch][cols]
+    uint16_t *xt;               // bf16 [batch_pad][cols]: rotated activations (workspace)
+    float *y;                   // fp32 [batch][rows]
+    float *part;                // fp32 [ksplit][batch_pad][rows] split-K partials (workspace)
+    int64_t rows, cols, tiles_per_row;
+    int batch, batch_pad, nb;   // nb: batch rows per block (16, 32 or 64)
+    int ksplit, tiles_per_split;
+    uint64_t sign_key;
+    int32_t *status;
+};
+
+struct GemmPlan {
+    int nb, batch_pad, ksplit, tiles_per_split;
+    uint64_t xt_bytes, part_bytes;  // workspace: X~, then the partials
+};
+
 // Launch helpers; return a cudaError_t.
 cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const DecodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
+cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s);
+void gemm_plan(int64_t rows, int64_t cols, int64_t batch, GemmPlan *p);
 // Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
 cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 

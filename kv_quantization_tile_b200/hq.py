@@ -28,7 +28,8 @@ LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
            "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
-           "hq_kv_attention_workspace_bytes", "hq_kv_attention"]
+           "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
+           "hq_decode_gemm"]
 
 
 class hq_stream(ctypes.Structure):
@@ -61,6 +62,9 @@ _SIGS = {
     "hq_test_encode_stalled": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
                                       _vp, _u64, _vp, _vp, ctypes.c_uint32]),
     "hq_kv_attention_workspace_bytes": (_i32, [_i64, _i64, _i32, _i32, ctypes.POINTER(_u64)]),
+    "hq_decode_gemm_workspace_bytes": (_i32, [_i64, _i64, _i64, ctypes.POINTER(_u64)]),
+    "hq_decode_gemm": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
+                              _u64, _vp, _vp]),
     "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
                                _i32, _f32, _f32, _u64, _u64, _vp, _f32, _vp, _vp, _u64, _vp, _vp]),
 }
@@ -226,6 +230,29 @@ def hq_decode_gemv(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, status
     st = s.struct()
     _check(_lib.hq_decode_gemv(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), _ptr(y),
                                _stream_handle(stream), _ptr(status)), "hq_decode_gemv")
+    return y
+
+
+def hq_decode_gemm_workspace_bytes(rows: int, cols: int, batch: int) -> int:
+    out = _u64(0)
+    _check(_lib.hq_decode_gemm_workspace_bytes(rows, cols, batch, ctypes.byref(out)), "hq_decode_gemm_workspace_bytes")
+    return out.value
+
+
+def alloc_gemm_workspace(rows: int, cols: int, batch: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(hq_decode_gemm_workspace_bytes(rows, cols, batch), 16), dtype=torch.uint8, device=device)
+
+
+def hq_decode_gemm(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, workspace, status=None, stream=None):
+    """Y = X W_hat^T for bf16 activations x [batch, cols] through the stream of
+    W (rows x cols, tile 256); y is fp32 [batch, rows]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == cols
+    batch = x.shape[0]
+    assert y.dtype == torch.float32 and y.is_contiguous() and y.numel() == batch * rows
+    st = s.struct()
+    _check(_lib.hq_decode_gemm(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch, _ptr(y),
+                               _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status)),
+           "hq_decode_gemm")
     return y
 
 

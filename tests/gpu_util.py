@@ -185,3 +185,27 @@ def assert_attention_close(out: np.ndarray, ref: np.ndarray, tol: np.ndarray):
         i = np.unravel_index(np.argmax(err / tol), err.shape)
         raise AssertionError(f"attention off at {i}: {out[i]} vs {ref[i]} (tol {tol[i]}, "
                              f"{int((err > tol).sum())} elements out)")
+
+
+def gemm_tolerance(ref: dict, rows, cols, lat, seed, X: np.ndarray, tile: int = 256) -> np.ndarray:
+    """Per output element, an error bound of the tensor-core batched product
+    against the binary64 oracle.  Each product term A_ri B_bi uses
+    A = bf16(Delta y) and B = bf16(x~) with x~ = H(s . x) from an fp32 transform
+    (error <= g(log2 n) ||x_j||_1 per element): |A B - z x~| <= (2u + u^2)
+    |z||x~| + (1 + u) |z| g(log2 n) ||x_j||_1 with u = 2^-8 (bf16); the fp32
+    accumulation over every term (tensor-core adds bounded with 2^-23 per
+    add, cols + 64 deep) adds (cols + 64) 2^-23 sum |z||x~|; all over n."""
+    u, u32 = 2.0**-8, 2.0**-23
+    tpr = cols // tile
+    W, _ = oracle.decode(ref, rows, cols, tile, lat, seed, threads=8)
+    H = scipy.linalg.hadamard(tile).astype(np.float64)
+    S = np.stack([oracle.signs(seed, j, tile) for j in range(tpr)]).astype(np.float64)
+    Z = np.abs((W.reshape(rows, tpr, tile) * S[None]) @ H)                    # |Delta y|
+    Xa = np.asarray(X, np.float64).reshape(-1, tpr, tile)
+    Xt = np.abs((Xa * S[None]) @ H)                                           # |x~|
+    xl1 = np.abs(Xa).sum(axis=2)                                              # ||x_bj||_1
+    dots = Xt.reshape(Xt.shape[0], -1) @ Z.reshape(rows, -1).T
+    rot = xl1 @ Z.sum(axis=2).T
+    L = math.log2(tile)
+    g = L * 2.0**-24 / (1 - L * 2.0**-24)
+    return ((2 * u + u * u + (cols + 64) * u32) * dots + (1 + u) * g * rot) / tile + 1e-30
