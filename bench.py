@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--leg", default=None, choices=["gemv", "gemm", "kv", "kv_attention"],
                    help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
     p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
+    p.add_argument("--batch", type=int, default=None, help="one batch size for --leg gemm")
     return p.parse_args()
 
 
@@ -579,7 +580,7 @@ def run_leg(args):
     if args.leg == "gemv":
         res = gemv_leg("cuda", peak)
     elif args.leg == "gemm":
-        res = gemm_leg("cuda", peak)
+        res = gemm_leg("cuda", peak, batches=(args.batch,) if args.batch else (1, 16, 64, 256))
     elif args.leg == "kv":
         res = kv_leg("cuda", peak)
     else:

@@ -332,7 +332,7 @@ int hq_decode_gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, ui
     if (!out || rows < 0 || cols < 0 || batch < 0 || cols % 256) return HQ_ERR_ARG;
     if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
     GemmPlan p{};
-    gemm_plan(rows, cols, batch, &p);
+    gemm_plan(rows, cols, batch, 2, &p);  // the most splits any launch picks
     *out = (p.xt_bytes + 255) / 256 * 256 + p.part_bytes;
     return HQ_OK;
 }
@@ -355,7 +355,7 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
         return cudaMemsetAsync(y, 0, sizeof(float) * (size_t)(batch * rows), s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
     GemmPlan p{};
-    gemm_plan(rows, cols, batch, &p);
+    gemm_plan(rows, cols, batch, 2, &p);  // workspace bound; the launch re-plans
     const uint64_t xt_span = (p.xt_bytes + 255) / 256 * 256;
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < xt_span + p.part_bytes) return HQ_ERR_WORKSPACE;
     a.x = static_cast<const uint16_t *>(x);

@@ -326,14 +326,18 @@ __global__ void splitk_reduce_kernel(const GemmArgs a)
 // ------------------------------------------------------------------ launch
 int gemm_block_batch(int64_t batch) { return batch <= 16 ? 16 : (batch <= 32 ? 32 : 64); }
 
-void gemm_plan(int64_t rows, int64_t cols, int64_t batch, GemmPlan *p)
+// Column splits: enough work items for about three waves of resident
+// blocks (blocks_per_sm per SM), so the last wave is nearly full.  The count
+// never grows when blocks_per_sm shrinks; two (the register limit of 512
+// threads x 64 registers) bounds the workspace.
+void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p)
 {
     p->nb = gemm_block_batch(batch);
     p->batch_pad = (int)(((batch + p->nb - 1) / p->nb) * p->nb);
     const int64_t tpr = cols / kGemmN;
     const int64_t blocks = ((rows + kGemmM - 1) / kGemmM) * (p->batch_pad / p->nb);
-    // column splits: enough work items for two resident blocks per SM
-    int64_t ks = (2 * (int64_t)sm_count() + blocks - 1) / (blocks > 0 ? blocks : 1);
+    const int64_t slots = 3 * (int64_t)sm_count() * (blocks_per_sm > 0 ? blocks_per_sm : 1);
+    int64_t ks = (slots + blocks - 1) / (blocks > 0 ? blocks : 1);
     if (ks > tpr) ks = tpr;
     if (ks < 1) ks = 1;
     int64_t tps = (tpr + ks - 1) / ks;
@@ -347,17 +351,39 @@ void gemm_plan(int64_t rows, int64_t cols, int64_t batch, GemmPlan *p)
 namespace {
 
 template <int D, int NB>
-cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s)
+cudaError_t launch_gemm_t(GemmArgs a, cudaStream_t s)
 {
     const size_t smem = gemm_operand_bytes(kGemmM) + gemm_operand_bytes(NB) +
                         (size_t)kGemmWarps * 2 * group_words(a.w.wmax) * 4;
     auto kern = gemm_tc_kernel<D, NB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // Resident blocks per SM: the register limit of 512 threads x 64
+    // registers is two; shared memory may allow fewer.  (Computed from the
+    // device limits: the occupancy query reported one block where two are
+    // resident.)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    int dev = 0, smem_sm = 0, reserved = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+    int per_sm = (int)((size_t)smem_sm / (smem + 256 + (size_t)reserved));
+    if (per_sm > 2) per_sm = 2;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    GemmPlan p{};
+    gemm_plan(a.rows, a.cols, a.batch, per_sm, &p);  // never more splits than the workspace holds
+    a.ksplit = p.ksplit;
+    a.tiles_per_split = p.tiles_per_split;
     // one block per work item (measured faster than a persistent grid here)
     const int64_t items = ((a.rows + kGemmM - 1) / kGemmM) * (a.batch_pad / NB) * a.ksplit;
     if (items >= ((int64_t)1 << 31)) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)(items > 0 ? items : 1), kGemmThreads, smem, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.ksplit == 1) return e;
+    int64_t n = (int64_t)a.batch * a.rows, blocks = (n + 255) / 256;
+    if (blocks > 8 * (int64_t)sm_count()) blocks = 8 * (int64_t)sm_count();
+    splitk_reduce_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -382,16 +408,11 @@ cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s)
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     switch (lattice) {
-    case 1: e = launch_gemm_d<1>(a, s); break;
-    case 2: e = launch_gemm_d<2>(a, s); break;
-    case 4: e = launch_gemm_d<4>(a, s); break;
-    default: e = launch_gemm_d<8>(a, s); break;
+    case 1: return launch_gemm_d<1>(a, s);
+    case 2: return launch_gemm_d<2>(a, s);
+    case 4: return launch_gemm_d<4>(a, s);
+    default: return launch_gemm_d<8>(a, s);
     }
-    if (e != cudaSuccess || a.ksplit == 1) return e;
-    int64_t n = (int64_t)a.batch * a.rows, blocks = (n + 255) / 256;
-    if (blocks > 8 * (int64_t)sm_count()) blocks = 8 * (int64_t)sm_count();
-    splitk_reduce_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(a);
-    return cudaGetLastError();
 }
 
 }  // namespace hq

@@ -104,7 +104,9 @@ cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const D
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);
 cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s);
-void gemm_plan(int64_t rows, int64_t cols, int64_t batch, GemmPlan *p);
+// Plan for blocks_per_sm resident blocks; the launch re-plans from the
+// kernel's occupancy (never more splits than for two blocks per SM).
+void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
 // Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
 cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 
