@@ -324,7 +324,10 @@ __global__ void splitk_reduce_kernel(const GemmArgs a)
 }
 
 // ------------------------------------------------------------------ launch
-int gemm_block_batch(int64_t batch) { return batch <= 16 ? 16 : (batch <= 32 ? 32 : 64); }
+int gemm_block_batch(int64_t batch)
+{
+    return batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : batch <= 128 ? 128 : 256;
+}
 
 // Column splits: enough work items for about three waves of resident
 // blocks (blocks_per_sm per SM), so the last wave is nearly full.  The count
@@ -393,7 +396,9 @@ cudaError_t launch_gemm_d(const GemmArgs &a, cudaStream_t s)
     switch (a.nb) {
     case 16: return launch_gemm_t<D, 16>(a, s);
     case 32: return launch_gemm_t<D, 32>(a, s);
-    default: return launch_gemm_t<D, 64>(a, s);
+    case 64: return launch_gemm_t<D, 64>(a, s);
+    case 128: return launch_gemm_t<D, 128>(a, s);
+    default: return launch_gemm_t<D, 256>(a, s);
     }
 }
 

@@ -86,7 +86,7 @@ struct GemmArgs {
     float *y;                   // fp32 [batch][rows]
     float *part;                // fp32 [ksplit][batch_pad][rows] split-K partials (workspace)
     int64_t rows, cols, tiles_per_row;
-    int batch, batch_pad, nb;   // nb: batch rows per block (16, 32 or 64)
+    int batch, batch_pad, nb;   // nb: batch rows per block (16, 32, 64, 128 or 256)
     int ksplit, tiles_per_split;
     uint64_t sign_key;
     int32_t *status;

@@ -58,7 +58,8 @@ def test_gemm_matches_oracle(lat, batch):
     check(ref, rows, cols, lat, 4.0, 7, acts(batch, cols, batch))
 
 
-@pytest.mark.parametrize("rows,cols,batch", [(128, 256, 3), (1, 512, 9), (333, 256, 70), (129, 4096, 33)])
+@pytest.mark.parametrize("rows,cols,batch", [(128, 256, 3), (1, 512, 9), (333, 256, 70), (129, 4096, 33),
+                                            (200, 512, 200), (130, 768, 300)])
 def test_gemm_shapes(rows, cols, batch):
     w = weights(rows, cols, rows)
     ref = oracle.encode(host_input(w), 256, "E8", 4.0, 5)
