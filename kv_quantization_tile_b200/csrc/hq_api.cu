@@ -122,7 +122,7 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     const uint64_t need = (uint64_t)ntiles * wmax;
     if (need >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
     if (out->payload_capacity_words < need) return HQ_ERR_CAPACITY;
-    const int G = encode_tiles_per_group(tile, wmax);
+    const int G = encode_tiles_per_group(tile, wmax, ntiles);
     const int64_t chunk_tiles = (int64_t)encode_chunk_tiles(tile) * G;
     const int64_t nchunks = (ntiles + chunk_tiles - 1) / chunk_tiles;
     const uint64_t ws_need = 256 + 8 * (uint64_t)nchunks;

@@ -524,11 +524,17 @@ int groups_for(int tile)
 
 // Tiles per group per chunk: as many as keep the two staged images within
 // 48 KB (at most 8), so a chunk spans up to 8 x (groups per block) tiles.
-int encode_tiles_per_group(int tile, uint32_t wmax)
+int encode_tiles_per_group(int tile, uint32_t wmax, int64_t ntiles)
 {
     const int gpb = groups_for(tile);
-    int g = (int)((48u * 1024u) / (2u * (uint32_t)gpb * wmax * 4u));
-    return g < 1 ? 1 : (g > 8 ? 8 : g);
+    int g = (int)((48u * 1024u) / (2u * (uint32_t)gpb * wmax * 4u));  // two staging images in 48 KB
+    g = g < 1 ? 1 : (g > 8 ? 8 : g);
+    // small matrices: smaller chunks, so every resident block gets about one
+    // (measured best against one-tile and three-per-block chunks)
+    const int64_t blocks = 4 * (int64_t)sm_count();
+    const int64_t gp = ntiles / ((int64_t)gpb * blocks);
+    if (gp < g) g = gp < 1 ? 1 : (int)gp;
+    return g;
 }
 
 // Smallest chunk for a tile length (one tile per group): sizes the workspace.

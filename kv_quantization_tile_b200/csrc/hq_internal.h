@@ -119,8 +119,9 @@ void attention_splits(int64_t heads, int64_t tokens, int group, int blocks_per_s
 
 // Smallest encode chunk (tiles) for a tile length; sizes the workspace.
 int encode_chunk_tiles(int tile);
-// Tiles per lane group per chunk for a tile length and worst-case tile words.
-int encode_tiles_per_group(int tile, uint32_t wmax);
+// Tiles per lane group per chunk for a tile length, worst-case tile words and
+// the call's tile count (small calls get small chunks to spread over the GPU).
+int encode_tiles_per_group(int tile, uint32_t wmax, int64_t ntiles);
 int sm_count();
 
 }  // namespace hq
