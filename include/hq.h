@@ -75,7 +75,8 @@ enum {
     HQ_ERR_UNSUPPORTED = 2,  /* valid request outside what this build handles */
     HQ_ERR_CAPACITY = 3,     /* payload capacity below the worst-case bound */
     HQ_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
-    HQ_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
+    HQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    HQ_ERR_FORMAT = 6        /* a checkpoint buffer is not a valid, intact container */
 };
 
 /* device status bits OR-ed into *d_status */
@@ -281,6 +282,41 @@ int hq_test_encode_stalled(const void *x, int dtype, int64_t rows, int64_t cols,
 int hq_encode_noalloc(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
                       float bps, uint64_t seed, const hq_stream *out, void *stream,
                       int32_t *d_status);
+
+/* ---------------------------------------------------------------- file
+ * Packed checkpoint container for one compressed matrix ([I9] a packed
+ * Rice-coded lattice-index format).  Host memory only: the caller copies the
+ * stream's arrays to the host (and back after reading).  Layout,
+ * little-endian, sections 8-byte aligned: a 128-byte header (magic "HQF1",
+ * version 1, flags, rows, cols, tile, lattice, bps, seed, ntiles,
+ * payload_words, section offsets, FNV-1a 64-bit checksums of the body and of
+ * the header), then tile_off (uint32 x ntiles + 1), tile_scale (uint16 x
+ * ntiles), tile_k (uint8 x ntiles) and the payload (uint32 x payload_words). */
+typedef struct hq_file_info {
+    int64_t rows, cols;
+    int32_t tile, lattice;
+    float bps;
+    uint32_t flags;          /* bit 0: KV stream (decode with dither) */
+    uint64_t seed;
+    uint64_t ntiles;         /* rows * cols / tile */
+    uint64_t payload_words;  /* tile_off[ntiles] */
+} hq_file_info;
+
+/* Bytes of the container for `info`.  HQ_ERR_ARG if the fields are not a
+ * valid shape and codec parameter set (ntiles must equal rows * cols / tile). */
+int hq_file_bytes(const hq_file_info *info, uint64_t *out);
+
+/* Write the container into buf (host, >= hq_file_bytes).  tile_off must end
+ * at payload_words.  HQ_ERR_CAPACITY if buf is too small. */
+int hq_file_write(const hq_file_info *info, const uint32_t *tile_off, const uint16_t *tile_scale,
+                  const uint8_t *tile_k, const uint32_t *payload, void *buf, uint64_t buf_bytes);
+
+/* Check a container (magic, version, header and body checksums, section
+ * layout, parameters, offsets non-decreasing from 0 to the payload size,
+ * k <= 15) and return its info and pointers into buf (any pointer argument
+ * may be NULL).  HQ_ERR_FORMAT for anything that does not check out. */
+int hq_file_read(const void *buf, uint64_t buf_bytes, hq_file_info *info, const uint32_t **tile_off,
+                 const uint16_t **tile_scale, const uint8_t **tile_k, const uint32_t **payload);
 
 #ifdef __cplusplus
 }

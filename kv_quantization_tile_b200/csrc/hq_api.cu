@@ -229,6 +229,7 @@ const char *hq_error_string(int code)
     case HQ_ERR_CAPACITY: return "payload capacity below the worst-case bound";
     case HQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case HQ_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case HQ_ERR_FORMAT: return "not a valid, intact checkpoint container";
     default: return "unknown error";
     }
 }

@@ -12,6 +12,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhq.so")
@@ -21,7 +22,7 @@ if not os.path.exists(_LIB_PATH):
 
 HQ_Z, HQ_A2, HQ_D4, HQ_E8 = 1, 2, 4, 8
 HQ_BF16, HQ_F32 = 0, 1
-HQ_OK, HQ_ERR_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_CAPACITY, HQ_ERR_WORKSPACE, HQ_ERR_CUDA = range(6)
+HQ_OK, HQ_ERR_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_CAPACITY, HQ_ERR_WORKSPACE, HQ_ERR_CUDA, HQ_ERR_FORMAT = range(7)
 HQ_ST_NONFINITE, HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT = 1, 2, 4, 8
 LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 
@@ -29,7 +30,13 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
            "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
-           "hq_decode_gemm"]
+           "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read"]
+
+
+class hq_file_info(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("tile", ctypes.c_int32),
+                ("lattice", ctypes.c_int32), ("bps", ctypes.c_float), ("flags", ctypes.c_uint32),
+                ("seed", ctypes.c_uint64), ("ntiles", ctypes.c_uint64), ("payload_words", ctypes.c_uint64)]
 
 
 class hq_stream(ctypes.Structure):
@@ -63,6 +70,10 @@ _SIGS = {
                                       _vp, _u64, _vp, _vp, ctypes.c_uint32]),
     "hq_kv_attention_workspace_bytes": (_i32, [_i64, _i64, _i32, _i32, ctypes.POINTER(_u64)]),
     "hq_decode_gemm_workspace_bytes": (_i32, [_i64, _i64, _i64, ctypes.POINTER(_u64)]),
+    "hq_file_bytes": (_i32, [ctypes.POINTER(hq_file_info), ctypes.POINTER(_u64)]),
+    "hq_file_write": (_i32, [ctypes.POINTER(hq_file_info), _vp, _vp, _vp, _vp, _vp, _u64]),
+    "hq_file_read": (_i32, [_vp, _u64, ctypes.POINTER(hq_file_info), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                            ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     "hq_decode_gemm": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
                               _u64, _vp, _vp]),
     "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
@@ -295,3 +306,62 @@ def hq_encode_noalloc(x, tile, lattice, bps, seed, out: Stream, status=None, str
     _check(_lib.hq_encode_noalloc(_ptr(x), _dtype_code(x), rows, cols, tile, _lat(lattice), bps, seed,
                                   ctypes.byref(s), _stream_handle(stream), _ptr(status)), "hq_encode_noalloc")
     return out
+
+
+# ----------------------------------------------------------------- files
+def stream_to_bytes(s: Stream, rows: int, cols: int, tile: int, lattice, bps: float, seed: int,
+                    dither: bool = False) -> bytes:
+    """The checkpoint container of a stream (its arrays are copied to the host)."""
+    off = s.tile_off.cpu().numpy().view(np.uint32)
+    words = int(off[-1])
+    scale = s.tile_scale.cpu().numpy().view(np.uint16)
+    kk = s.tile_k.cpu().numpy()
+    pay = s.payload[:words].cpu().numpy().view(np.uint32)
+    info = hq_file_info(rows, cols, tile, _lat(lattice), bps, 1 if dither else 0, seed, off.size - 1, words)
+    n = _u64(0)
+    _check(_lib.hq_file_bytes(ctypes.byref(info), ctypes.byref(n)), "hq_file_bytes")
+    buf = np.zeros(n.value, dtype=np.uint8)
+    _check(_lib.hq_file_write(ctypes.byref(info), off.ctypes.data, scale.ctypes.data if scale.size else None,
+                              kk.ctypes.data if kk.size else None, pay.ctypes.data if pay.size else None,
+                              buf.ctypes.data, buf.size), "hq_file_write")
+    return buf.tobytes()
+
+
+def stream_from_bytes(data: bytes, device="cuda") -> tuple[Stream, dict]:
+    """Check a container and return (device Stream, meta) with meta holding
+    rows, cols, tile, lattice, bps, seed and dither."""
+    buf = np.frombuffer(data, dtype=np.uint8)
+    info = hq_file_info()
+    ptrs = [_vp() for _ in range(4)]
+    _check(_lib.hq_file_read(buf.ctypes.data, buf.size, ctypes.byref(info), *[ctypes.byref(p) for p in ptrs]),
+           "hq_file_read")
+    base = buf.ctypes.data
+    n, words = int(info.ntiles), int(info.payload_words)
+
+    def view(p, dtype, count):
+        start = (p.value or base) - base
+        return np.frombuffer(data, dtype=dtype, count=count, offset=start).copy()
+
+    off = view(ptrs[0], np.uint32, n + 1)
+    scale = view(ptrs[1], np.uint16, n)
+    kk = view(ptrs[2], np.uint8, n)
+    pay = view(ptrs[3], np.uint32, words)
+    pay_t = torch.zeros(max(words, 1), dtype=torch.int32)
+    pay_t[:words] = torch.from_numpy(pay.view(np.int32))
+    stream = Stream(payload=pay_t.to(device), tile_off=torch.from_numpy(off.view(np.int32)).to(device),
+                    tile_scale=torch.from_numpy(scale.view(np.int16)).to(device),
+                    tile_k=torch.from_numpy(kk).to(device))
+    names = {v: k for k, v in LATTICES.items()}
+    meta = {"rows": int(info.rows), "cols": int(info.cols), "tile": int(info.tile), "lattice": names[info.lattice],
+            "bps": float(info.bps), "seed": int(info.seed), "dither": bool(info.flags & 1)}
+    return stream, meta
+
+
+def save_stream(path: str, s: Stream, rows, cols, tile, lattice, bps, seed, dither=False) -> None:
+    with open(path, "wb") as f:
+        f.write(stream_to_bytes(s, rows, cols, tile, lattice, bps, seed, dither))
+
+
+def load_stream(path: str, device="cuda") -> tuple[Stream, dict]:
+    with open(path, "rb") as f:
+        return stream_from_bytes(f.read(), device)

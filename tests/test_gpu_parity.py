@@ -213,3 +213,17 @@ def test_long_unary_codes(lat):
         w64, _ = oracle.decode(ref, rows, n, n, lat, seed)
         assert gst == 0
         assert_recon_close(out, w64, n, seed, False)
+
+
+def test_checkpoint_round_trip_on_gpu(tmp_path):
+    """GPU encode -> container file -> GPU decode gives the same matrix."""
+    x = make_input(33, 1024, 5)
+    s, st = gpu_encode(x, 256, "E8", 4.0, 11)
+    assert st == 0
+    path = str(tmp_path / "w.hqf")
+    hq.save_stream(path, s, 33, 1024, 256, "E8", 4.0, 11)
+    s2, meta = hq.load_stream(path, DEV)
+    assert meta["rows"] == 33 and meta["lattice"] == "E8" and not meta["dither"]
+    a, _ = gpu_decode(s, 33, 1024, 256, "E8", 4.0, 11)
+    b, _ = gpu_decode(s2, 33, 1024, 256, "E8", 4.0, 11)
+    assert np.array_equal(a, b)
