@@ -77,10 +77,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     }
 }
 
-template <int N, int D, int EPL>
-__global__ void __launch_bounds__(kDecodeWarps * 32) gemv_kernel(const DecodeArgs a)
+template <int N, int D, int EPL, int W>
+__global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(const DecodeArgs a)  // 64 registers up to 256
 {
-    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kDecodeWarps * TPW;
+    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = W * TPW;
     constexpr int SW = EPL / 4 - 1;
     extern __shared__ __align__(16) uint32_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) gemv_kernel(const DecodeArg
     }
     __syncthreads();
 
-    for (int64_t row = (int64_t)blockIdx.x * kDecodeWarps + warp; row < a.rows; row += (int64_t)gridDim.x * kDecodeWarps) {
+    for (int64_t row = (int64_t)blockIdx.x * W + warp; row < a.rows; row += (int64_t)gridDim.x * W) {
         float acc = 0.0f;
         for (int64_t j = lane / LPT; j < tpr; j += TPW) {
             const int64_t t = row * tpr + j;
@@ -202,17 +202,49 @@ cudaError_t launch_decode_n(int lattice, bool dither, int dtype, const DecodeArg
     }
 }
 
+// Blocks of W warps each hold the rotated x (cols floats) in shared memory;
+// when that copy is large, 16-warp blocks keep as many warps resident as
+// 8-warp blocks do with a small one.  Resident blocks per SM come from the
+// kernel's registers and shared memory and the device limits.
+template <int N, int D, int W>
+cudaError_t launch_gemv_w(const DecodeArgs &a, int64_t cols, cudaStream_t s)
+{
+    constexpr int EPL = epl_for<N>(), GPB = W * (32 / (N / EPL));
+    const size_t smem = (size_t)a.sign_words * 8 + (size_t)cols * 4 + (size_t)GPB * group_words(a.wmax) * 4;
+    auto kern = gemv_kernel<N, D, EPL, W>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa{};
+    int dev = 0, smem_sm = 0, reserved = 0, regs_sm = 0, thr_sm = 0;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess) return e;
+    const int threads = W * 32;
+    int per_sm = thr_sm / threads;
+    const int by_regs = regs_sm / (threads * (fa.numRegs > 0 ? fa.numRegs : 64));
+    const int by_smem = (int)((size_t)smem_sm / (smem + fa.sharedSizeBytes + (size_t)reserved));
+    if (by_regs < per_sm) per_sm = by_regs;
+    if (by_smem < per_sm) per_sm = by_smem;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int64_t blocks = (int64_t)sm_count() * per_sm, work = (a.rows + W - 1) / W;
+    if (blocks > work) blocks = work;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, threads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <int N, int D>
 cudaError_t launch_gemv_t(const DecodeArgs &a, int64_t cols, cudaStream_t s)
 {
-    constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
-    const size_t smem = (size_t)a.sign_words * 8 + (size_t)cols * 4 + (size_t)GPB * group_words(a.wmax) * 4;
-    auto kern = gemv_kernel<N, D, EPL>;
-    unsigned blocks = 0;
-    cudaError_t e = grid_for(kern, smem, (a.rows + kDecodeWarps - 1) / kDecodeWarps, blocks);
-    if (e != cudaSuccess) return e;
-    kern<<<blocks, kDecodeWarps * 32, smem, s>>>(a);
-    return cudaGetLastError();
+    // 32 coordinates per lane (tiles of 512, 1024) need more than 64
+    // registers, so those keep 8-warp blocks
+    if constexpr (N <= 256) {
+        if (cols * 4 > 32 * 1024) return launch_gemv_w<N, D, 16>(a, cols, s);
+    }
+    return launch_gemv_w<N, D, 8>(a, cols, s);
 }
 
 template <int N>
