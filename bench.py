@@ -342,8 +342,11 @@ def run_ours(args):
 
 
 def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier):
-    """Same step through the C ABI from pinned host memory: H2D of the seven
-    inputs, encode, decode, D2H of the seven decoded matrices, all timed."""
+    """Same work through the C ABI from pinned host memory: per matrix, H2D of
+    its input, encode, decode, D2H of the decoded matrix, all timed.  As a user
+    would drive the API, copies run on their own streams: the input of one
+    matrix crosses PCIe while another is encoded and a third is read back
+    (per-matrix events order the reuse of every buffer across steps)."""
     import torch
 
     from kv_quantization_tile_b200 import hq
@@ -351,15 +354,35 @@ def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barri
     host_in = [m["x"].cpu().pin_memory() for m in ctx]
     host_out = [torch.empty(m["shape"], dtype=torch.bfloat16).pin_memory() for m in ctx]
     dev_in = [torch.empty_like(m["x"]) for m in ctx]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    n = len(ctx)
+    loaded = [torch.cuda.Event() for _ in range(n)]   # input m on the device
+    encoded = [torch.cuda.Event() for _ in range(n)]  # input m consumed
+    decoded = [torch.cuda.Event() for _ in range(n)]  # output m ready
+    read = [torch.cuda.Event() for _ in range(n)]     # output m copied out
+    for e in encoded + read:
+        e.record(stream)
 
     def step():
-        for m, hi, di in zip(ctx, host_in, dev_in):
-            di.copy_(hi, non_blocking=True)
-            hq.hq_encode(di, TILE, LAT, BPS, SEED, m["s"], m["ws"], status)
-        for m, ho in zip(ctx, host_out):
+        for i, (m, hi, di) in enumerate(zip(ctx, host_in, dev_in)):
+            s_in.wait_event(encoded[i])
+            with torch.cuda.stream(s_in):
+                di.copy_(hi, non_blocking=True)
+            loaded[i].record(s_in)
+        for i, (m, di, ho) in enumerate(zip(ctx, dev_in, host_out)):
             r, c = m["shape"]
-            hq.hq_decode(m["s"], r, c, TILE, LAT, BPS, SEED, m["y"], status)
-            ho.copy_(m["y"], non_blocking=True)
+            stream.wait_event(loaded[i])
+            stream.wait_event(read[i])
+            with torch.cuda.stream(stream):
+                hq.hq_encode(di, TILE, LAT, BPS, SEED, m["s"], m["ws"], status, stream=stream)
+                encoded[i].record(stream)
+                hq.hq_decode(m["s"], r, c, TILE, LAT, BPS, SEED, m["y"], status, stream=stream)
+                decoded[i].record(stream)
+            s_out.wait_event(decoded[i])
+            with torch.cuda.stream(s_out):
+                ho.copy_(m["y"], non_blocking=True)
+            read[i].record(s_out)
+        stream.wait_stream(s_out)
 
     steps = max(3, min(args.steps, 5))
     step()
@@ -367,6 +390,7 @@ def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barri
     barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    s_in.wait_stream(stream)
     for _ in range(steps):
         step()
     b.record(stream)
@@ -374,7 +398,8 @@ def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barri
     ms = max_over_ranks(a.elapsed_time(b) / steps)
     nbytes = 2 * n_elem
     return {"value": round(world * 4 * n_elem / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+            "overlap": "H2D, compute and D2H on three streams, pipelined across the seven matrices"}
 
 
 def flush_l2(buf):
