@@ -351,6 +351,9 @@ def e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barri
 
     from kv_quantization_tile_b200 import hq
 
+    # a small matrix first and last: the pipeline fills and drains quickly
+    order = {"k": 0, "q": 1, "gate": 2, "up": 3, "down": 4, "o": 5, "v": 6}
+    ctx = sorted(ctx, key=lambda m: order.get(m["name"], 3))
     host_in = [m["x"].cpu().pin_memory() for m in ctx]
     host_out = [torch.empty(m["shape"], dtype=torch.bfloat16).pin_memory() for m in ctx]
     dev_in = [torch.empty_like(m["x"]) for m in ctx]
