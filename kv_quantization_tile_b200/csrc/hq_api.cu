@@ -1,6 +1,7 @@
 // hq_api.cu -- host side of the C ABI declared in include/hq.h: argument
 // validation, sizing rules, hash keys and kernel dispatch.  No allocation,
 // no synchronisation; everything is enqueued on the caller's stream.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,15 +16,15 @@ namespace hq {
 
 int sm_count()
 {
-    static int cached[64] = { 0 };
+    static std::atomic<int> cached[64];  // zero-initialised; a race only stores the same value twice
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 }  // namespace hq
