@@ -62,12 +62,6 @@ __device__ __forceinline__ void named_arrive(int id, int threads)
 // Decoupled look-back run by one whole warp: publish this chunk's aggregate,
 // then sum predecessors 32 at a time until an inclusive prefix is found.
 // Returns the exclusive prefix (same value in every lane).
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 
 __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, uint64_t agg, int lane,
                                         bool publish, bool &timed_out)

@@ -81,10 +81,13 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
 
-// Bounded wait for phase `parity` of an mbarrier; false if it gave up.
+// Bounded wait for phase `parity` of an mbarrier (2^24 polls or 0.5 s of
+// the global timer, whichever first); false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
 {
+    const uint64_t t0 = global_ns();
     for (uint32_t i = 0; i < kSpinLimit; i++) {
+        if ((i & 1023u) == 1023u && global_ns() - t0 > kWaitLimitNs) return false;
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"

@@ -18,6 +18,14 @@ constexpr uint64_t kValueMask = (1ull << 62) - 1;
 constexpr uint32_t kSpinLimit = 1u << 24;          // polls before a wait gives up ...
 constexpr uint64_t kWaitLimitNs = 500ull * 1000000;  // ... or 0.5 s of waiting, whichever first
 
+// Nanoseconds of the GPU's global timer (bounds every wait).
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 struct EncodeArgs {
     const void *x;
     int64_t ntiles;
