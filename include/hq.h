@@ -209,6 +209,16 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
                    uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
+/* Testing hook for failure detection (no counterpart on the pages):
+ * hq_decode_gemm in which column tile `stalled_tile` never issues or commits
+ * its tensor-core products, so the bounded wait for them runs out (0.5 s):
+ * the blocks that reach it raise HQ_ST_TIMEOUT, leave with no tensor-core
+ * work in flight, free their tensor memory and return; the output is
+ * invalid, the device stays usable.  Not for production use. */
+int hq_test_gemm_stalled(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                         uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                         uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stalled_tile);
+
 /* Bytes of device workspace hq_kv_attention needs: 256-byte-rounded
  * counters (heads * ceil(group / queries per block) uint32) followed by
  * heads * group * splits * (head_dim + 2) floats of per-split partial

@@ -339,9 +339,13 @@ int hq_decode_gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, ui
     return HQ_OK;
 }
 
-int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t seed,
-                   const void *x, int64_t batch, float *y, void *workspace, uint64_t workspace_bytes, void *stream,
-                   int32_t *d_status)
+}  // extern "C"
+
+namespace {
+
+int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                     uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                     uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stall_tile)
 {
     GemmArgs a{};
     int64_t ntiles = 0;
@@ -374,7 +378,28 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
     a.tiles_per_split = p.tiles_per_split;
     a.sign_key = hash_key(seed, 1);
     a.status = d_status;
+    a.stall_tile = stall_tile;
     return launch_gemm(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps, uint64_t seed,
+                   const void *x, int64_t batch, float *y, void *workspace, uint64_t workspace_bytes, void *stream,
+                   int32_t *d_status)
+{
+    return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
+                            d_status, -1);
+}
+
+int hq_test_gemm_stalled(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                         uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                         uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stalled_tile)
+{
+    return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
+                            d_status, stalled_tile);
 }
 
 int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim, int group, uint64_t *out)

@@ -233,9 +233,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         const int64_t j1 = j0 + a.tiles_per_split < a.tiles_per_row ? j0 + a.tiles_per_split : a.tiles_per_row;
         for (int64_t j = j0; j < j1; j++) {
             if (pending) {  // the previous MMAs have read A and B
-                if (!mbar_wait(bar, parity)) fail = true;
+                const bool ok = mbar_wait(bar, parity);
                 parity ^= 1u;
                 pending = false;
+                if (__syncthreads_or(!ok)) {  // every thread leaves together; nothing is in flight
+                    fail = true;
+                    break;
+                }
             }
             // A: rows r0 .. r0 + 127 of column tile j, lane l's chunks 2l and 2l + 1
             for (int m = gid; m < kGemmM; m += GPB) {
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
-            if (tid == 0) {
+            if (tid == 0 && j != a.stall_tile) {
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < N / 16; s++) {
@@ -283,9 +287,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
             pending = true;
         }
         if (pending) {
-            if (!mbar_wait(bar, parity)) fail = true;
+            const bool ok = mbar_wait(bar, parity);
             parity ^= 1u;
             pending = false;
+            if (__syncthreads_or(!ok)) fail = true;
         }
         tc_fence_after();
         // epilogue: warp w < 4 owns TMEM lanes (rows) 32 w .. 32 w + 31
@@ -309,6 +314,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         tc_fence_before();
         __syncthreads();  // the accumulator is read before the next item overwrites it
         tc_fence_after();
+        if (fail) break;  // block-uniform: stop after a wait that gave up
     }
     if (fail && tid == 0 && a.status) atomicOr(a.status, kStatusTimeout);
     if (warp == 0) tmem_dealloc(tmem, NCOLS);

@@ -98,6 +98,7 @@ struct GemmArgs {
     int ksplit, tiles_per_split;
     uint64_t sign_key;
     int32_t *status;
+    int64_t stall_tile;         // test hook: this column tile never commits its MMAs (-1: none)
 };
 
 struct GemmPlan {

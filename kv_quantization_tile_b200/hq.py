@@ -30,7 +30,7 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
            "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
-           "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read"]
+           "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled"]
 
 
 class hq_file_info(ctypes.Structure):
@@ -70,6 +70,8 @@ _SIGS = {
                                       _vp, _u64, _vp, _vp, ctypes.c_uint32]),
     "hq_kv_attention_workspace_bytes": (_i32, [_i64, _i64, _i32, _i32, ctypes.POINTER(_u64)]),
     "hq_decode_gemm_workspace_bytes": (_i32, [_i64, _i64, _i64, ctypes.POINTER(_u64)]),
+    "hq_test_gemm_stalled": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp,
+                                    _vp, _u64, _vp, _vp, _i64]),
     "hq_file_bytes": (_i32, [ctypes.POINTER(hq_file_info), ctypes.POINTER(_u64)]),
     "hq_file_write": (_i32, [ctypes.POINTER(hq_file_info), _vp, _vp, _vp, _vp, _vp, _u64]),
     "hq_file_read": (_i32, [_vp, _u64, ctypes.POINTER(hq_file_info), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
@@ -264,6 +266,18 @@ def hq_decode_gemm(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, worksp
     _check(_lib.hq_decode_gemm(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch, _ptr(y),
                                _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status)),
            "hq_decode_gemm")
+    return y
+
+
+def hq_test_gemm_stalled(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, workspace, stalled_tile: int,
+                         status=None, stream=None):
+    """hq_decode_gemm with one column tile's tensor-core work withheld (a
+    failure-detection test hook): the bounded wait runs out and HQ_ST_TIMEOUT
+    is raised."""
+    st = s.struct()
+    _check(_lib.hq_test_gemm_stalled(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), x.shape[0],
+                                     _ptr(y), _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status),
+                                     stalled_tile), "hq_test_gemm_stalled")
     return y
 
 

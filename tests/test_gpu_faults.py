@@ -43,3 +43,33 @@ def test_stalled_prefix_slot_times_out_and_device_stays_usable():
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert_streams_equal(fetch(s), oracle.encode(host_input(x), tile, "E8", 4.0, 42))
+
+
+def test_stalled_tensor_core_tile_times_out_and_device_stays_usable():
+    """The batched product waits (bounded) on an mbarrier for each column
+    tile's tensor-core products.  A testing hook withholds one tile's
+    products and commit: the blocks that wait for it give up after 0.5 s,
+    raise HQ_ST_TIMEOUT, free their tensor memory and return; a normal call
+    right after matches the oracle."""
+    from gpu_util import device_stream, gemm_tolerance
+    g = torch.Generator(device="cpu").manual_seed(5)
+    rows, cols = 256, 1024
+    w = (torch.randn(rows, cols, generator=g) * 0.02).to(torch.bfloat16)
+    ref = oracle.encode(host_input(w), 256, "E8", 4.0, 9)
+    s = device_stream(ref)
+    x = torch.randn(16, cols, generator=g).to(torch.bfloat16).to(DEV)
+    y = torch.empty(16, rows, dtype=torch.float32, device=DEV)
+    ws = hq.alloc_gemm_workspace(rows, cols, 16, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.time()
+    hq.hq_test_gemm_stalled(s, rows, cols, 256, "E8", 4.0, 9, x, y, ws, 1, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hq.HQ_ST_TIMEOUT
+    assert time.time() - t0 < 10.0
+    status.zero_()
+    hq.hq_decode_gemm(s, rows, cols, 256, "E8", 4.0, 9, x, y, ws, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    X = x.float().cpu().numpy().astype(np.float64)
+    want = oracle.gemm(ref, rows, cols, 256, "E8", 9, X)
+    assert np.all(np.abs(y.cpu().numpy() - want) <= gemm_tolerance(ref, rows, cols, "E8", 9, X))
