@@ -83,6 +83,17 @@ def lib() -> ctypes.CDLL:
                                            i64, vp]),
                 "hqo_gemv_rows": (i32, [vp, u64, vp, vp, vp, i64, i64, i32, i32, u64, vp, i64,
                                         i64, vp]),
+                "hqo_min_slot_words": (i32, [i32, i32]),
+                "hqo_fixed_slot_words": (i32, [i32, i32, f32]),
+                "hqo_fixed_start_rate": (f32, [i32, i32]),
+                "hqo_fixed_scale": (ctypes.c_uint16, [vp, i32, i32, ctypes.c_uint16, u64, u64, u64, i32,
+                                                      vp]),
+                "hqo_encode_tile_fixed": (i32, [vp, i32, i32, i32, u64, u64, u64, i32, vp, vp, vp, vp,
+                                                vp]),
+                "hqo_encode_tiles_fixed": (i32, [vp, i32, i64, i32, i32, i32, u64, i32, i64, i64, vp, vp,
+                                                 vp, vp]),
+                "hqo_decode_tiles_fixed": (i32, [vp, u64, i32, vp, vp, i64, i32, i32, u64, i32, i64, i64,
+                                                 vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -326,7 +337,10 @@ def encode(x, tile: int, lattice, bps: float, seed: int, dither: bool = False, t
 
 def decode(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int,
            dither: bool = False, threads: int = 1) -> tuple[np.ndarray, int]:
-    """binary64 decode of a whole stream; returns (out[rows, cols], status)."""
+    """binary64 decode of a whole stream; returns (out[rows, cols], status).
+    A fixed-rate stream (a dict with a "slot" entry) goes to decode_fixed."""
+    if "slot" in stream:
+        return decode_fixed(stream, rows, cols, tile, lattice, seed, dither, threads)
     d = _lat(lattice)
     ntiles = rows * (cols // tile)
     out = np.zeros((rows, cols), np.float64)
@@ -361,6 +375,16 @@ def gemv(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, x,
     """y[r] = sum_c w_hat[r, c] x[c] in binary64 for rows [r0, r1)."""
     d = _lat(lattice)
     r1 = rows if r1 is None else r1
+    if "slot" in stream:
+        W, st = decode_fixed(stream, rows, cols, tile, lattice, seed)
+        if st:
+            raise ValueError("corrupt stream")
+        return W[r0:r1] @ np.asarray(x, dtype=np.float64)
+    if "slot" in stream:
+        W, st = decode_fixed(stream, rows, cols, tile, lattice, seed)
+        if st:
+            raise ValueError("corrupt stream")
+        return W[r0:r1] @ np.asarray(x, dtype=np.float64)
     xa = np.ascontiguousarray(x, dtype=np.float64)
     y = np.zeros(max(r1 - r0, 1), np.float64)
     pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
@@ -406,3 +430,148 @@ def kv_attention(k_stream: dict, v_stream: dict, heads: int, tokens: int, head_d
         p = np.exp(s - s.max())
         out[qh] = (p / p.sum()) @ V[h * tokens:(h + 1) * tokens]
     return out
+
+
+# ---------------------------------------------------------------- fixed rate
+def min_slot_words(n: int, lattice) -> int:
+    """Smallest fixed-rate slot: the all-zero tile's words."""
+    return lib().hqo_min_slot_words(n, _lat(lattice))
+
+
+def fixed_slot_words(n: int, lattice, bps: float) -> int:
+    """Slot words for a total rate of bps bits per coordinate (20 bits of
+    side information per tile included); -1 below the minimum slot."""
+    return lib().hqo_fixed_slot_words(n, _lat(lattice), bps)
+
+
+def fixed_start_rate(n: int, slot_words: int) -> float:
+    return lib().hqo_fixed_start_rate(n, slot_words)
+
+
+def fixed_scale(v, lattice, c0: int, budget_bits: int, seed: int, t: int = 0, dither: bool = False):
+    """The fixed-rate scale search on a rotated tile v: (bf16 bits, trials)."""
+    va = np.ascontiguousarray(v, dtype=np.float32)
+    tr = ctypes.c_int(0)
+    sb = lib().hqo_fixed_scale(_p(va), va.size, _lat(lattice), c0, budget_bits, seed, t, int(dither),
+                               ctypes.byref(tr))
+    return int(sb), tr.value
+
+
+def coded_bits(v, lattice, scale_bits: int, seed: int = 0, t: int = 0, dither: bool = False) -> int:
+    """Coded size in bits of the rotated tile v at one scale, from the
+    variable-rate encoder's own steps (quantize, best k, pack length)."""
+    d = _lat(lattice)
+    va = np.ascontiguousarray(v, dtype=np.float32)
+    n = va.size
+    inv = np.float32(1.0) / np.float32(np.uint32(scale_bits << 16).view(np.float32))
+    z = np.zeros(n, np.int32)
+    cos = np.zeros(n // d, np.uint8)
+    for q in range(n // d):
+        x = va[q * d:(q + 1) * d] * inv
+        if dither:
+            x = (x + globals()["dither"](d, seed, t, q)).astype(np.float32)
+        cos[q], z[q * d:(q + 1) * d], _ = nearest(d, x)
+    u = np.concatenate([symbols(d, z[q * d:(q + 1) * d]) for q in range(n // d)])
+    k = best_k(u)
+    return (n // d if d in (2, 8) else 0) + rice_cost(u, k)
+
+
+def encode_tile_fixed(w, lattice, slot_words: int, seed: int, j: int = 0, t: int = 0, dither: bool = False):
+    """One fixed-rate tile: dict(scale, k, slot (all slot_words words), words
+    (the tile's own count), trials, status)."""
+    d = _lat(lattice)
+    wa = np.ascontiguousarray(w, dtype=np.float32)
+    slot = np.zeros(max(slot_words, 1), np.uint32)
+    sc = ctypes.c_uint16(0)
+    kk = ctypes.c_uint8(0)
+    tr = ctypes.c_int(0)
+    st = ctypes.c_int(0)
+    nw = lib().hqo_encode_tile_fixed(_p(wa), wa.size, d, slot_words, seed, j, t, int(dither), ctypes.byref(sc),
+                                     ctypes.byref(kk), _p(slot), ctypes.byref(tr), ctypes.byref(st))
+    if nw < 0:
+        raise ValueError("slot below the minimum")
+    return {"scale": int(sc.value), "k": int(kk.value), "slot": slot[:slot_words], "words": nw,
+            "trials": tr.value, "status": st.value}
+
+
+def pack_k(k) -> np.ndarray:
+    """Rice parameters two per byte: tile t in bits 4 (t mod 2) .. +3 of byte t // 2."""
+    ka = np.asarray(k, dtype=np.uint8)
+    out = np.zeros((ka.size + 1) // 2, np.uint8)
+    out[:] = ka[0::2] & 15
+    out[: ka[1::2].size] |= (ka[1::2] & 15) << 4
+    return out
+
+
+def unpack_k(kpack, ntiles: int) -> np.ndarray:
+    kp = np.asarray(kpack, dtype=np.uint8)
+    t = np.arange(ntiles)
+    return ((kp[t >> 1] >> (4 * (t & 1))) & 15).astype(np.uint8)
+
+
+def _encode_tiles_fixed(x, tile, lattice, slot_words, seed, dither, t0, t1):
+    xa, dt = _as_bits(x)
+    nt = t1 - t0
+    slots = np.zeros(max(nt, 1) * slot_words, np.uint32)
+    sc = np.zeros(max(nt, 1), np.uint16)
+    kk = np.zeros(max(nt, 1), np.uint8)
+    tr = np.zeros(max(nt, 1), np.int32)
+    st = lib().hqo_encode_tiles_fixed(_p(xa), dt, xa.shape[1], tile, _lat(lattice), slot_words, seed,
+                                      int(dither), t0, t1, _p(slots), _p(sc), _p(kk), _p(tr))
+    if st < 0:
+        raise ValueError("slot below the minimum")
+    return slots[: nt * slot_words], sc[:nt], kk[:nt], tr[:nt], st
+
+
+def encode_fixed(x, tile: int, lattice, slot_words: int, seed: int, dither: bool = False,
+                 threads: int = 1) -> dict:
+    """Fixed-rate encode of a whole matrix.  Returns dict(payload (ntiles *
+    slot words), scale, k, kpack, trials, status, slot)."""
+    rows, cols = x.shape
+    assert cols % tile == 0
+    ntiles = rows * (cols // tile)
+    ranges = _ranges(ntiles, threads * 4)
+    if threads > 1 and len(ranges) > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            parts = list(ex.map(lambda r: _encode_tiles_fixed(x, tile, lattice, slot_words, seed, dither, *r),
+                                ranges))
+    else:
+        parts = [_encode_tiles_fixed(x, tile, lattice, slot_words, seed, dither, *r) for r in ranges]
+    cat = (lambda i, dt: np.concatenate([p[i] for p in parts]) if parts else np.zeros(0, dt))
+    status = 0
+    for p in parts:
+        status |= p[4]
+    k = cat(2, np.uint8)
+    return {"payload": cat(0, np.uint32), "scale": cat(1, np.uint16), "k": k, "kpack": pack_k(k),
+            "trials": cat(3, np.int32), "status": status, "slot": slot_words}
+
+
+def decode_fixed(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, dither: bool = False,
+                 threads: int = 1) -> tuple[np.ndarray, int]:
+    """binary64 decode of a fixed-rate stream; k is read from its packed form."""
+    d = _lat(lattice)
+    ntiles = rows * (cols // tile)
+    out = np.zeros((rows, cols), np.float64)
+    pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
+    cap = pay.size
+    if pay.size == 0:
+        pay = np.zeros(1, np.uint32)
+    sc = np.ascontiguousarray(stream["scale"], dtype=np.uint16)
+    kk = np.ascontiguousarray(unpack_k(stream["kpack"], ntiles))
+    S = int(stream["slot"])
+    L = lib()
+
+    def run(r):
+        return L.hqo_decode_tiles_fixed(_p(pay), cap, S, _p(sc) if sc.size else 0, _p(kk) if kk.size else 0,
+                                        cols, tile, d, seed, int(dither), r[0], r[1], _p(out))
+
+    ranges = _ranges(ntiles, threads * 4)
+    if threads > 1 and len(ranges) > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            sts = list(ex.map(run, ranges))
+    else:
+        sts = [run(r) for r in ranges]
+    st = 0
+    for x in sts:
+        st |= x
+    return out, st

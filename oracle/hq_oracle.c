@@ -416,10 +416,11 @@ int hqo_pack_tile(int lattice, int n, int k, const uint8_t *coset, const uint32_
 }
 
 /* Parse one tile; 0 on success, HQO_CORRUPT if the words do not hold a
- * canonical tile (a read past the end, a one bit in the padding, or a word
- * count other than ceil(bits / 32)). */
-int hqo_unpack_tile(int lattice, int n, int k, const uint32_t *words, int nwords,
-                    uint8_t *coset, uint32_t *u)
+ * canonical tile (a read past the end, a one bit in the padding, or -- when
+ * `exact` -- a word count other than ceil(bits / 32); a fixed-rate slot may
+ * end in whole words of zero padding). */
+static int unpack_words(int lattice, int n, int k, const uint32_t *words, int nwords,
+                        uint8_t *coset, uint32_t *u, int exact)
 {
     uint64_t end = (uint64_t)nwords * 32u, pos = 0;
     int d = lattice;
@@ -453,33 +454,24 @@ int hqo_unpack_tile(int lattice, int n, int k, const uint32_t *words, int nwords
     }
     for (uint64_t p = pos; p < end; p++)
         if (get_bit(words, p)) return HQO_CORRUPT;
-    if ((pos + 31) / 32 != (uint64_t)nwords) return HQO_CORRUPT;
+    if (exact && (pos + 31) / 32 != (uint64_t)nwords) return HQO_CORRUPT;
     return 0;
 }
 
-/* ------------------------------------------------------------------ */
-/* One tile, end to end [V1 (i)-(iv), V2].
- * w: n binary32 inputs (bf16 inputs are widened exactly by the caller).
- * j: column tile (signs), t: tile index (dither).  Outputs the bf16 bits of
- * Delta, k, the words, and optionally the pre-strip integer coordinates
- * z[n] and coset bits c[n/d].  Returns the word count, -1 if cap_words is
- * too small.  *status gets HQO_NONFINITE for a non-finite tile. */
-int hqo_encode_tile(const float *w, int n, int lattice, float bps, uint64_t seed,
-                    uint64_t j, uint64_t t, int dither, uint16_t *scale_out, uint8_t *k_out,
-                    uint32_t *words, int cap_words, int32_t *z_out, uint8_t *c_out, int *status)
+int hqo_unpack_tile(int lattice, int n, int k, const uint32_t *words, int nwords,
+                    uint8_t *coset, uint32_t *u)
 {
-    float v[HQO_MAX_TILE];
-    int32_t z[HQO_MAX_TILE];
-    uint32_t u[HQO_MAX_TILE];
-    uint8_t coset[HQO_MAX_TILE];
-    int d = lattice, nv = n / lattice, nonfinite = 0;
+    return unpack_words(lattice, n, k, words, nwords, coset, u, 1);
+}
 
-    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * w[i];
-    hqo_fwht_f32(v, n);
-    float S = hqo_sumsq(w, n);
-    uint16_t sb = hqo_tile_scale(S, hqo_rate_constant(lattice, bps), &nonfinite);
-    if (nonfinite) *status |= HQO_NONFINITE;
-
+/* ------------------------------------------------------------------ */
+/* Quantize the rotated tile v at the scale with bf16 bits sb (0: all-zero
+ * tile): y = Q(v / Delta [+ delta]) per vector, then the strip and zigzag of
+ * its integer coordinates into the symbols u. */
+static void quantize_tile(const float *v, int n, int lattice, uint16_t sb, uint64_t seed, uint64_t t,
+                          int dither, int32_t *z, uint8_t *coset, uint32_t *u)
+{
+    int d = lattice, nv = n / lattice;
     if (sb == 0) {
         for (int i = 0; i < n; i++) z[i] = 0;
         for (int q = 0; q < nv; q++) coset[q] = 0;
@@ -498,6 +490,31 @@ int hqo_encode_tile(const float *w, int n, int lattice, float bps, uint64_t seed
         }
     }
     for (int q = 0; q < nv; q++) hqo_symbols(lattice, &z[q * d], &u[q * d]);
+}
+
+/* One tile, end to end [V1 (i)-(iv), V2].
+ * w: n binary32 inputs (bf16 inputs are widened exactly by the caller).
+ * j: column tile (signs), t: tile index (dither).  Outputs the bf16 bits of
+ * Delta, k, the words, and optionally the pre-strip integer coordinates
+ * z[n] and coset bits c[n/d].  Returns the word count, -1 if cap_words is
+ * too small.  *status gets HQO_NONFINITE for a non-finite tile. */
+int hqo_encode_tile(const float *w, int n, int lattice, float bps, uint64_t seed,
+                    uint64_t j, uint64_t t, int dither, uint16_t *scale_out, uint8_t *k_out,
+                    uint32_t *words, int cap_words, int32_t *z_out, uint8_t *c_out, int *status)
+{
+    float v[HQO_MAX_TILE];
+    int32_t z[HQO_MAX_TILE];
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    int nv = n / lattice, nonfinite = 0;
+
+    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * w[i];
+    hqo_fwht_f32(v, n);
+    float S = hqo_sumsq(w, n);
+    uint16_t sb = hqo_tile_scale(S, hqo_rate_constant(lattice, bps), &nonfinite);
+    if (nonfinite) *status |= HQO_NONFINITE;
+
+    quantize_tile(v, n, lattice, sb, seed, t, dither, z, coset, u);
     int k = hqo_best_k(u, n);
     *scale_out = sb;
     *k_out = (uint8_t)k;
@@ -508,16 +525,17 @@ int hqo_encode_tile(const float *w, int n, int lattice, float bps, uint64_t seed
 
 /* Decode one tile into binary64 (before any output rounding):
  * w_hat = s . H(Delta (p - delta)) / n with p the lattice point.
- * Returns 0 or HQO_CORRUPT (output zeroed). */
-int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint16_t scale,
-                    int k, uint64_t seed, uint64_t j, uint64_t t, int dither, double *out)
+ * Returns 0 or HQO_CORRUPT (output zeroed).  `exact`: the words are the
+ * tile's own (variable-rate stream); else a fixed-rate slot. */
+static int decode_words(const uint32_t *words, int nwords, int n, int lattice, uint16_t scale,
+                        int k, uint64_t seed, uint64_t j, uint64_t t, int dither, double *out, int exact)
 {
     uint32_t u[HQO_MAX_TILE];
     uint8_t coset[HQO_MAX_TILE];
     int32_t z[8];
     double v[HQO_MAX_TILE];
     int d = lattice, nv = n / lattice;
-    int st = hqo_unpack_tile(lattice, n, k, words, nwords, coset, u);
+    int st = unpack_words(lattice, n, k, words, nwords, coset, u, exact);
     /* the encoder only writes Delta = 0 or a positive, normal, finite bf16 */
     if (scale != 0 && ((scale & 0x8000u) || (scale & 0x7F80u) == 0 || (scale & 0x7F80u) == 0x7F80u))
         st = HQO_CORRUPT;
@@ -545,6 +563,217 @@ int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint1
     hqo_fwht_f64(v, n);
     for (int i = 0; i < n; i++) out[i] = (double)hqo_sign(seed, j, (uint32_t)i) * v[i] / (double)n;
     return 0;
+}
+
+int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint16_t scale,
+                    int k, uint64_t seed, uint64_t j, uint64_t t, int dither, double *out)
+{
+    return decode_words(words, nwords, n, lattice, scale, k, seed, j, t, dither, out, 1);
+}
+
+/* ------------------------------------------------------------------ */
+/* Fixed-rate tiles: compact headers and exact rate control.  The pages
+ * quote whole-model ratios that count every bit spent (about 3.9x for the
+ * weights, 3.79x for the KV cache at 4 bps: [V1] abstract "End-to-end ...
+ * compresses"), and name the per-tile scale as the rate's control.  Reading:
+ * every tile gets a slot of S words; its tile offset is then t S and is not
+ * stored, k is stored in 4 bits, so a tile's side information is the bf16
+ * Delta and k (20 bits).  Delta is searched so that the coded tile fits its
+ * slot, which makes the rate exact: (32 S + 20) / n bits per coordinate.
+ * The slot holds the same tile layout as a variable-rate tile, followed by
+ * zero words up to S.
+ *
+ * Coded size at the scale with bf16 bits c: C + n (1 + k) + sum(u >> k)
+ * with u the tile's symbols at that scale and k their best Rice parameter
+ * (C = coset bits).  A scale fits if that size is at most 32 S bits.
+ *
+ * Search (bf16 bit patterns of positive normal numbers are ordered like the
+ * numbers; 128 patterns per octave).  c0 = the closed-form scale at the
+ * slot's rate.  Bounds: lo_lim = max(0x0080, c0 - 512), hi_lim = min(0x7F7F,
+ * c0 + 512) (four octaves either way).
+ *   c0 fits:  step down from c0 by 4, 8, 16, ... (clamped at lo_lim)
+ *             while the candidate fits; the first that does not becomes lo
+ *             (the last that fits is hi).  If lo_lim itself fits, the answer
+ *             is lo_lim.
+ *   otherwise: step up likewise from c0 (clamped at hi_lim) until a
+ *             candidate fits (hi; the last that did not is lo).  If hi_lim
+ *             does not fit, the tile is stored as an all-zero tile
+ *             (Delta = 0), which always fits a legal slot.
+ *   Then bisect: while hi - lo > 1, mid = floor((lo + hi) / 2) replaces hi
+ *   if it fits, else lo.  The answer is hi: a fitting scale whose next
+ *   smaller bf16 value does not fit (when the search ended by bisection).
+ * A tile whose closed-form scale is 0 (non-finite, zero or negligible
+ * energy) is the all-zero tile, as in the variable-rate stream. */
+
+/* smallest legal slot: the all-zero tile (k = 0, n one bits, C coset bits) */
+int hqo_min_slot_words(int n, int lattice)
+{
+    int c = (lattice == 8 || lattice == 2) ? n / lattice : 0;
+    return (c + n + 31) / 32;
+}
+
+/* slot for a total rate of `bps` bits per coordinate including the 20 bits
+ * of side information: floor((bps n - 20) / 32), or -1 below the minimum */
+int hqo_fixed_slot_words(int n, int lattice, float bps)
+{
+    double s = floor(((double)bps * (double)n - 20.0) / 32.0);
+    if (s < (double)hqo_min_slot_words(n, lattice)) return -1;
+    return (int)s;
+}
+
+static uint64_t coded_bits(const float *v, int n, int lattice, uint16_t c, uint64_t seed, uint64_t t,
+                           int dither)
+{
+    int32_t z[HQO_MAX_TILE];
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    quantize_tile(v, n, lattice, c, seed, t, dither, z, coset, u);
+    uint64_t cb = (lattice == 8 || lattice == 2) ? (uint64_t)(n / lattice) : 0;
+    return cb + hqo_rice_cost(u, n, hqo_best_k(u, n));
+}
+
+/* The fixed-rate scale search above; *trials counts the sizes evaluated. */
+uint16_t hqo_fixed_scale(const float *v, int n, int lattice, uint16_t c0, uint64_t budget_bits,
+                         uint64_t seed, uint64_t t, int dither, int *trials)
+{
+    int tr = 0;
+    if (c0 == 0) {
+        if (trials) *trials = 0;
+        return 0;
+    }
+    int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
+    int hi_lim = (int)c0 + 512 < 0x7F7F ? (int)c0 + 512 : 0x7F7F;
+    int lo, hi, step = 4;
+    tr++;
+    if (coded_bits(v, n, lattice, c0, seed, t, dither) <= budget_bits) {
+        hi = c0;
+        for (;;) {
+            if (hi == lo_lim) {
+                if (trials) *trials = tr;
+                return (uint16_t)hi;
+            }
+            int cand = hi - step > lo_lim ? hi - step : lo_lim;
+            tr++;
+            if (coded_bits(v, n, lattice, (uint16_t)cand, seed, t, dither) <= budget_bits) {
+                hi = cand;
+                step *= 2;
+            } else {
+                lo = cand;
+                break;
+            }
+        }
+    } else {
+        lo = c0;
+        for (;;) {
+            if (lo == hi_lim) {
+                if (trials) *trials = tr;
+                return 0;
+            }
+            int cand = lo + step < hi_lim ? lo + step : hi_lim;
+            tr++;
+            if (coded_bits(v, n, lattice, (uint16_t)cand, seed, t, dither) <= budget_bits) {
+                hi = cand;
+                break;
+            }
+            lo = cand;
+            step *= 2;
+        }
+    }
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        tr++;
+        if (coded_bits(v, n, lattice, (uint16_t)mid, seed, t, dither) <= budget_bits) hi = mid;
+        else lo = mid;
+    }
+    if (trials) *trials = tr;
+    return (uint16_t)hi;
+}
+
+/* Closed-form start of the search: the scale rule at the slot's payload
+ * rate 32 S / n less 5/32 bit (about what the Rice code and the coset bits
+ * spend over the closed form's entropy on Gaussian tiles, so the search
+ * starts a few bf16 steps from its answer), at most 8 bits per coordinate.
+ * The start only steers the search; every answer fits the slot. */
+float hqo_fixed_start_rate(int n, int slot_words)
+{
+    double r = 32.0 * (double)slot_words / (double)n - 0.15625;
+    return (float)(r < 8.0 ? r : 8.0);
+}
+
+/* One fixed-rate tile: fills all slot_words words of `slot` (the tile, then
+ * zeros).  Returns the tile's own word count, -1 if the slot is below the
+ * minimum.  *status gets HQO_NONFINITE for a non-finite tile. */
+int hqo_encode_tile_fixed(const float *w, int n, int lattice, int slot_words, uint64_t seed, uint64_t j,
+                          uint64_t t, int dither, uint16_t *scale_out, uint8_t *k_out, uint32_t *slot,
+                          int *trials, int *status)
+{
+    float v[HQO_MAX_TILE];
+    int32_t z[HQO_MAX_TILE];
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    int nonfinite = 0;
+    if (slot_words < hqo_min_slot_words(n, lattice)) return -1;
+
+    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * w[i];
+    hqo_fwht_f32(v, n);
+    float S = hqo_sumsq(w, n);
+    float c = hqo_rate_constant(lattice, hqo_fixed_start_rate(n, slot_words));
+    uint16_t c0 = hqo_tile_scale(S, c, &nonfinite);
+    if (nonfinite) *status |= HQO_NONFINITE;
+    uint16_t sb = hqo_fixed_scale(v, n, lattice, c0, 32u * (uint64_t)slot_words, seed, t, dither, trials);
+
+    quantize_tile(v, n, lattice, sb, seed, t, dither, z, coset, u);
+    int k = hqo_best_k(u, n);
+    *scale_out = sb;
+    *k_out = (uint8_t)k;
+    return hqo_pack_tile(lattice, n, k, coset, u, slot, slot_words);
+}
+
+/* Tiles [t0, t1) of a matrix (as in hqo_encode_tiles) into consecutive
+ * slots; trials[t - t0] gets each tile's search length. */
+int hqo_encode_tiles_fixed(const void *x, int dtype, int64_t cols, int n, int lattice, int slot_words,
+                           uint64_t seed, int dither, int64_t t0, int64_t t1, uint32_t *slots,
+                           uint16_t *scale, uint8_t *kk, int32_t *trials)
+{
+    float w[HQO_MAX_TILE];
+    int64_t tpr = cols / n;
+    int status = 0;
+    for (int64_t t = t0; t < t1; t++) {
+        int64_t r = t / tpr, j = t % tpr;
+        int64_t base = r * cols + j * n;
+        for (int i = 0; i < n; i++) {
+            if (dtype == 0) w[i] = bf16_to_float(((const uint16_t *)x)[base + i]);
+            else w[i] = ((const float *)x)[base + i];
+        }
+        int tr = 0;
+        int nw = hqo_encode_tile_fixed(w, n, lattice, slot_words, seed, (uint64_t)j, (uint64_t)t, dither,
+                                       &scale[t - t0], &kk[t - t0], slots + (t - t0) * (int64_t)slot_words,
+                                       &tr, &status);
+        if (nw < 0) return -1;
+        trials[t - t0] = tr;
+    }
+    return status;
+}
+
+/* Decode tiles [t0, t1) of a fixed-rate stream: tile t is words
+ * [t S, t S + S) of the payload (cap words), k[t] unpacked by the caller. */
+int hqo_decode_tiles_fixed(const uint32_t *payload, uint64_t cap, int slot_words, const uint16_t *scale,
+                           const uint8_t *kk, int64_t cols, int n, int lattice, uint64_t seed, int dither,
+                           int64_t t0, int64_t t1, double *out)
+{
+    int64_t tpr = cols / n;
+    int status = 0;
+    for (int64_t t = t0; t < t1; t++) {
+        int64_t r = t / tpr, j = t % tpr;
+        if ((uint64_t)(t + 1) * (uint64_t)slot_words > cap) {
+            for (int i = 0; i < n; i++) out[r * cols + j * n + i] = 0.0;
+            status |= HQO_CORRUPT;
+            continue;
+        }
+        status |= decode_words(payload + t * (int64_t)slot_words, slot_words, n, lattice, scale[t], kk[t], seed,
+                               (uint64_t)j, (uint64_t)t, dither, out + r * cols + j * n, 0);
+    }
+    return status;
 }
 
 /* ------------------------------------------------------------------ */
