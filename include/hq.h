@@ -83,15 +83,23 @@ enum {
 enum { HQ_ST_NONFINITE = 1, HQ_ST_CAPACITY = 2, HQ_ST_CORRUPT = 4, HQ_ST_TIMEOUT = 8 };
 
 /* A compressed matrix.  Host struct; all pointers are device memory owned by
- * the caller.  Sizes: payload >= hq_max_payload_words(...) words for encode
- * (the exact count is tile_off[ntiles] afterwards), tile_off ntiles + 1,
- * tile_scale ntiles, tile_k ntiles. */
+ * the caller.
+ * Variable rate (slot_words = 0): payload >= hq_max_payload_words(...) words
+ * for encode (the exact count is tile_off[ntiles] afterwards), tile_off
+ * ntiles + 1, tile_scale ntiles, tile_k ntiles.
+ * Fixed rate (slot_words = S > 0, written by hq_encode_fixed /
+ * hq_kv_encode_fixed): tile t occupies payload words [t S, t S + S) (the
+ * tile layout above, then zero words), payload >= ntiles S words, tile_off
+ * is not used (may be NULL), tile_scale ntiles, tile_k (ntiles + 1) / 2
+ * bytes holding k of tile t in bits 4 (t mod 2) .. 4 (t mod 2) + 3 of byte
+ * t / 2.  Every decoder below accepts either kind. */
 typedef struct hq_stream {
     uint32_t *payload;
     uint64_t payload_capacity_words;
     uint32_t *tile_off;
     uint16_t *tile_scale;
     uint8_t *tile_k;
+    uint32_t slot_words;
 } hq_stream;
 
 /* Static description of a return code (never NULL). */
@@ -151,14 +159,54 @@ int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile,
                  float bps, uint64_t seed, const hq_stream *out, void *workspace,
                  uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
+/* ------------------------------------------------------------------
+ * Fixed rate: compact headers and exact rate control.  The pages quote
+ * whole-model compression ratios that count every stored bit (about 3.9x
+ * for the weights and 3.79x for the KV cache at 4 bps, [V1] abstract) and
+ * name the per-tile scale as the control of the rate.  Reading: each tile
+ * gets a slot of S words, so its offset t S is implicit, k is kept in 4
+ * bits, and the tile's only side information is the bf16 Delta and k (20
+ * bits): (32 S + 20) / n bits per coordinate, exactly.  Delta is searched
+ * per tile so the coded tile fits its slot: from the closed-form scale at
+ * the rate 32 S / n - 5/32, steps of 4, 8, 16, ... bf16 patterns towards the
+ * boundary (at most four octaves either way), then bisection, ending at a
+ * fitting Delta whose next finer bf16 value does not fit.  A tile that fits
+ * at no scale of that range (possible only with dither at very small slots)
+ * is stored as the all-zero tile. */
+
+/* Smallest slot: the all-zero tile, (n/d coset bits (E8, A2) + n) / 32
+ * rounded up.  Host only. */
+int hq_min_slot_words(int tile, int lattice, uint32_t *out);
+
+/* Slot for a total rate of `bps` bits per coordinate, side information
+ * included: floor((bps n - 20) / 32).  HQ_ERR_ARG if that is below
+ * hq_min_slot_words or an argument is invalid.  Host only. */
+int hq_fixed_slot_words(int tile, int lattice, float bps, uint32_t *out);
+
+/* Fixed-rate encode.  Arguments as hq_encode except:
+ *   out        out->slot_words = S with hq_min_slot_words <= S <= n / 4;
+ *              payload_capacity_words >= ntiles S (< 2^32); tile_off unused
+ * No workspace: tiles are independent.  Every tile's slot is written whole
+ * (zero words after the tile), tile_scale[t] and the packed k. */
+int hq_encode_fixed(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+                    uint64_t seed, const hq_stream *out, void *stream, int32_t *d_status);
+
+/* Fixed-rate KV-cache encode: as hq_encode_fixed with the subtractive
+ * dither of hq_kv_encode; decode with hq_kv_decode or hq_kv_attention. */
+int hq_kv_encode_fixed(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice,
+                       uint64_t seed, const hq_stream *out, void *stream, int32_t *d_status);
+
 /* Decode ([V2] algebraic decoding): y = s . H (Delta y_lattice) / n per tile,
  * rounded to `dtype` (bf16 round-to-nearest-even, or fp32).
  *   in         stream written by hq_encode with the same shape, tile,
- *              lattice, bps and seed
+ *              lattice, bps and seed, or by hq_encode_fixed with the same
+ *              shape, tile, lattice and seed (bps must still be valid; the
+ *              slot sets the rate)
  *   y          device, rows x cols, 16-byte aligned
  * A tile whose words are not a canonical tile (bad offsets, k > 15, wrong
  * symbol count, a set padding bit) is written as zeros and HQ_ST_CORRUPT is
- * raised; no read leaves [tile_off[t], tile_off[t+1]) or the capacity. */
+ * raised; no read leaves [tile_off[t], tile_off[t+1]) (the slot, for a
+ * fixed-rate stream) or the capacity. */
 int hq_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
               uint64_t seed, void *y, int dtype, void *stream, int32_t *d_status);
 

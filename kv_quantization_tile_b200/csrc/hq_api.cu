@@ -85,8 +85,41 @@ A2Consts a2_consts() { return A2Consts{ (float)std::sqrt(3.0), (float)(1.0 / std
 int check_stream(const hq_stream *s, int64_t ntiles, bool need_payload)
 {
     if (!s) return HQ_ERR_ARG;
-    if (!s->tile_off) return HQ_ERR_ARG;
+    if (!s->slot_words && !s->tile_off) return HQ_ERR_ARG;  // fixed-rate streams keep no offsets
     if (ntiles > 0 && (!s->tile_scale || !s->tile_k || (need_payload && !s->payload))) return HQ_ERR_ARG;
+    return HQ_OK;
+}
+
+// Fixed-rate slots.  The smallest holds the all-zero tile (coset bits and n
+// one bits); the largest allowed is 8 bits per coordinate.
+uint32_t min_slot_words(int tile, int lattice)
+{
+    const uint32_t coset = (lattice == HQ_E8 || lattice == HQ_A2) ? (uint32_t)(tile / lattice) : 0u;
+    return (coset + (uint32_t)tile + 31u) / 32u;
+}
+
+bool valid_slot(int tile, int lattice, uint32_t slot)
+{
+    return slot >= min_slot_words(tile, lattice) && slot <= (uint32_t)tile / 4u;
+}
+
+// Start of the fixed-rate scale search: the closed-form rule at the slot's
+// payload rate less 5/32 bit (about what the Rice code and the coset bits
+// spend over the rule's entropy on Gaussian tiles), at most 8 bits.
+float fixed_start_rate(int tile, uint32_t slot)
+{
+    const double r = 32.0 * (double)slot / (double)tile - 0.15625;
+    return (float)(r < 8.0 ? r : 8.0);
+}
+
+// Fixed-rate stream of `ntiles` tiles: slot legal, every slot inside the
+// payload, offsets t * slot within 32 bits.
+int check_fixed_stream(const hq_stream *s, int64_t ntiles, int tile, int lattice)
+{
+    if (!valid_slot(tile, lattice, s->slot_words)) return HQ_ERR_ARG;
+    const uint64_t need = (uint64_t)ntiles * s->slot_words;
+    if (need >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
+    if (s->payload_capacity_words < need) return HQ_ERR_CAPACITY;
     return HQ_OK;
 }
 
@@ -116,6 +149,7 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     if (rc) return rc;
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     if ((rc = check_stream(out, ntiles, true))) return rc;
+    if (out->slot_words) return HQ_ERR_ARG;  // a fixed-rate stream: hq_encode_fixed
     cudaStream_t s = (cudaStream_t)stream;
     if (ntiles == 0) return cudaMemsetAsync(out->tile_off, 0, sizeof(uint32_t), s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
@@ -158,12 +192,49 @@ int encode_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, 
     return launch_encode(tile, lattice, dither, dtype, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
+int encode_fixed_impl(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, uint64_t seed,
+                      const hq_stream *out, void *stream, int32_t *d_status, bool dither)
+{
+    int64_t ntiles = 0;
+    int rc = common_shape(rows, cols, tile, lattice, 1.0f, &ntiles);
+    if (rc) return rc;
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (!out || !out->slot_words) return HQ_ERR_ARG;
+    if ((rc = check_stream(out, ntiles, true))) return rc;
+    if ((rc = check_fixed_stream(out, ntiles, tile, lattice))) return rc;
+    if (ntiles == 0) return HQ_OK;
+    if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
+    EncodeArgs a{};
+    a.x = x;
+    a.ntiles = ntiles;
+    a.tiles_per_row = cols / tile;
+    a.c = rate_constant(lattice, fixed_start_rate(tile, out->slot_words));
+    a.a2 = a2_consts();
+    a.sign_key = hash_key(seed, 1);
+    a.dither_key = hash_key(seed, 2);
+    a.payload = out->payload;
+    a.cap = out->payload_capacity_words;
+    a.scale = out->tile_scale;
+    a.kk = out->tile_k;
+    a.status = d_status;
+    a.wmax = out->slot_words;
+    const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
+    a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
+    a.k_hint = rice_hint(a.c);
+    a.tpr_div = make_fastdiv((uint32_t)(cols / tile));
+    a.stall_chunk = 0xffffffffu;
+    a.slot_words = out->slot_words;
+    return launch_encode_fixed(tile, lattice, dither, dtype, a, (cudaStream_t)stream) == cudaSuccess ? HQ_OK
+                                                                                                     : HQ_ERR_CUDA;
+}
+
 int decode_common(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                   uint64_t seed, DecodeArgs &a, int64_t *ntiles)
 {
     int rc = common_shape(rows, cols, tile, lattice, bps, ntiles);
     if (rc) return rc;
     if ((rc = check_stream(in, *ntiles, true))) return rc;
+    if (in->slot_words && (rc = check_fixed_stream(in, *ntiles, tile, lattice))) return rc;
     a.payload = in->payload;
     a.cap = in->payload_capacity_words;
     a.off = in->tile_off;
@@ -174,7 +245,8 @@ int decode_common(const hq_stream *in, int64_t rows, int64_t cols, int tile, int
     a.a2 = a2_consts();
     a.sign_key = hash_key(seed, 1);
     a.dither_key = hash_key(seed, 2);
-    a.wmax = tile_bound_words(tile, lattice, bps);
+    a.wmax = in->slot_words ? in->slot_words : tile_bound_words(tile, lattice, bps);
+    a.slot = in->slot_words;
     a.rows = rows;
     const int64_t sign_words = (cols / tile) * (tile >= 64 ? tile / 64 : 1);
     a.sign_words = sign_words <= 2048 ? (int)sign_words : 0;
@@ -261,6 +333,34 @@ int hq_max_payload_words(int64_t rows, int64_t cols, int tile, int lattice, floa
     if (w >= (1ull << 32)) return HQ_ERR_UNSUPPORTED;
     *out = w;
     return HQ_OK;
+}
+
+int hq_min_slot_words(int tile, int lattice, uint32_t *out)
+{
+    if (!out || !valid_tile(tile) || !valid_lattice(lattice)) return HQ_ERR_ARG;
+    *out = min_slot_words(tile, lattice);
+    return HQ_OK;
+}
+
+int hq_fixed_slot_words(int tile, int lattice, float bps, uint32_t *out)
+{
+    if (!out || !valid_tile(tile) || !valid_lattice(lattice) || !valid_bps(bps)) return HQ_ERR_ARG;
+    const double s = std::floor(((double)bps * (double)tile - 20.0) / 32.0);
+    if (s < (double)min_slot_words(tile, lattice)) return HQ_ERR_ARG;
+    *out = (uint32_t)s;
+    return HQ_OK;
+}
+
+int hq_encode_fixed(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, uint64_t seed,
+                    const hq_stream *out, void *stream, int32_t *d_status)
+{
+    return encode_fixed_impl(x, dtype, rows, cols, tile, lattice, seed, out, stream, d_status, false);
+}
+
+int hq_kv_encode_fixed(const void *x, int dtype, int64_t rows, int64_t cols, int tile, int lattice, uint64_t seed,
+                       const hq_stream *out, void *stream, int32_t *d_status)
+{
+    return encode_fixed_impl(x, dtype, rows, cols, tile, lattice, seed, out, stream, d_status, true);
 }
 
 int hq_encode_workspace_bytes(int64_t rows, int64_t cols, int tile, uint64_t *out)

@@ -135,6 +135,169 @@ __device__ __forceinline__ void unpack_raw(const RawTile<EPL, F32IN> &r, float (
     }
 }
 
+// Nearest lattice points of this lane's EPL / D vectors of v / Delta
+// (+ dither), stripped and zigzagged into u; returns the lane's coset bits
+// (bit q for vector q).  sb = 0: the all-zero tile.
+template <int D, int EPL, bool DITHER>
+__device__ __forceinline__ uint32_t quantize_lane(const float (&v)[EPL], uint32_t sb, uint64_t tkey, int l,
+                                                  const A2Consts &a2, uint32_t (&u)[EPL])
+{
+    constexpr int VPL = EPL / D;
+    uint32_t cbits = 0;
+#pragma unroll
+    for (int r = 0; r < EPL; r++) u[r] = 0;
+    if (sb != 0) {
+        const float inv = __frcp_rn(bf16_bits_to_float(sb));
+        float r4[4];
+#pragma unroll
+        for (int q = 0; q < VPL; q++) {
+            float x[D], p[D];
+            int z[D], c;
+#pragma unroll
+            for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
+            if constexpr (DITHER) {
+                float dl[D];
+                dither_vec<D, EPL>(tkey, l, q, r4, dl, a2);
+#pragma unroll
+                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+            }
+            nearest<D>(x, c, z, p, a2);
+            cbits |= (uint32_t)c << q;
+#pragma unroll
+            for (int m = 0; m < D; m++) {
+                int s = z[m];
+                if constexpr (D == 8 || D == 4) {
+                    if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
+                }
+                u[q * D + m] = zigzag(s);
+            }
+        }
+    }
+    return cbits;
+}
+
+// Rice parameter: smallest k minimising sum(u >> k) + N (1 + k) over the
+// group's symbols.  One pass gives the sums at k0-1, k0, k0+1 (k0 = the
+// rate's typical k); the cost is convex in k, so k0 is optimal iff
+// C(k0-1) > C(k0) <= C(k0+1), and only otherwise does the search walk on.
+// `part` gets this lane's sum(u >> k) at the returned k.
+template <int N, int EPL, int LPT>
+__device__ __forceinline__ int rice_param(const uint32_t (&u)[EPL], unsigned mask, int k_hint, uint32_t &part)
+{
+    int k = k_hint;
+    part = 0;
+    const int km = k > 0 ? k - 1 : 0;
+    uint32_t s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int r = 0; r < EPL; r++) {
+        const uint32_t aa = u[r] >> km;
+        s0 += aa;
+        s1 += aa >> 1;
+        s2 += aa >> 2;
+    }
+    const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
+                   S2 = group_sum<LPT>(mask, s2);
+    // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
+    // sum(k) - sum(k + 1) > N
+    bool up = false, down = false;
+    if (k == 0) {
+        if (S0 - S1 <= (uint32_t)N) {
+            part = s0;                       // C(1) >= C(0)
+        } else if (S1 - S2 <= (uint32_t)N) {
+            k = 1;                           // C(1) < C(0), C(2) >= C(1)
+            part = s1;
+        } else {
+            k = 2;
+            part = s2;
+            up = true;
+        }
+    } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
+        k = km;
+        part = s0;
+        down = true;
+    } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
+        k = k + 1;
+        part = s2;
+        up = true;
+    } else {
+        part = s1;
+    }
+    while (down && k > 0) {
+        uint32_t sd = 0;
+#pragma unroll
+        for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
+        if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
+        --k;
+        part = sd;
+    }
+    while (up && k < 15) {
+        uint32_t su = 0;
+#pragma unroll
+        for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
+        if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
+        ++k;
+        part = su;
+    }
+    return k;
+}
+
+// Pack this lane's share of a tile into a zeroed shared-memory image: its
+// coset bits, the k low bits of its symbols, and its unary parts starting
+// uoff bits into the tile's unary section.
+template <int N, int D, int EPL>
+__device__ __forceinline__ void pack_lane(uint32_t *tbuf, int l, int k, uint32_t cbits, const uint32_t (&u)[EPL],
+                                          uint32_t uoff)
+{
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
+    constexpr int VPL = EPL / D;
+    if constexpr (C > 0) or_bits32(tbuf, (uint32_t)l * VPL, cbits, VPL);
+    if (k) {
+        const uint32_t lowmask = (1u << k) - 1u;
+        const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
+        if (k <= 4) {  // 8 codes fit one 32-bit word
+#pragma unroll
+            for (int r0 = 0; r0 < EPL; r0 += 8) {
+                uint32_t acc = 0;
+#pragma unroll
+                for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                or_bits32(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
+            }
+        } else {
+#pragma unroll
+            for (int r0 = 0; r0 < EPL; r0 += 4) {
+                uint64_t acc = 0;
+#pragma unroll
+                for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+                or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
+            }
+        }
+    }
+    // unary parts: eight codes at a time into a 32-bit bitmap
+    uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
+#pragma unroll
+    for (int r0 = 0; r0 < EPL; r0 += 8) {
+        uint32_t bm = 0, rel = 0;
+#pragma unroll
+        for (int m = 0; m < 8; m++) {
+            const uint32_t pbit = rel + (u[r0 + m] >> k);
+            bm |= shl32(1u, pbit);
+            rel = pbit + 1;
+        }
+        if (rel <= 32) {
+            or_bits32(tbuf, upos, bm, (int)rel);
+        } else {  // a long code: set the terminators one by one
+            uint32_t pr = upos;
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                pr += u[r0 + m] >> k;
+                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
+                ++pr;
+            }
+        }
+        upos += rel;
+    }
+}
+
 }  // namespace
 
 // Resident blocks per SM the compiler must fit registers for: 4 (64 registers)
@@ -148,7 +311,6 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
     constexpr int NCW = kEncodeWarps - 1;  // compute warps; the last warp scans and stores
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = NCW * TPW;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;  // coset bits per tile
-    constexpr int VPL = EPL / D;                          // vectors per lane
     constexpr int WPT = N / 64 > 0 ? N / 64 : 1;          // sign words per tile
     static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
     constexpr int kAll = kEncodeWarps * 32, kCompute = NCW * 32;
@@ -238,97 +400,12 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 
                 // ---- nearest point, strip, zigzag
                 uint32_t u[EPL];
-                uint32_t cbits = 0;
-    #pragma unroll
-                for (int r = 0; r < EPL; r++) u[r] = 0;
-                if (sb != 0) {
-                    const float inv = __frcp_rn(bf16_bits_to_float(sb));
-                    const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
-                    float r4[4];
-    #pragma unroll
-                    for (int q = 0; q < VPL; q++) {
-                        float x[D], p[D];
-                        int z[D], c;
-    #pragma unroll
-                        for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
-                        if constexpr (DITHER) {
-                            float dl[D];
-                            dither_vec<D, EPL>(tkey, l, q, r4, dl, a.a2);
-    #pragma unroll
-                            for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
-                        }
-                        nearest<D>(x, c, z, p, a.a2);
-                        cbits |= (uint32_t)c << q;
-    #pragma unroll
-                        for (int m = 0; m < D; m++) {
-                            int s = z[m];
-                            if constexpr (D == 8 || D == 4) {
-                                if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
-                            }
-                            u[q * D + m] = zigzag(s);
-                        }
-                    }
-                }
+                const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
+                const uint32_t cbits = quantize_lane<D, EPL, DITHER>(v, sb, tkey, l, a.a2, u);
 
-                // ---- Rice parameter: smallest k minimising sum(u >> k) + N (1 + k).
-                // One pass gives the sums at k0-1, k0, k0+1 (k0 = the rate's typical k);
-                // the cost is convex in k, so k0 is optimal iff C(k0-1) > C(k0) <= C(k0+1).
-                int k = a.k_hint;
-                uint32_t part = 0;  // this lane's sum(u >> k) at the chosen k
-                {
-                    const int km = k > 0 ? k - 1 : 0;
-                    uint32_t s0 = 0, s1 = 0, s2 = 0;
-    #pragma unroll
-                    for (int r = 0; r < EPL; r++) {
-                        const uint32_t aa = u[r] >> km;
-                        s0 += aa;
-                        s1 += aa >> 1;
-                        s2 += aa >> 2;
-                    }
-                    const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
-                                   S2 = group_sum<LPT>(mask, s2);
-                    // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
-                    // sum(k) - sum(k + 1) > N
-                    bool up = false, down = false;
-                    if (k == 0) {
-                        if (S0 - S1 <= (uint32_t)N) {
-                            part = s0;                       // C(1) >= C(0)
-                        } else if (S1 - S2 <= (uint32_t)N) {
-                            k = 1;                           // C(1) < C(0), C(2) >= C(1)
-                            part = s1;
-                        } else {
-                            k = 2;
-                            part = s2;
-                            up = true;
-                        }
-                    } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
-                        k = km;
-                        part = s0;
-                        down = true;
-                    } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
-                        k = k + 1;
-                        part = s2;
-                        up = true;
-                    } else {
-                        part = s1;
-                    }
-                    while (down && k > 0) {
-                        uint32_t sd = 0;
-    #pragma unroll
-                        for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
-                        if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
-                        --k;
-                        part = sd;
-                    }
-                    while (up && k < 15) {
-                        uint32_t su = 0;
-    #pragma unroll
-                        for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
-                        if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
-                        ++k;
-                        part = su;
-                    }
-                }
+                // ---- Rice parameter (exact argmin)
+                uint32_t part;  // this lane's sum(u >> k) at the chosen k
+                const int k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
 
                 // ---- lengths
                 const uint32_t ul = part + EPL;  // unary bits of this lane
@@ -341,54 +418,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 
                 // ---- pack into the group's image (zeroed at chunk start)
                 uint32_t *tbuf = gstage + goff;
-                if (active && !overflow) {
-                    if constexpr (C > 0) or_bits32(tbuf, (uint32_t)l * VPL, cbits, VPL);
-                    if (k) {
-                        const uint32_t lowmask = (1u << k) - 1u;
-                        const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
-                        if (k <= 4) {  // 8 codes fit one 32-bit word
-    #pragma unroll
-                            for (int r0 = 0; r0 < EPL; r0 += 8) {
-                                uint32_t acc = 0;
-    #pragma unroll
-                                for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                                or_bits32(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
-                            }
-                        } else {
-    #pragma unroll
-                            for (int r0 = 0; r0 < EPL; r0 += 4) {
-                                uint64_t acc = 0;
-    #pragma unroll
-                                for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                                or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
-                            }
-                        }
-                    }
-                    // unary parts: eight codes at a time into a 32-bit bitmap
-                    uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
-    #pragma unroll
-                    for (int r0 = 0; r0 < EPL; r0 += 8) {
-                        uint32_t bm = 0, rel = 0;
-    #pragma unroll
-                        for (int m = 0; m < 8; m++) {
-                            const uint32_t pbit = rel + (u[r0 + m] >> k);
-                            bm |= shl32(1u, pbit);
-                            rel = pbit + 1;
-                        }
-                        if (rel <= 32) {
-                            or_bits32(tbuf, upos, bm, (int)rel);
-                        } else {  // a long code: set the terminators one by one
-                            uint32_t pr = upos;
-    #pragma unroll
-                            for (int m = 0; m < 8; m++) {
-                                pr += u[r0 + m] >> k;
-                                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
-                                ++pr;
-                            }
-                        }
-                        upos += rel;
-                    }
-                }
+                if (active && !overflow) pack_lane<N, D, EPL>(tbuf, l, k, cbits, u, uoff);
                 if (overflow && l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
                 if (l == 0) {
                     tile_w[gid * G + gi] = goff;
@@ -453,6 +483,158 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
     }
 }
 
+// ------------------------------------------------------------ fixed rate
+// Fixed-rate tiles: every tile owns a slot of S words at word t S, so no
+// offsets are computed or stored and tiles are independent.  Per tile the
+// scale Delta is searched over bf16 bit patterns so that the coded tile fits
+// its slot: from the closed-form scale c0, steps of 4, 8, 16, ... patterns
+// towards the boundary (down while it fits, up until it fits; four octaves
+// at most either way), then bisection to a fitting scale whose next finer
+// pattern does not fit.  If no scale of the range fits, the tile is stored
+// as the all-zero tile, which a legal slot always holds.  Each probe
+// quantizes the rotated tile (held in registers) and prices it with the Rice
+// parameter search; the probe's size is group-uniform, so each group walks
+// its own search.  A group encodes the pair of tiles 2p, 2p + 1, which share
+// the byte of packed 4-bit Rice parameters, into a zeroed shared-memory slot
+// image and stores it whole.
+
+constexpr int kFixedWarps = 8;
+// Resident blocks the registers are budgeted for: the rotated tile, the
+// next tile's raw words and a probe's symbols are live together, which
+// spills at 64 or 80 registers but fits 128 without spills.
+constexpr int fixed_min_blocks(int epl) { return epl >= 32 ? 1 : 2; }
+constexpr int kFixedMaxProbes = 64;  // the search needs at most about 20
+
+// Coded bits of the rotated tile at scale pattern c: C + N (1 + k) + sum(u >> k).
+template <int N, int D, int EPL, bool DITHER>
+__device__ __forceinline__ uint32_t fixed_probe_bits(const float (&v)[EPL], uint32_t c, uint64_t tkey, int l,
+                                                     const A2Consts &a2, unsigned mask, int k_hint)
+{
+    constexpr int LPT = N / EPL;
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
+    uint32_t u[EPL];
+    quantize_lane<D, EPL, DITHER>(v, c, tkey, l, a2, u);
+    uint32_t part;
+    const int k = rice_param<N, EPL, LPT>(u, mask, k_hint, part);
+    return (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part);
+}
+
+// The scale search as one probe site driven by a small state machine
+// (start probe, walk down, walk up, bisect), so the probe is inlined once.
+template <int N, int D, int EPL, bool DITHER>
+__device__ __forceinline__ uint32_t fixed_scale(const float (&v)[EPL], uint32_t c0, uint32_t budget, uint64_t tkey,
+                                                int l, const A2Consts &a2, unsigned mask, int k_hint)
+{
+    if (c0 == 0) return 0;
+    const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
+    const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
+    enum { kStart, kDown, kUp, kBisect };
+    int phase = kStart, lo = 0, hi = (int)c0, step = 4, c = (int)c0;
+    for (int probe = 0; probe < kFixedMaxProbes; probe++) {
+        const bool f = fixed_probe_bits<N, D, EPL, DITHER>(v, (uint32_t)c, tkey, l, a2, mask, k_hint) <= budget;
+        if (phase == kStart) {
+            if (f) { hi = c; phase = kDown; } else { lo = c; phase = kUp; }
+        } else if (phase == kDown) {
+            if (f) { hi = c; step *= 2; } else { lo = c; phase = kBisect; }
+        } else if (phase == kUp) {
+            if (f) { hi = c; phase = kBisect; } else { lo = c; step *= 2; }
+        } else {
+            if (f) hi = c; else lo = c;
+        }
+        if (phase == kDown) {
+            if (hi == lo_lim) return (uint32_t)hi;
+            c = hi - step > lo_lim ? hi - step : lo_lim;
+        } else if (phase == kUp) {
+            if (lo == hi_lim) return 0u;
+            c = lo + step < hi_lim ? lo + step : hi_lim;
+        } else {
+            if (hi - lo <= 1) return (uint32_t)hi;
+            c = (lo + hi) >> 1;
+        }
+    }
+    return phase == kUp ? 0u : (uint32_t)hi;  // not reached: the walk and the bisection end well before
+}
+
+template <int N, int D, int EPL, bool DITHER, bool F32IN>
+__global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
+    encode_fixed_kernel(const EncodeArgs a)
+{
+    constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kFixedWarps * TPW;
+    constexpr int WPT = N / 64 > 0 ? N / 64 : 1;
+    static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
+    const uint32_t S = a.slot_words;
+    const uint32_t istride = (S + 1 + 3) & ~3u;  // slot image + a guard word, 16-byte multiple
+    extern __shared__ __align__(16) uint32_t smem[];
+    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);
+    uint32_t *images = smem + 2 * ((a.sign_words + 1) & ~1);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < a.sign_words; i += kFixedWarps * 32) {
+        const uint64_t j = (uint64_t)(i / WPT), m = (uint64_t)(i % WPT);
+        sign_tab[i] = mix64(mix64(a.sign_key ^ j) ^ m);
+    }
+    __syncthreads();
+
+    const int l = lane % LPT;
+    const int gid = warp * TPW + lane / LPT;
+    const unsigned mask = group_mask<LPT>(lane);
+    uint32_t *img = images + (size_t)gid * istride;
+    const int64_t npairs = (a.ntiles + 1) >> 1;
+    const uint32_t tpr = (uint32_t)a.tiles_per_row;
+    const uint32_t budget = 32u * S;
+
+    for (int64_t p = (int64_t)blockIdx.x * GPB + gid; p < npairs; p += (int64_t)gridDim.x * GPB) {
+        uint32_t kbyte = 0;
+        RawTile<EPL, F32IN> raw;
+        const int64_t tp = 2 * p;
+        load_raw<EPL, F32IN>(a.x, tp * N + (int64_t)l * EPL, raw);
+        uint32_t jj = (uint32_t)tp - fast_div((uint32_t)tp, a.tpr_div) * tpr;
+#pragma unroll 1
+        for (int h = 0; h < 2; h++) {
+            const int64_t t = tp + h;
+            if (t >= a.ntiles) break;  // group-uniform
+            // ---- signs, then prefetch the pair's second tile
+            const uint32_t i0 = (uint32_t)l * EPL;
+            const uint64_t sw = a.sign_words ? sign_tab[(uint64_t)jj * WPT + (i0 >> 6)]
+                                             : mix64(mix64(a.sign_key ^ (uint64_t)jj) ^ (uint64_t)(i0 >> 6));
+            const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
+            float v[EPL];
+            unpack_raw<EPL, F32IN>(raw, v);
+#pragma unroll
+            for (int r = 0; r < EPL; r++)
+                v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
+            if (h == 0 && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
+            if (++jj == tpr) jj = 0;
+
+            // ---- rotation, closed-form start, scale search
+            const float Ssq = sumsq<EPL, LPT>(v, mask);
+            fwht<EPL, LPT>(v, mask, l);
+            bool nonfinite;
+            const uint32_t c0 = tile_scale_bits(Ssq, a.c, nonfinite);
+            if (nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
+            const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
+            const uint32_t sb = fixed_scale<N, D, EPL, DITHER>(v, c0, budget, tkey, l, a.a2, mask, a.k_hint);
+
+            // ---- the chosen scale: quantize, Rice parameter, pack, store the slot
+            uint32_t u[EPL];
+            const uint32_t cbits = quantize_lane<D, EPL, DITHER>(v, sb, tkey, l, a.a2, u);
+            uint32_t part;
+            const int k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
+            const uint32_t uoff = group_excl_scan<LPT>(mask, part + EPL, l);
+            for (uint32_t i = l; i < istride; i += LPT) img[i] = 0u;
+            __syncwarp(mask);
+            pack_lane<N, D, EPL>(img, l, k, cbits, u, uoff);
+            __syncwarp(mask);
+            uint32_t *dst = a.payload + (uint64_t)t * S;
+            for (uint32_t i = l; i < S; i += LPT) dst[i] = img[i];
+            __syncwarp(mask);  // the image is reused by the next tile
+            if (l == 0) a.scale[t] = (uint16_t)sb;
+            kbyte |= (uint32_t)k << (4 * h);
+        }
+        if (l == 0) a.kk[p] = (uint8_t)kbyte;
+    }
+}
+
 // ------------------------------------------------------------------ launch
 namespace {
 
@@ -503,6 +685,46 @@ cudaError_t launch_encode_n(int lattice, bool dither, int dtype, const EncodeArg
     }
 }
 
+template <int N, int D, bool DITHER, bool F32IN>
+cudaError_t launch_encode_fixed_t(const EncodeArgs &a, cudaStream_t s)
+{
+    constexpr int EPL = epl_for<N>(), GPB = kFixedWarps * (32 / (N / EPL));
+    const size_t istride = (a.slot_words + 1 + 3) & ~(size_t)3;
+    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + (size_t)GPB * istride * 4;
+    auto kern = encode_fixed_kernel<N, D, EPL, DITHER, F32IN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFixedWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t npairs = (a.ntiles + 1) / 2;
+    int64_t blocks = (npairs + GPB - 1) / GPB;
+    const int64_t wave = (int64_t)sm_count() * per_sm;
+    if (blocks > wave) blocks = wave;
+    kern<<<(unsigned)blocks, kFixedWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int N, int D>
+cudaError_t launch_encode_fixed_nd(bool dither, int dtype, const EncodeArgs &a, cudaStream_t s)
+{
+    if (dither)
+        return dtype ? launch_encode_fixed_t<N, D, true, true>(a, s) : launch_encode_fixed_t<N, D, true, false>(a, s);
+    return dtype ? launch_encode_fixed_t<N, D, false, true>(a, s) : launch_encode_fixed_t<N, D, false, false>(a, s);
+}
+
+template <int N>
+cudaError_t launch_encode_fixed_n(int lattice, bool dither, int dtype, const EncodeArgs &a, cudaStream_t s)
+{
+    switch (lattice) {
+    case 1: return launch_encode_fixed_nd<N, 1>(dither, dtype, a, s);
+    case 2: return launch_encode_fixed_nd<N, 2>(dither, dtype, a, s);
+    case 4: return launch_encode_fixed_nd<N, 4>(dither, dtype, a, s);
+    default: return launch_encode_fixed_nd<N, 8>(dither, dtype, a, s);
+    }
+}
+
 int groups_for(int tile)
 {
     switch (tile) {
@@ -543,6 +765,18 @@ cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const E
     case 256: return launch_encode_n<256>(lattice, dither, dtype, a, s);
     case 512: return launch_encode_n<512>(lattice, dither, dtype, a, s);
     default: return launch_encode_n<1024>(lattice, dither, dtype, a, s);
+    }
+}
+
+cudaError_t launch_encode_fixed(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
+                                cudaStream_t s)
+{
+    switch (tile) {
+    case 64: return launch_encode_fixed_n<64>(lattice, dither, dtype, a, s);
+    case 128: return launch_encode_fixed_n<128>(lattice, dither, dtype, a, s);
+    case 256: return launch_encode_fixed_n<256>(lattice, dither, dtype, a, s);
+    case 512: return launch_encode_fixed_n<512>(lattice, dither, dtype, a, s);
+    default: return launch_encode_fixed_n<1024>(lattice, dither, dtype, a, s);
     }
 }
 

@@ -49,6 +49,7 @@ struct EncodeArgs {
     int k_hint;           // the rate's typical Rice parameter (search start)
     FastDiv tpr_div;      // division by tiles_per_row
     uint32_t stall_chunk; // test hook: this chunk never publishes its prefix (0xffffffff: none)
+    uint32_t slot_words;  // fixed-rate encode: words per tile slot (kk then holds packed 4-bit k)
 };
 
 struct DecodeArgs {
@@ -70,6 +71,8 @@ struct DecodeArgs {
     int64_t rows;
     int sign_words;       // sign words cached per block (0: hash them per tile)
     FastDiv tpr_div;      // division by tiles_per_row
+    uint32_t slot;        // fixed-rate stream: words per tile slot, tile t at t * slot, k packed
+                          // two per byte (0: variable rate, offsets from off[], one k per byte)
 };
 
 // Batch-1 attention over K and V codec streams (one tile per cached vector).
@@ -109,6 +112,8 @@ struct GemmPlan {
 // Launch helpers; return a cudaError_t.
 cudaError_t launch_encode(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
                           cudaStream_t s);
+cudaError_t launch_encode_fixed(int tile, int lattice, bool dither, int dtype, const EncodeArgs &a,
+                                cudaStream_t s);
 cudaError_t launch_decode(int tile, int lattice, bool dither, int dtype, const DecodeArgs &a,
                           cudaStream_t s);
 cudaError_t launch_gemv(int tile, int lattice, const DecodeArgs &a, int64_t cols, cudaStream_t s);

@@ -16,6 +16,10 @@
 // (offsets out of order or past the capacity, k > 15, a scale that is not 0
 // or a positive normal bf16, a terminator count other than n, a word count
 // other than its bits need) parses to zeros and is reported as bad.
+// A fixed-rate stream (a.slot > 0) puts tile t at words [t S, t S + S) and
+// its k in 4 bits; the slot may end in zero words, so the last lane's span
+// ends at the last one bit of the slot (found by a max over the group)
+// rather than in the last word, and only the word-count rule is dropped.
 #pragma once
 
 #include "hq_internal.h"
@@ -55,8 +59,18 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     constexpr int VPL = EPL / D;
     uint32_t *starts = wbuf + a.wmax + 4;
 
-    const uint32_t o0 = a.off[t], o1 = a.off[t + 1];
-    const int k = a.kk[t];
+    const bool fixed = a.slot != 0;
+    uint32_t o0, o1;
+    int k;
+    if (fixed) {
+        o0 = (uint32_t)t * a.slot;  // the host keeps ntiles * slot below 2^32
+        o1 = o0 + a.slot;
+        k = (a.kk[t >> 1] >> ((t & 1) * 4)) & 15;
+    } else {
+        o0 = a.off[t];
+        o1 = a.off[t + 1];
+        k = a.kk[t];
+    }
     sb = a.scale[t];
     // Delta is 0 or a positive, normal, finite bf16 in any canonical tile
     const uint32_t ex = sb & 0x7f80u;
@@ -76,7 +90,7 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     // word holding terminator m*EPL - 1 yields lane m's start
     const uint32_t wu0 = U0 >> 5;
     const uint32_t nwu = W > wu0 ? W - wu0 : 0;  // unary words (the first shared with the low parts)
-    uint32_t found = 0;
+    uint32_t found = 0, last_nz = 0;  // last_nz: 1 + the last unary word holding a one bit (fixed rate)
     bool last_empty = false;
     for (uint32_t wb = 0; wb < nwu; wb += LPT) {
         const uint32_t wi = wb + l;
@@ -92,13 +106,15 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
         if (wi < nwu) {
             const uint32_t before = found + incl - c, after = found + incl;
             if (wi == nwu - 1 && c == 0) last_empty = true;  // padding after the last terminator
+            if (fixed && c) last_nz = wi + 1;
             for (uint32_t m = (before + EPL) / EPL; m < (uint32_t)LPT && m * EPL <= after; m++)
                 starts[m] = (wu0 + wi) * 32u + select_bit(v, m * EPL - 1u - before) + 1u - U0;
         }
         found += __shfl_sync(mask, incl, LPT - 1, LPT);
     }
     const bool pad_word = __any_sync(mask, last_empty);
-    if (!bad && (found != (uint32_t)N || pad_word)) bad = true;
+    if (!bad && (found != (uint32_t)N || (pad_word && !fixed))) bad = true;
+    if (fixed) last_nz = group_max<LPT>(mask, last_nz);
     __syncwarp(mask);
 
 #pragma unroll
@@ -112,8 +128,11 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     // the next lane's start bounds this lane's codes
     uint32_t end = __shfl_down_sync(mask, start, 1, LPT);
     if (l == LPT - 1) {
-        const uint32_t v = wbuf[W - 1] & (nwu == 1 ? (0xffffffffu << (U0 & 31)) : 0xffffffffu);
-        end = (W - 1) * 32u + (31u - __clz(v)) + 1u - U0;
+        // the word of the tile's last terminator: the last word, or for a
+        // fixed-rate slot the last unary word holding a one bit
+        const uint32_t wl = fixed ? wu0 + last_nz - 1u : W - 1u;
+        const uint32_t v = wbuf[wl] & (wl == wu0 ? (0xffffffffu << (U0 & 31)) : 0xffffffffu);
+        end = wl * 32u + (31u - __clz(v)) + 1u - U0;
     }
 
     // ---- coset bits and low parts

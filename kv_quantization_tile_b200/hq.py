@@ -30,7 +30,8 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_max_payload_words", "hq_encode_workspace_bytes", "hq_encode", "hq_kv_encode",
            "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
-           "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled"]
+           "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled",
+           "hq_min_slot_words", "hq_fixed_slot_words", "hq_encode_fixed", "hq_kv_encode_fixed"]
 
 
 class hq_file_info(ctypes.Structure):
@@ -42,7 +43,7 @@ class hq_file_info(ctypes.Structure):
 class hq_stream(ctypes.Structure):
     _fields_ = [("payload", ctypes.c_void_p), ("payload_capacity_words", ctypes.c_uint64),
                 ("tile_off", ctypes.c_void_p), ("tile_scale", ctypes.c_void_p),
-                ("tile_k", ctypes.c_void_p)]
+                ("tile_k", ctypes.c_void_p), ("slot_words", ctypes.c_uint32)]
 
 
 _lib = ctypes.CDLL(_LIB_PATH)
@@ -76,6 +77,10 @@ _SIGS = {
     "hq_file_write": (_i32, [ctypes.POINTER(hq_file_info), _vp, _vp, _vp, _vp, _vp, _u64]),
     "hq_file_read": (_i32, [_vp, _u64, ctypes.POINTER(hq_file_info), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                             ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    "hq_min_slot_words": (_i32, [_i32, _i32, ctypes.POINTER(ctypes.c_uint32)]),
+    "hq_fixed_slot_words": (_i32, [_i32, _i32, _f32, ctypes.POINTER(ctypes.c_uint32)]),
+    "hq_encode_fixed": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _u64, ctypes.POINTER(hq_stream), _vp, _vp]),
+    "hq_kv_encode_fixed": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _u64, ctypes.POINTER(hq_stream), _vp, _vp]),
     "hq_decode_gemm": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
                               _u64, _vp, _vp]),
     "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
@@ -166,23 +171,32 @@ def hq_encode_workspace_bytes(rows: int, cols: int, tile: int) -> int:
 # ----------------------------------------------------------------- streams
 @dataclass
 class Stream:
-    """Device buffers of one compressed matrix (all owned by torch)."""
+    """Device buffers of one compressed matrix (all owned by torch).
+    slot_words > 0 marks a fixed-rate stream: tile t in payload words
+    [t S, t S + S), no offsets (tile_off empty), k packed two per byte."""
     payload: torch.Tensor      # int32 words (bit patterns of uint32)
-    tile_off: torch.Tensor     # int32, ntiles + 1 (uint32 offsets)
+    tile_off: torch.Tensor     # int32, ntiles + 1 (uint32 offsets); empty for fixed rate
     tile_scale: torch.Tensor   # int16, ntiles (bf16 bits of Delta)
-    tile_k: torch.Tensor       # uint8, ntiles
+    tile_k: torch.Tensor       # uint8, ntiles (fixed rate: (ntiles + 1) // 2 packed bytes)
+    slot_words: int = 0
 
     def struct(self) -> hq_stream:
-        return hq_stream(_ptr(self.payload), self.payload.numel(), _ptr(self.tile_off),
+        return hq_stream(_ptr(self.payload), self.payload.numel(),
+                         _ptr(self.tile_off) if self.tile_off.numel() else 0,
                          _ptr(self.tile_scale) if self.tile_scale.numel() else 0,
-                         _ptr(self.tile_k) if self.tile_k.numel() else 0)
+                         _ptr(self.tile_k) if self.tile_k.numel() else 0, self.slot_words)
 
     def words(self) -> int:
-        """Payload words actually used (reads tile_off[-1]; synchronises)."""
+        """Payload words actually used (variable rate: reads tile_off[-1] and synchronises)."""
+        if self.slot_words:
+            return self.tile_scale.numel() * self.slot_words
         return int(self.tile_off[-1].item()) & 0xFFFFFFFF
 
     def nbytes(self) -> int:
-        """Compressed bytes: used payload words plus the per-tile headers."""
+        """Compressed bytes: used payload words plus the per-tile headers
+        (fixed rate: bf16 Delta and a 4-bit k per tile, rounded to bytes)."""
+        if self.slot_words:
+            return 4 * self.words() + 2 * self.tile_scale.numel() + self.tile_k.numel()
         return 4 * self.words() + 4 * self.tile_off.numel() + 2 * self.tile_scale.numel() + self.tile_k.numel()
 
 
@@ -194,6 +208,28 @@ def alloc_stream(rows: int, cols: int, tile: int, lattice, bps: float, device="c
                   tile_off=torch.empty(ntiles + 1, dtype=torch.int32, device=device),
                   tile_scale=torch.empty(ntiles, dtype=torch.int16, device=device),
                   tile_k=torch.empty(ntiles, dtype=torch.uint8, device=device))
+
+
+def hq_min_slot_words(tile: int, lattice) -> int:
+    out = ctypes.c_uint32(0)
+    _check(_lib.hq_min_slot_words(tile, _lat(lattice), ctypes.byref(out)), "hq_min_slot_words")
+    return out.value
+
+
+def hq_fixed_slot_words(tile: int, lattice, bps: float) -> int:
+    out = ctypes.c_uint32(0)
+    _check(_lib.hq_fixed_slot_words(tile, _lat(lattice), bps, ctypes.byref(out)), "hq_fixed_slot_words")
+    return out.value
+
+
+def alloc_fixed_stream(rows: int, cols: int, tile: int, slot_words: int, device="cuda") -> Stream:
+    """Buffers of a fixed-rate stream with slots of slot_words words."""
+    ntiles = rows * (cols // tile)
+    return Stream(payload=torch.empty(max(ntiles * slot_words, 1), dtype=torch.int32, device=device),
+                  tile_off=torch.empty(0, dtype=torch.int32, device=device),
+                  tile_scale=torch.empty(ntiles, dtype=torch.int16, device=device),
+                  tile_k=torch.empty((ntiles + 1) // 2, dtype=torch.uint8, device=device),
+                  slot_words=slot_words)
 
 
 def alloc_workspace(rows: int, cols: int, tile: int, device="cuda") -> torch.Tensor:
@@ -218,6 +254,25 @@ def hq_encode(x, tile, lattice, bps, seed, out: Stream, workspace, status=None, 
 
 def hq_kv_encode(x, tile, lattice, bps, seed, out: Stream, workspace, status=None, stream=None) -> Stream:
     return _encode(_lib.hq_kv_encode, x, tile, lattice, bps, seed, out, workspace, status, stream)
+
+
+def _encode_fixed(fn, x: torch.Tensor, tile: int, lattice, seed: int, out: Stream, status, stream):
+    assert x.is_contiguous() and x.dim() == 2
+    rows, cols = x.shape
+    s = out.struct()
+    _check(fn(_ptr(x), _dtype_code(x), rows, cols, tile, _lat(lattice), seed, ctypes.byref(s),
+              _stream_handle(stream), _ptr(status)), fn.__name__)
+    return out
+
+
+def hq_encode_fixed(x, tile, lattice, seed, out: Stream, status=None, stream=None) -> Stream:
+    """Fixed-rate encode into out (from alloc_fixed_stream): every tile fits
+    its slot, with Delta searched per tile."""
+    return _encode_fixed(_lib.hq_encode_fixed, x, tile, lattice, seed, out, status, stream)
+
+
+def hq_kv_encode_fixed(x, tile, lattice, seed, out: Stream, status=None, stream=None) -> Stream:
+    return _encode_fixed(_lib.hq_kv_encode_fixed, x, tile, lattice, seed, out, status, stream)
 
 
 def _decode(fn, s: Stream, rows: int, cols: int, tile: int, lattice, bps: float, seed: int,
@@ -326,6 +381,8 @@ def hq_encode_noalloc(x, tile, lattice, bps, seed, out: Stream, status=None, str
 def stream_to_bytes(s: Stream, rows: int, cols: int, tile: int, lattice, bps: float, seed: int,
                     dither: bool = False) -> bytes:
     """The checkpoint container of a stream (its arrays are copied to the host)."""
+    if s.slot_words:
+        raise ValueError("the checkpoint container holds variable-rate streams only")
     off = s.tile_off.cpu().numpy().view(np.uint32)
     words = int(off[-1])
     scale = s.tile_scale.cpu().numpy().view(np.uint16)

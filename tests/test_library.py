@@ -155,3 +155,45 @@ def test_kv_attention_sizing_and_validation():
     assert call(wsb=64) == hq.HQ_ERR_WORKSPACE
     assert call(heads=70000) == hq.HQ_ERR_UNSUPPORTED
     assert call(heads=0) == hq.HQ_OK  # nothing to do, nothing launched
+
+
+def test_fixed_rate_sizing_and_validation():
+    for tile in (64, 128, 256, 512, 1024):
+        for lat in LATS:
+            assert hq.hq_min_slot_words(tile, lat) == oracle.min_slot_words(tile, lat)
+            for bps in (1.0, 2.0, 3.3, 4.0, 8.0):
+                want = oracle.fixed_slot_words(tile, lat, bps)
+                if want < 0:
+                    with pytest.raises(hq.HQError):
+                        hq.hq_fixed_slot_words(tile, lat, bps)
+                else:
+                    assert hq.hq_fixed_slot_words(tile, lat, bps) == want
+    lib = hq.library()
+    ARG = hq.HQ_ERR_ARG
+
+    def enc(x, rows, cols, tile, lat, st, fn=lib.hq_encode_fixed):
+        return fn(x, 0, rows, cols, tile, lat, 0, ctypes.byref(st) if st is not None else None, None, None)
+
+    ok = hq.hq_stream(16, 1 << 20, 0, 16, 16, 31)
+    assert enc(16, 4, 256, 256, 8, None) == ARG                                   # no stream
+    assert enc(16, 4, 256, 256, 8, hq.hq_stream(16, 1 << 20, 0, 16, 16, 0)) == ARG  # slot 0
+    assert enc(16, 4, 256, 256, 8, hq.hq_stream(16, 1 << 20, 0, 16, 16, 8)) == ARG  # below the minimum (9)
+    assert enc(16, 4, 256, 256, 8, hq.hq_stream(16, 1 << 20, 0, 16, 16, 65)) == ARG  # above n / 4
+    assert enc(16, 4, 256, 256, 8, hq.hq_stream(16, 100, 0, 16, 16, 31)) == hq.HQ_ERR_CAPACITY
+    assert enc(16, 1 << 27, 256, 256, 8, hq.hq_stream(16, 1 << 40, 0, 16, 16, 64)) == hq.HQ_ERR_UNSUPPORTED
+    assert enc(0, 4, 256, 256, 8, ok) == ARG                                      # x NULL
+    assert enc(18, 4, 256, 256, 8, ok) == ARG                                     # x misaligned
+    assert enc(16, 4, 256, 256, 3, ok) == ARG                                     # lattice
+    assert enc(16, 4, 250, 256, 8, ok) == ARG                                     # cols % tile
+    assert enc(16, 4, 256, 256, 8, hq.hq_stream(16, 1 << 20, 0, 0, 16, 31)) == ARG  # no scales
+    # a fixed-rate stream is not a variable-rate encode target
+    assert lib.hq_encode(16, 0, 4, 256, 256, 8, 4.0, 0, ctypes.byref(hq.hq_stream(16, 1 << 20, 16, 16, 16, 31)),
+                         16, 1 << 20, None, None) == ARG
+    # decoders check the slot and the capacity of fixed-rate streams
+    assert lib.hq_decode(ctypes.byref(hq.hq_stream(16, 1 << 20, 0, 16, 16, 8)), 4, 256, 256, 8, 4.0, 0, 16, 0,
+                         None, None) == ARG
+    assert lib.hq_decode(ctypes.byref(hq.hq_stream(16, 100, 0, 16, 16, 31)), 4, 256, 256, 8, 4.0, 0, 16, 0,
+                         None, None) == hq.HQ_ERR_CAPACITY
+    # variable-rate streams still need their offsets
+    assert lib.hq_decode(ctypes.byref(hq.hq_stream(16, 1 << 20, 0, 16, 16, 0)), 4, 256, 256, 8, 4.0, 0, 16, 0,
+                         None, None) == ARG
