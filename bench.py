@@ -45,7 +45,7 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
-    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "kv", "kv_attention"],
+    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "kv", "kv_attention", "fixed"],
                    help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
     p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
     p.add_argument("--batch", type=int, default=None, help="one batch size for --leg gemm")
@@ -333,7 +333,7 @@ def run_ours(args):
         out["e2e"] = e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier)
         if rank == 0:
             out["paths"] = {"gemv": gemv_leg(dev, peak), "gemm": gemm_leg(dev, peak), "kv": kv_leg(dev, peak),
-                            "kv_attention": attention_leg(dev, peak)}
+                            "kv_attention": attention_leg(dev, peak), "fixed_rate": fixed_leg(dev, peak)}
             out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out))
@@ -603,6 +603,94 @@ def attention_leg(dev, peak, group=4):
             "decode_then_sdpa_us": round(t_dec * 1e3, 2), "speedup_vs_bf16_sdpa": round(t_sdpa / t, 3)}
 
 
+def fixed_leg(dev, peak):
+    """Fixed-rate streams at 4 bits per weight in total (side information
+    included): the seven Llama-3.1-8B layer matrices (tile 256, E8, slot 31)
+    and one KV layer's K and V with dither (tile 128, E8, slot 15); encode
+    (with its per-tile scale search) and decode timed with CUDA events,
+    inputs far larger than L2; plus the batch-1 decode-GEMV on the fixed
+    14336x4096 stream.  The reconstruction error is reported beside the
+    variable-rate stream's at its nominal 4 bps."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    res = {}
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    flushbuf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def run(mats, tile, dither, tag):
+        slot = hq.hq_fixed_slot_words(tile, LAT, BPS)
+        ctx = []
+        for x in mats:
+            r, c = x.shape
+            ctx.append((x, hq.alloc_fixed_stream(r, c, tile, slot, dev), torch.empty_like(x)))
+        enc_fn = hq.hq_kv_encode_fixed if dither else hq.hq_encode_fixed
+        dec_fn = hq.hq_kv_decode if dither else hq.hq_decode
+
+        def enc():
+            for x, s, _ in ctx:
+                enc_fn(x, tile, LAT, SEED, s, st)
+
+        def dec():
+            for x, s, y in ctx:
+                dec_fn(s, x.shape[0], x.shape[1], tile, LAT, BPS, SEED, y, st)
+
+        for _ in range(3):
+            enc(); dec()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        n = sum(x.numel() for x, _, _ in ctx)
+        cb = sum(s.nbytes() for _, s, _ in ctx)
+        te = time_launches(enc, lambda: flush_l2(flushbuf), reps=5)
+        td = time_launches(dec, lambda: flush_l2(flushbuf), reps=5)
+        num = sum(float(((y.float() - x.float()) ** 2).sum()) for x, _, y in ctx)
+        den = sum(float((x.float() ** 2).sum()) for x, _, _ in ctx)
+        # the variable-rate stream of the same inputs at its nominal rate, for comparison
+        vnum, vbytes = 0.0, 0
+        for x, _, y in ctx:
+            r, c = x.shape
+            v = hq.alloc_stream(r, c, tile, LAT, BPS, dev)
+            (hq.hq_kv_encode if dither else hq.hq_encode)(x, tile, LAT, BPS, SEED, v, hq.alloc_workspace(r, c, tile, dev), st)
+            dec_fn(v, r, c, tile, LAT, BPS, SEED, y, st)
+            vnum += float(((y.float() - x.float()) ** 2).sum())
+            vbytes += v.nbytes()
+            del v
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        res[tag] = {"slot_words": slot, "tile": tile, "bits_per_value_total": round(8 * cb / n, 4),
+                    "encode_ms": round(te, 4), "decode_ms": round(td, 4),
+                    "encode_alg_gbs": round((2 * n + cb) / te / 1e6, 1),
+                    "decode_alg_gbs": round((2 * n + cb) / td / 1e6, 1),
+                    "encode_frac": round((2 * n + cb) / te / 1e6 / peak, 4),
+                    "decode_frac": round((2 * n + cb) / td / 1e6 / peak, 4),
+                    "rel_rmse": round(math.sqrt(num / den), 5),
+                    "variable_rate": {"bits_per_value_total": round(8 * vbytes / n, 4),
+                                      "rel_rmse": round(math.sqrt(vnum / den), 5)}}
+        return ctx
+
+    ctx = run([m for _, m in workloads.llama_layer(dev)], TILE, False, "llama_layer_e8")
+    del ctx
+    k, v = workloads.kv_layer(dev)
+    ctx = run([k, v], 128, True, "kv_layer_e8")
+    del ctx, k, v
+    w1, _, x1, _ = workloads.gemv_case(dev)
+    r, c = w1.shape
+    slot = hq.hq_fixed_slot_words(TILE, LAT, BPS)
+    s = hq.alloc_fixed_stream(r, c, TILE, slot, dev)
+    hq.hq_encode_fixed(w1, TILE, LAT, SEED, s, st)
+    y = torch.empty(r, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        hq.hq_decode_gemv(s, r, c, TILE, LAT, BPS, SEED, x1, y, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ms = time_launches(lambda: hq.hq_decode_gemv(s, r, c, TILE, LAT, BPS, SEED, x1, y, st), lambda: flush_l2(flushbuf))
+    nb = s.nbytes() + 2 * c + 4 * r
+    res["gemv_14336x4096"] = {"us": round(ms * 1e3, 2), "alg_gbs": round(nb / ms / 1e6, 1),
+                              "frac": round(nb / ms / 1e6 / peak, 4), "compressed_bytes": nb - 2 * c - 4 * r}
+    return res
+
+
 def run_leg(args):
     peak, _ = peaks()
     if args.leg == "gemv":
@@ -611,6 +699,8 @@ def run_leg(args):
         res = gemm_leg("cuda", peak, batches=(args.batch,) if args.batch else (1, 16, 64, 256))
     elif args.leg == "kv":
         res = kv_leg("cuda", peak)
+    elif args.leg == "fixed":
+        res = fixed_leg("cuda", peak)
     else:
         res = attention_leg("cuda", peak, group=args.group)
     print(json.dumps({"leg": args.leg, **res}))

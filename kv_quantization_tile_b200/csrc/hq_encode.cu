@@ -500,60 +500,12 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 
 constexpr int kFixedWarps = 8;
 // Resident blocks the registers are budgeted for: the rotated tile, the
-// next tile's raw words and a probe's symbols are live together, which
-// spills at 64 or 80 registers but fits 128 without spills.
-constexpr int fixed_min_blocks(int epl) { return epl >= 32 ? 1 : 2; }
+// next tile's raw words and a probe's symbols are live together.  At 80
+// registers (3 blocks per SM) E8 spills a few words, yet measured faster
+// than 128 registers without spills (2 blocks) and no slower than 64 (4).
+constexpr int fixed_min_blocks(int epl) { return epl >= 32 ? 1 : 3; }
 constexpr int kFixedMaxProbes = 64;  // the search needs at most about 20
-
-// Coded bits of the rotated tile at scale pattern c: C + N (1 + k) + sum(u >> k).
-template <int N, int D, int EPL, bool DITHER>
-__device__ __forceinline__ uint32_t fixed_probe_bits(const float (&v)[EPL], uint32_t c, uint64_t tkey, int l,
-                                                     const A2Consts &a2, unsigned mask, int k_hint)
-{
-    constexpr int LPT = N / EPL;
-    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
-    uint32_t u[EPL];
-    quantize_lane<D, EPL, DITHER>(v, c, tkey, l, a2, u);
-    uint32_t part;
-    const int k = rice_param<N, EPL, LPT>(u, mask, k_hint, part);
-    return (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part);
-}
-
-// The scale search as one probe site driven by a small state machine
-// (start probe, walk down, walk up, bisect), so the probe is inlined once.
-template <int N, int D, int EPL, bool DITHER>
-__device__ __forceinline__ uint32_t fixed_scale(const float (&v)[EPL], uint32_t c0, uint32_t budget, uint64_t tkey,
-                                                int l, const A2Consts &a2, unsigned mask, int k_hint)
-{
-    if (c0 == 0) return 0;
-    const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
-    const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
-    enum { kStart, kDown, kUp, kBisect };
-    int phase = kStart, lo = 0, hi = (int)c0, step = 4, c = (int)c0;
-    for (int probe = 0; probe < kFixedMaxProbes; probe++) {
-        const bool f = fixed_probe_bits<N, D, EPL, DITHER>(v, (uint32_t)c, tkey, l, a2, mask, k_hint) <= budget;
-        if (phase == kStart) {
-            if (f) { hi = c; phase = kDown; } else { lo = c; phase = kUp; }
-        } else if (phase == kDown) {
-            if (f) { hi = c; step *= 2; } else { lo = c; phase = kBisect; }
-        } else if (phase == kUp) {
-            if (f) { hi = c; phase = kBisect; } else { lo = c; step *= 2; }
-        } else {
-            if (f) hi = c; else lo = c;
-        }
-        if (phase == kDown) {
-            if (hi == lo_lim) return (uint32_t)hi;
-            c = hi - step > lo_lim ? hi - step : lo_lim;
-        } else if (phase == kUp) {
-            if (lo == hi_lim) return 0u;
-            c = lo + step < hi_lim ? lo + step : hi_lim;
-        } else {
-            if (hi - lo <= 1) return (uint32_t)hi;
-            c = (lo + hi) >> 1;
-        }
-    }
-    return phase == kUp ? 0u : (uint32_t)hi;  // not reached: the walk and the bisection end well before
-}
+enum { kStart, kDown, kUp, kBisect, kFinal };  // scale search phases
 
 template <int N, int D, int EPL, bool DITHER, bool F32IN>
 __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
@@ -561,6 +513,7 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kFixedWarps * TPW;
     constexpr int WPT = N / 64 > 0 ? N / 64 : 1;
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
     static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
     const uint32_t S = a.slot_words;
     const uint32_t istride = (S + 1 + 3) & ~3u;  // slot image + a guard word, 16-byte multiple
@@ -613,13 +566,54 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             const uint32_t c0 = tile_scale_bits(Ssq, a.c, nonfinite);
             if (nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
             const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
-            const uint32_t sb = fixed_scale<N, D, EPL, DITHER>(v, c0, budget, tkey, l, a.a2, mask, a.k_hint);
 
-            // ---- the chosen scale: quantize, Rice parameter, pack, store the slot
-            uint32_t u[EPL];
-            const uint32_t cbits = quantize_lane<D, EPL, DITHER>(v, sb, tkey, l, a.a2, u);
-            uint32_t part;
-            const int k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
+            // ---- scale search: one probe site (quantize + Rice parameter) serves
+            // every probe and the final pass; a state machine picks the next
+            // pattern.  When the search ends on the pattern just probed, that
+            // probe's symbols are the tile's and no final pass runs.
+            const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
+            const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
+            int phase = c0 ? kStart : kFinal, lo = 0, hi = (int)c0, step = 4, c = (int)c0;
+            uint32_t u[EPL], cbits, part;
+            int k;
+            for (int probe = 0;; probe++) {
+                cbits = quantize_lane<D, EPL, DITHER>(v, (uint32_t)c, tkey, l, a.a2, u);
+                k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
+                if (phase == kFinal) break;
+                const bool f = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part) <= budget;
+                if (phase == kStart) {
+                    if (f) { hi = c; phase = kDown; } else { lo = c; phase = kUp; }
+                } else if (phase == kDown) {
+                    if (f) { hi = c; step *= 2; } else { lo = c; phase = kBisect; }
+                } else if (phase == kUp) {
+                    if (f) { hi = c; phase = kBisect; } else { lo = c; step *= 2; }
+                } else {
+                    if (f) hi = c; else lo = c;
+                }
+                int next = -1, answer = -1;  // the next probe, or the search's answer
+                if (phase == kDown) {
+                    if (hi == lo_lim) answer = hi;
+                    else next = hi - step > lo_lim ? hi - step : lo_lim;
+                } else if (phase == kUp) {
+                    if (lo == hi_lim) answer = 0;  // no scale of the range fits: the all-zero tile
+                    else next = lo + step < hi_lim ? lo + step : hi_lim;
+                } else {
+                    if (hi - lo <= 1) answer = hi;
+                    else next = (lo + hi) >> 1;
+                }
+                if (answer < 0 && probe + 1 >= kFixedMaxProbes)  // not reached: the search ends well before
+                    answer = phase == kUp ? 0 : hi;
+                if (answer < 0) {
+                    c = next;
+                } else {
+                    if (answer == c && f) break;  // the last probe is the answer
+                    c = answer;
+                    phase = kFinal;
+                }
+            }
+            const uint32_t sb = (uint32_t)c;
+
+            // ---- pack the chosen symbols, store the slot
             const uint32_t uoff = group_excl_scan<LPT>(mask, part + EPL, l);
             for (uint32_t i = l; i < istride; i += LPT) img[i] = 0u;
             __syncwarp(mask);
