@@ -349,15 +349,19 @@ int hq_encode_noalloc(const void *x, int dtype, int64_t rows, int64_t cols, int 
  * version 1, flags, rows, cols, tile, lattice, bps, seed, ntiles,
  * payload_words, section offsets, FNV-1a 64-bit checksums of the body and of
  * the header), then tile_off (uint32 x ntiles + 1), tile_scale (uint16 x
- * ntiles), tile_k (uint8 x ntiles) and the payload (uint32 x payload_words). */
+ * ntiles), tile_k (uint8 x ntiles) and the payload (uint32 x payload_words).
+ * A fixed-rate stream (flags bit 1, slot_words in the header word after bps)
+ * has no tile_off section, its tile_k section holds the packed 4-bit k
+ * ((ntiles + 1) / 2 bytes) and its payload is ntiles x slot_words words. */
 typedef struct hq_file_info {
     int64_t rows, cols;
     int32_t tile, lattice;
     float bps;
-    uint32_t flags;          /* bit 0: KV stream (decode with dither) */
+    uint32_t flags;          /* bit 0: KV stream (decode with dither); bit 1: fixed-rate stream */
     uint64_t seed;
     uint64_t ntiles;         /* rows * cols / tile */
-    uint64_t payload_words;  /* tile_off[ntiles] */
+    uint64_t payload_words;  /* tile_off[ntiles]; fixed rate: ntiles * slot_words */
+    uint32_t slot_words;     /* fixed rate: the slot (hq_min_slot_words .. tile / 4); else 0 */
 } hq_file_info;
 
 /* Bytes of the container for `info`.  HQ_ERR_ARG if the fields are not a
@@ -365,14 +369,17 @@ typedef struct hq_file_info {
 int hq_file_bytes(const hq_file_info *info, uint64_t *out);
 
 /* Write the container into buf (host, >= hq_file_bytes).  tile_off must end
- * at payload_words.  HQ_ERR_CAPACITY if buf is too small. */
+ * at payload_words (fixed rate: tile_off is not read and may be NULL).
+ * HQ_ERR_CAPACITY if buf is too small. */
 int hq_file_write(const hq_file_info *info, const uint32_t *tile_off, const uint16_t *tile_scale,
                   const uint8_t *tile_k, const uint32_t *payload, void *buf, uint64_t buf_bytes);
 
 /* Check a container (magic, version, header and body checksums, section
  * layout, parameters, offsets non-decreasing from 0 to the payload size,
- * k <= 15) and return its info and pointers into buf (any pointer argument
- * may be NULL).  HQ_ERR_FORMAT for anything that does not check out. */
+ * k <= 15; fixed rate: a legal slot, payload = ntiles x slot, the unused
+ * half of an odd tile count's last k byte zero) and return its info and
+ * pointers into buf (any pointer argument may be NULL; *tile_off is NULL for
+ * a fixed-rate stream).  HQ_ERR_FORMAT for anything that does not check out. */
 int hq_file_read(const void *buf, uint64_t buf_bytes, hq_file_info *info, const uint32_t **tile_off,
                  const uint16_t **tile_scale, const uint8_t **tile_k, const uint32_t **payload);
 

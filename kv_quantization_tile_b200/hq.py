@@ -37,7 +37,8 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
 class hq_file_info(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("tile", ctypes.c_int32),
                 ("lattice", ctypes.c_int32), ("bps", ctypes.c_float), ("flags", ctypes.c_uint32),
-                ("seed", ctypes.c_uint64), ("ntiles", ctypes.c_uint64), ("payload_words", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("ntiles", ctypes.c_uint64), ("payload_words", ctypes.c_uint64),
+                ("slot_words", ctypes.c_uint32)]
 
 
 class hq_stream(ctypes.Structure):
@@ -381,18 +382,25 @@ def hq_encode_noalloc(x, tile, lattice, bps, seed, out: Stream, status=None, str
 def stream_to_bytes(s: Stream, rows: int, cols: int, tile: int, lattice, bps: float, seed: int,
                     dither: bool = False) -> bytes:
     """The checkpoint container of a stream (its arrays are copied to the host)."""
-    if s.slot_words:
-        raise ValueError("the checkpoint container holds variable-rate streams only")
-    off = s.tile_off.cpu().numpy().view(np.uint32)
-    words = int(off[-1])
     scale = s.tile_scale.cpu().numpy().view(np.uint16)
     kk = s.tile_k.cpu().numpy()
+    ntiles = rows * (cols // tile)
+    if s.slot_words:
+        off = None
+        words = ntiles * s.slot_words
+        flags = 2
+    else:
+        off = s.tile_off.cpu().numpy().view(np.uint32)
+        words = int(off[-1])
+        flags = 0
     pay = s.payload[:words].cpu().numpy().view(np.uint32)
-    info = hq_file_info(rows, cols, tile, _lat(lattice), bps, 1 if dither else 0, seed, off.size - 1, words)
+    info = hq_file_info(rows, cols, tile, _lat(lattice), bps, flags | (1 if dither else 0), seed, ntiles, words,
+                        s.slot_words)
     n = _u64(0)
     _check(_lib.hq_file_bytes(ctypes.byref(info), ctypes.byref(n)), "hq_file_bytes")
     buf = np.zeros(n.value, dtype=np.uint8)
-    _check(_lib.hq_file_write(ctypes.byref(info), off.ctypes.data, scale.ctypes.data if scale.size else None,
+    _check(_lib.hq_file_write(ctypes.byref(info), off.ctypes.data if off is not None else None,
+                              scale.ctypes.data if scale.size else None,
                               kk.ctypes.data if kk.size else None, pay.ctypes.data if pay.size else None,
                               buf.ctypes.data, buf.size), "hq_file_write")
     return buf.tobytes()
@@ -413,18 +421,20 @@ def stream_from_bytes(data: bytes, device="cuda") -> tuple[Stream, dict]:
         start = (p.value or base) - base
         return np.frombuffer(data, dtype=dtype, count=count, offset=start).copy()
 
-    off = view(ptrs[0], np.uint32, n + 1)
+    fixed = bool(info.flags & 2)
+    off = np.zeros(0, np.uint32) if fixed else view(ptrs[0], np.uint32, n + 1)
     scale = view(ptrs[1], np.uint16, n)
-    kk = view(ptrs[2], np.uint8, n)
+    kk = view(ptrs[2], np.uint8, (n + 1) // 2 if fixed else n)
     pay = view(ptrs[3], np.uint32, words)
     pay_t = torch.zeros(max(words, 1), dtype=torch.int32)
     pay_t[:words] = torch.from_numpy(pay.view(np.int32))
     stream = Stream(payload=pay_t.to(device), tile_off=torch.from_numpy(off.view(np.int32)).to(device),
                     tile_scale=torch.from_numpy(scale.view(np.int16)).to(device),
-                    tile_k=torch.from_numpy(kk).to(device))
+                    tile_k=torch.from_numpy(kk).to(device), slot_words=int(info.slot_words))
     names = {v: k for k, v in LATTICES.items()}
     meta = {"rows": int(info.rows), "cols": int(info.cols), "tile": int(info.tile), "lattice": names[info.lattice],
-            "bps": float(info.bps), "seed": int(info.seed), "dither": bool(info.flags & 1)}
+            "bps": float(info.bps), "seed": int(info.seed), "dither": bool(info.flags & 1),
+            "slot_words": int(info.slot_words)}
     return stream, meta
 
 

@@ -267,3 +267,26 @@ def test_fixed_round_trip_through_gpu_encode():
     # exact rate: slot words plus 20 bits of side information per tile
     ntiles = rows * cols // tile
     assert s.nbytes() == 4 * ntiles * slot + 2 * ntiles + (ntiles + 1) // 2
+
+
+def test_fixed_checkpoint_round_trip(tmp_path):
+    """GPU fixed-rate encode -> container file -> GPU decode is bit-identical
+    to decoding the stream straight from the encoder."""
+    rows, cols, tile, lat = 21, 768, 128, "E8"
+    slot = hq.hq_fixed_slot_words(tile, lat, 4.0)
+    x = make_input(rows, cols, 12)
+    s, st = gpu_encode_fixed(x, tile, lat, slot, 55, dither=True)
+    assert st == 0
+    path = str(tmp_path / "kv.hq")
+    hq.save_stream(path, s, rows, cols, tile, lat, 4.0, 55, dither=True)
+    s2, meta = hq.load_stream(path, DEV)
+    assert meta["slot_words"] == slot and meta["dither"]
+    outs = []
+    for stream in (s, s2):
+        y = torch.empty(rows, cols, dtype=torch.float32, device=DEV)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        hq.hq_kv_decode(stream, rows, cols, tile, lat, 4.0, 55, y, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        outs.append(y.cpu())
+    assert torch.equal(outs[0], outs[1])
