@@ -167,10 +167,11 @@ int hq_kv_encode(const void *x, int dtype, int64_t rows, int64_t cols, int tile,
  * gets a slot of S words, so its offset t S is implicit, k is kept in 4
  * bits, and the tile's only side information is the bf16 Delta and k (20
  * bits): (32 S + 20) / n bits per coordinate, exactly.  Delta is searched
- * per tile so the coded tile fits its slot: from the closed-form scale at
- * the rate 32 S / n - 5/32, steps of 4, 8, 16, ... bf16 patterns towards the
- * boundary (at most four octaves either way), then bisection, ending at a
- * fitting Delta whose next finer bf16 value does not fit.  A tile that fits
+ * per tile so the coded tile fits its slot: the size at the closed-form
+ * scale c0 (rate 32 S / n - 5/32) predicts a start (one bf16 step moves the
+ * size by about n / 128 bits), then steps of 1, 2, 4, ... bf16 patterns
+ * towards the boundary (within four octaves of c0), then bisection, ending
+ * at a fitting Delta whose next finer bf16 value does not fit.  A tile that fits
  * at no scale of that range (possible only with dither at very small slots)
  * is stored as the all-zero tile. */
 

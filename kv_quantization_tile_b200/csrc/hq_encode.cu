@@ -487,10 +487,11 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 // Fixed-rate tiles: every tile owns a slot of S words at word t S, so no
 // offsets are computed or stored and tiles are independent.  Per tile the
 // scale Delta is searched over bf16 bit patterns so that the coded tile fits
-// its slot: from the closed-form scale c0, steps of 4, 8, 16, ... patterns
+// its slot: the closed-form scale c0's size predicts a start (a pattern step
+// moves the size by about N / 128 bits), then steps of 1, 2, 4, ... patterns
 // towards the boundary (down while it fits, up until it fits; four octaves
-// at most either way), then bisection to a fitting scale whose next finer
-// pattern does not fit.  If no scale of the range fits, the tile is stored
+// from c0 at most either way), then bisection to a fitting scale whose next
+// finer pattern does not fit.  If no scale of the range fits, the tile is stored
 // as the all-zero tile, which a legal slot always holds.  Each probe
 // quantizes the rotated tile (held in registers) and prices it with the Rice
 // parameter search; the probe's size is group-uniform, so each group walks
@@ -505,7 +506,7 @@ constexpr int kFixedWarps = 8;
 // than 128 registers without spills (2 blocks) and no slower than 64 (4).
 constexpr int fixed_min_blocks(int epl) { return epl >= 32 ? 1 : 3; }
 constexpr int kFixedMaxProbes = 64;  // the search needs at most about 20
-enum { kStart, kDown, kUp, kBisect, kFinal };  // scale search phases
+enum { kPredict, kStart, kDown, kUp, kBisect, kFinal };  // scale search phases
 
 template <int N, int D, int EPL, bool DITHER, bool F32IN>
 __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
@@ -573,14 +574,27 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             // probe's symbols are the tile's and no final pass runs.
             const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
             const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
-            int phase = c0 ? kStart : kFinal, lo = 0, hi = (int)c0, step = 4, c = (int)c0;
+            int phase = c0 ? kPredict : kFinal, lo = 0, hi = (int)c0, step = 1, c = (int)c0;
             uint32_t u[EPL], cbits, part;
             int k;
             for (int probe = 0;; probe++) {
                 cbits = quantize_lane<D, EPL, DITHER>(v, (uint32_t)c, tkey, l, a.a2, u);
                 k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
                 if (phase == kFinal) break;
-                const bool f = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part) <= budget;
+                const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part);
+                const bool f = bits <= budget;
+                if (phase == kPredict) {
+                    // a pattern step moves the size by about N / 128 bits: start
+                    // from c0 + floor(128 (bits - budget) / N), clamped
+                    const int num = 128 * ((int)bits - (int)budget);
+                    const int shift = num >= 0 ? num / N : -((-num + N - 1) / N);
+                    const int start = c + shift < lo_lim ? lo_lim : (c + shift > hi_lim ? hi_lim : c + shift);
+                    phase = kStart;
+                    if (start != c) {
+                        c = start;
+                        continue;
+                    }
+                }
                 if (phase == kStart) {
                     if (f) { hi = c; phase = kDown; } else { lo = c; phase = kUp; }
                 } else if (phase == kDown) {

@@ -591,11 +591,15 @@ int hqo_decode_tile(const uint32_t *words, int nwords, int n, int lattice, uint1
  * numbers; 128 patterns per octave).  c0 = the closed-form scale at the
  * slot's rate.  Bounds: lo_lim = max(0x0080, c0 - 512), hi_lim = min(0x7F7F,
  * c0 + 512) (four octaves either way).
- *   c0 fits:  step down from c0 by 4, 8, 16, ... (clamped at lo_lim)
- *             while the candidate fits; the first that does not becomes lo
- *             (the last that fits is hi).  If lo_lim itself fits, the answer
- *             is lo_lim.
- *   otherwise: step up likewise from c0 (clamped at hi_lim) until a
+ *   Predict: one pattern step changes every coordinate's rate by 1/128 bit,
+ *             so the size moves by about n / 128 bits per step; from c0's
+ *             size b0 the start is s = c0 + floor(128 (b0 - budget) / n),
+ *             clamped to [lo_lim, hi_lim] (s = c0 reuses c0's size).
+ *   s fits:   step down from s by 1, 2, 4, ... (clamped at lo_lim) while
+ *             the candidate fits; the first that does not becomes lo (the
+ *             last that fits is hi).  If lo_lim itself fits, the answer is
+ *             lo_lim.
+ *   otherwise: step up likewise from s (clamped at hi_lim) until a
  *             candidate fits (hi; the last that did not is lo).  If hi_lim
  *             does not fit, the tile is stored as an all-zero tile
  *             (Delta = 0), which always fits a legal slot.
@@ -643,10 +647,22 @@ uint16_t hqo_fixed_scale(const float *v, int n, int lattice, uint16_t c0, uint64
     }
     int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
     int hi_lim = (int)c0 + 512 < 0x7F7F ? (int)c0 + 512 : 0x7F7F;
-    int lo, hi, step = 4;
+    int lo, hi, step = 1;
     tr++;
-    if (coded_bits(v, n, lattice, c0, seed, t, dither) <= budget_bits) {
-        hi = c0;
+    uint64_t b0 = coded_bits(v, n, lattice, c0, seed, t, dither);
+    int64_t num = 128 * ((int64_t)b0 - (int64_t)budget_bits);
+    int64_t shift = num >= 0 ? num / n : -((-num + n - 1) / n); /* floor(num / n) */
+    int64_t s64 = (int64_t)c0 + shift;
+    int start = s64 < lo_lim ? lo_lim : (s64 > hi_lim ? hi_lim : (int)s64);
+    int fits_start;
+    if (start == (int)c0) {
+        fits_start = b0 <= budget_bits;
+    } else {
+        tr++;
+        fits_start = coded_bits(v, n, lattice, (uint16_t)start, seed, t, dither) <= budget_bits;
+    }
+    if (fits_start) {
+        hi = start;
         for (;;) {
             if (hi == lo_lim) {
                 if (trials) *trials = tr;
@@ -663,7 +679,7 @@ uint16_t hqo_fixed_scale(const float *v, int n, int lattice, uint16_t c0, uint64
             }
         }
     } else {
-        lo = c0;
+        lo = start;
         for (;;) {
             if (lo == hi_lim) {
                 if (trials) *trials = tr;
