@@ -166,3 +166,44 @@ def test_every_tile_of_the_llama_and_kv_layers_is_bit_exact():
     print(f"{flipped} differing tiles of {total}")
     assert total == 851968 + 524288
     assert flipped == 0
+
+
+@pytest.mark.parametrize("case", ["llama_layer", "kv_layer"])
+def test_fixed_rate_full_size_sampled_tiles(case):
+    """Fixed-rate streams at full size (31-word slots for the Llama layer at
+    tile 256, 15-word slots for the dithered KV layer at tile 128): tiles are
+    independent, so the oracle re-encodes sampled tiles alone and their
+    slots, scales and packed Rice parameters must match bit for bit; sampled
+    decoded tiles match the oracle's decode of its own slots."""
+    if case == "llama_layer":
+        mats, tile, dither = [m for _, m in workloads.llama_layer(DEV)], 256, False
+    else:
+        mats, tile, dither = list(workloads.kv_layer(DEV)), 128, True
+    lat, seed = "E8", 42
+    slot = hq.hq_fixed_slot_words(tile, lat, 4.0)
+    for mi, x in enumerate(mats):
+        rows, cols = x.shape
+        ntiles = rows * (cols // tile)
+        s = hq.alloc_fixed_stream(rows, cols, tile, slot, DEV)
+        st = torch.zeros(1, dtype=torch.int32, device=DEV)
+        (hq.hq_kv_encode_fixed if dither else hq.hq_encode_fixed)(x, tile, lat, seed, s, st)
+        y = torch.empty(rows, cols, dtype=torch.float32, device=DEV)
+        (hq.hq_kv_decode if dither else hq.hq_decode)(s, rows, cols, tile, lat, 4.0, seed, y, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        tiles = sample_tiles(ntiles, 48, 7 * mi + tile, tile)
+        pay = s.payload.view(-1, slot)[torch.tensor(tiles, device=DEV)].cpu().numpy().view(np.uint32)
+        sc = s.tile_scale[torch.tensor(tiles, device=DEV)].cpu().numpy().view(np.uint16)
+        kp = s.tile_k.cpu().numpy()
+        tpr = cols // tile
+        for i, t in enumerate(tiles):
+            r, j = divmod(t, tpr)
+            e = oracle.encode_tile_fixed(tile_input(x, tile, t), lat, slot, seed, j=j, t=t, dither=dither)
+            assert e["scale"] == sc[i], (mi, t)
+            assert e["k"] == (kp[t >> 1] >> (4 * (t & 1))) & 15, (mi, t)
+            assert np.array_equal(e["slot"], pay[i]), (mi, t)
+            st1, ref = oracle.decode_tile(e["slot"][: e["words"]], tile, lat, e["scale"], e["k"], seed, j, t, dither)
+            assert st1 == 0
+            got = y[r, j * tile:(j + 1) * tile].cpu().numpy().astype(np.float64)
+            scale = np.abs(scipy.linalg.hadamard(tile) @ (oracle.signs(seed, j, tile) * ref)).max()
+            assert np.all(np.abs(got - ref) <= 1e-5 * scale + 1e-30), (mi, t)
