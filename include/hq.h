@@ -289,8 +289,10 @@ int hq_kv_attention_workspace_bytes(int64_t heads, int64_t tokens, int head_dim,
  * each stream, in fp32, without forming them: q is rotated once with the K
  * signs, scores come from the K stream's lattice points, and values are
  * accumulated in the rotated domain with one inverse rotation per query.
- *   k, v        streams written by hq_kv_encode of a (heads * tokens) x
- *               head_dim slab, tile = head_dim, with lattice, bps_k / bps_v
+ *   k, v        streams written by hq_kv_encode (or both by
+ *               hq_kv_encode_fixed; a variable-rate K with a fixed-rate V,
+ *               or the reverse, is HQ_ERR_UNSUPPORTED) of a (heads * tokens)
+ *               x head_dim slab, tile = head_dim, with lattice, bps_k / bps_v
  *               and seed_k / seed_v
  *   heads       KV heads (<= 65535), tokens >= 0 cached vectors per head
  *   head_dim    64, 128 or 256

@@ -524,6 +524,7 @@ int hq_kv_attention(const hq_stream *k, const hq_stream *v, int64_t heads, int64
     int rc = decode_common(k, heads * tokens, head_dim, head_dim, lattice, bps_k, seed_k, a.k, &nk);
     if (rc) return rc;
     if ((rc = decode_common(v, heads * tokens, head_dim, head_dim, lattice, bps_v, seed_v, a.v, &nv))) return rc;
+    if ((a.k.slot != 0) != (a.v.slot != 0)) return HQ_ERR_UNSUPPORTED;  // K and V of one kind
     if (heads == 0) return HQ_OK;
     cudaStream_t s = (cudaStream_t)stream;
     if (!out || !aligned(out, 16)) return HQ_ERR_ARG;

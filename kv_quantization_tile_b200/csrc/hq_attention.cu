@@ -73,7 +73,7 @@ __device__ __forceinline__ void block_reduce(float (&v)[GB], float *red)
 // the GB x n/32 column accumulators of head_dim 256 would spill.
 constexpr int attn_min_blocks(int n, int gb) { return n * gb >= 2048 ? 2 : (n == 256 && n * gb >= 1024 ? 3 : 4); }
 
-template <int N, int D, int EPL, int GB>
+template <int N, int D, int EPL, int GB, bool FIXED>
 __global__ void __launch_bounds__(kAttnThreads, attn_min_blocks(N, GB)) kv_attention_kernel(const AttnArgs a)
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kAttnWarps * TPW, C4 = EPL / 4;
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kAttnThreads, attn_min_blocks(N, GB)) kv_atten
         const int64_t tg = (int64_t)h * a.tokens + t0 + i;
         float pt[EPL];
         uint32_t sbits;
-        const bool bad = parse_tile<N, D, EPL>(a.k, tg, wbuf, mask, l, pt, sbits);
+        const bool bad = parse_tile<N, D, EPL, FIXED>(a.k, tg, wbuf, mask, l, pt, sbits);
         if (!bad && sbits) sub_dither<D, EPL>(mix64(a.k.dither_key ^ (uint64_t)tg), l, pt, a.k.a2);
         float dot[GB];
 #pragma unroll
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kAttnThreads, attn_min_blocks(N, GB)) kv_atten
             const int64_t tg = (int64_t)h * a.tokens + t0 + i;
             float pt[EPL];
             uint32_t sbits;
-            const bool bad = parse_tile<N, D, EPL>(a.v, tg, wbuf, mask, l, pt, sbits);
+            const bool bad = parse_tile<N, D, EPL, FIXED>(a.v, tg, wbuf, mask, l, pt, sbits);
             if (!bad && sbits) sub_dither<D, EPL>(mix64(a.v.dither_key ^ (uint64_t)tg), l, pt, a.v.a2);
             float4 *row = reinterpret_cast<float4 *>(zw + grp * N + l * EPL);
             const int sw = (l * U4 >> 3) & (U4 - 1);
@@ -383,7 +383,7 @@ cudaError_t launch_attention_t(AttnArgs a, int zchunks, cudaStream_t s)
 {
     constexpr int EPL = attn_epl<N, GB>();
     const uint32_t wmax = a.k.wmax > a.v.wmax ? a.k.wmax : a.v.wmax;
-    auto kern = kv_attention_kernel<N, D, EPL, GB>;
+    auto kern = a.k.slot ? kv_attention_kernel<N, D, EPL, GB, true> : kv_attention_kernel<N, D, EPL, GB, false>;
     const size_t smem_max = attn_smem<N, GB>(wmax, 4096 / GB);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
     if (e != cudaSuccess) return e;

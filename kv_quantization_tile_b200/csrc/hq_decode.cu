@@ -25,11 +25,10 @@ constexpr int kDecodeWarps = 8;
 
 }  // namespace
 
-template <int N, int D, int EPL, bool DITHER, bool F32OUT>
+template <int N, int D, int EPL, bool DITHER, bool F32OUT, bool FIXED>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeArgs a)
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kDecodeWarps * TPW;
-    constexpr int VPL = EPL / D;
     extern __shared__ __align__(16) uint32_t sm[];
     unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -42,7 +41,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     for (int64_t t = (int64_t)blockIdx.x * GPB + gid; t < a.ntiles; t += (int64_t)gridDim.x * GPB) {
         float pt[EPL];
         uint32_t sb;
-        const bool bad = parse_tile<N, D, EPL>(a, t, wbuf, mask, l, pt, sb);
+        const bool bad = parse_tile<N, D, EPL, FIXED>(a, t, wbuf, mask, l, pt, sb);
         if constexpr (DITHER) {
             if (!bad && sb) sub_dither<D, EPL>(mix64(a.dither_key ^ (uint64_t)t), l, pt, a.a2);
         }
@@ -77,7 +76,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     }
 }
 
-template <int N, int D, int EPL, int W>
+template <int N, int D, int EPL, int W, bool FIXED>
 __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(const DecodeArgs a)  // 64 registers up to 256
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = W * TPW;
@@ -125,7 +124,7 @@ __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(con
             const int64_t t = row * tpr + j;
             float pt[EPL];
             uint32_t sb;
-            const bool bad = parse_tile<N, D, EPL>(a, t, wbuf, mask, l, pt, sb);
+            const bool bad = parse_tile<N, D, EPL, FIXED>(a, t, wbuf, mask, l, pt, sb);
             const float4 *src = reinterpret_cast<const float4 *>(xt + j * N + l * EPL);
             float dot = 0.0f;
 #pragma unroll
@@ -176,7 +175,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
     constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
     const size_t smem = (size_t)a.sign_words * 8 + (size_t)GPB * group_words(a.wmax) * 4;
-    auto kern = decode_kernel<N, D, EPL, DITHER, F32OUT>;
+    auto kern = a.slot ? decode_kernel<N, D, EPL, DITHER, F32OUT, true> : decode_kernel<N, D, EPL, DITHER, F32OUT, false>;
     unsigned blocks = 0;
     cudaError_t e = grid_for(kern, smem, (a.ntiles + GPB - 1) / GPB, blocks);
     if (e != cudaSuccess) return e;
@@ -211,7 +210,7 @@ cudaError_t launch_gemv_w(const DecodeArgs &a, int64_t cols, cudaStream_t s)
 {
     constexpr int EPL = epl_for<N>(), GPB = W * (32 / (N / EPL));
     const size_t smem = (size_t)a.sign_words * 8 + (size_t)cols * 4 + (size_t)GPB * group_words(a.wmax) * 4;
-    auto kern = gemv_kernel<N, D, EPL, W>;
+    auto kern = a.slot ? gemv_kernel<N, D, EPL, W, true> : gemv_kernel<N, D, EPL, W, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaFuncAttributes fa{};

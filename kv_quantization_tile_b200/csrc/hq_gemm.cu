@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(256) rotate_x_kernel(const GemmArgs a)
 // TMEM accumulator and commits them to an mbarrier that the next tile's
 // writers wait on (bounded).  After an item's last tile, warps 0-3 read the
 // accumulator (row = TMEM lane) and store it.
-template <int D, int NB>
+template <int D, int NB, bool FIXED>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs a)
 {
     constexpr int N = kGemmN, EPL = 16, LPT = 16, TPW = 2, GPB = kGemmWarps * TPW;
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
                 uint32_t sb = 0;
                 bool bad = false;
                 if (r < a.rows) {
-                    bad = parse_tile<N, D, EPL>(a.w, r * a.tiles_per_row + j, wbuf, mask, l, pt, sb);
+                    bad = parse_tile<N, D, EPL, FIXED>(a.w, r * a.tiles_per_row + j, wbuf, mask, l, pt, sb);
                 } else {
 #pragma unroll
                     for (int i = 0; i < EPL; i++) pt[i] = 0.0f;
@@ -367,7 +367,7 @@ cudaError_t launch_gemm_t(GemmArgs a, cudaStream_t s)
 {
     const size_t smem = gemm_operand_bytes(kGemmM) + gemm_operand_bytes(NB) +
                         (size_t)kGemmWarps * 2 * group_words(a.w.wmax) * 4;
-    auto kern = gemm_tc_kernel<D, NB>;
+    auto kern = a.w.slot ? gemm_tc_kernel<D, NB, true> : gemm_tc_kernel<D, NB, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // Resident blocks per SM: the register limit of 512 threads x 64

@@ -16,10 +16,10 @@
 // (offsets out of order or past the capacity, k > 15, a scale that is not 0
 // or a positive normal bf16, a terminator count other than n, a word count
 // other than its bits need) parses to zeros and is reported as bad.
-// A fixed-rate stream (a.slot > 0) puts tile t at words [t S, t S + S) and
-// its k in 4 bits; the slot may end in zero words, so the last lane's span
-// ends at the last one bit of the slot (found by a max over the group)
-// rather than in the last word, and only the word-count rule is dropped.
+// A fixed-rate stream (FIXED, a.slot > 0) puts tile t at words [t S, t S + S) and
+// its k in 4 bits; the slot may end in zero words, so only the word-count
+// rule is dropped.  For both kinds the last lane's span ends at the last one
+// bit of the tile's words (a max over the group finds its word).
 #pragma once
 
 #include "hq_internal.h"
@@ -50,7 +50,7 @@ __device__ __forceinline__ uint32_t select_bit(uint32_t v, uint32_t r)
 
 // Parse tile t into lattice point coordinates pt (binary32).  Returns true
 // if the tile is not canonical (pt is then zero and sb is 0).
-template <int N, int D, int EPL>
+template <int N, int D, int EPL, bool FIXED>
 __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint32_t *wbuf,
                                            unsigned mask, int l, float (&pt)[EPL], uint32_t &sb)
 {
@@ -59,10 +59,10 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     constexpr int VPL = EPL / D;
     uint32_t *starts = wbuf + a.wmax + 4;
 
-    const bool fixed = a.slot != 0;
+    constexpr bool fixed = FIXED;  // the stream kind is a launch-time choice (a.slot != 0)
     uint32_t o0, o1;
     int k;
-    if (fixed) {
+    if constexpr (fixed) {
         o0 = (uint32_t)t * a.slot;  // the host keeps ntiles * slot below 2^32
         o1 = o0 + a.slot;
         k = (a.kk[t >> 1] >> ((t & 1) * 4)) & 15;
@@ -90,8 +90,7 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     // word holding terminator m*EPL - 1 yields lane m's start
     const uint32_t wu0 = U0 >> 5;
     const uint32_t nwu = W > wu0 ? W - wu0 : 0;  // unary words (the first shared with the low parts)
-    uint32_t found = 0, last_nz = 0;  // last_nz: 1 + the last unary word holding a one bit (fixed rate)
-    bool last_empty = false;
+    uint32_t found = 0, last_nz = 0;  // last_nz: 1 + the last unary word holding a one bit
     for (uint32_t wb = 0; wb < nwu; wb += LPT) {
         const uint32_t wi = wb + l;
         uint32_t v = wi < nwu ? wbuf[wu0 + wi] : 0u;
@@ -105,16 +104,15 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
         }
         if (wi < nwu) {
             const uint32_t before = found + incl - c, after = found + incl;
-            if (wi == nwu - 1 && c == 0) last_empty = true;  // padding after the last terminator
-            if (fixed && c) last_nz = wi + 1;
+            if (c) last_nz = wi + 1;
             for (uint32_t m = (before + EPL) / EPL; m < (uint32_t)LPT && m * EPL <= after; m++)
                 starts[m] = (wu0 + wi) * 32u + select_bit(v, m * EPL - 1u - before) + 1u - U0;
         }
         found += __shfl_sync(mask, incl, LPT - 1, LPT);
     }
-    const bool pad_word = __any_sync(mask, last_empty);
-    if (!bad && (found != (uint32_t)N || (pad_word && !fixed))) bad = true;
-    if (fixed) last_nz = group_max<LPT>(mask, last_nz);
+    last_nz = group_max<LPT>(mask, last_nz);
+    // a variable-rate tile ends in its last word (no whole word of padding)
+    if (!bad && (found != (uint32_t)N || (!fixed && last_nz != nwu))) bad = true;
     __syncwarp(mask);
 
 #pragma unroll
@@ -128,9 +126,9 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     // the next lane's start bounds this lane's codes
     uint32_t end = __shfl_down_sync(mask, start, 1, LPT);
     if (l == LPT - 1) {
-        // the word of the tile's last terminator: the last word, or for a
-        // fixed-rate slot the last unary word holding a one bit
-        const uint32_t wl = fixed ? wu0 + last_nz - 1u : W - 1u;
+        // the word of the tile's last terminator: the last unary word holding
+        // a one bit (the last word of a variable-rate tile)
+        const uint32_t wl = wu0 + last_nz - 1u;
         const uint32_t v = wbuf[wl] & (wl == wu0 ? (0xffffffffu << (U0 & 31)) : 0xffffffffu);
         end = wl * 32u + (31u - __clz(v)) + 1u - U0;
     }

@@ -197,3 +197,12 @@ def test_fixed_rate_sizing_and_validation():
     # variable-rate streams still need their offsets
     assert lib.hq_decode(ctypes.byref(hq.hq_stream(16, 1 << 20, 0, 16, 16, 0)), 4, 256, 256, 8, 4.0, 0, 16, 0,
                          None, None) == ARG
+
+
+def test_attention_needs_one_stream_kind():
+    lib = hq.library()
+    fixed = hq.hq_stream(16, 1 << 20, 0, 16, 16, 15)
+    var = hq.hq_stream(16, 1 << 20, 16, 16, 16, 0)
+    for k, v in ((fixed, var), (var, fixed)):
+        assert lib.hq_kv_attention(hq.ctypes.byref(k), hq.ctypes.byref(v), 2, 64, 128, 1, 8, 4.0, 4.0, 1, 2, 16, 0.1,
+                                   16, 16, 1 << 20, None, None) == hq.HQ_ERR_UNSUPPORTED
