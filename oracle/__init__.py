@@ -94,6 +94,10 @@ def lib() -> ctypes.CDLL:
                                                  vp, vp]),
                 "hqo_decode_tiles_fixed": (i32, [vp, u64, i32, vp, vp, i64, i32, i32, u64, i32, i64, i64,
                                                  vp]),
+                "hqo_act_quant_i8": (None, [vp, i32, u64, u64, vp, vp]),
+                "hqo_tile_points_i8": (i32, [vp, i32, i32, i32, i32, i32, vp, vp]),
+                "hqo_gemm_i8_rows": (i32, [vp, u64, vp, i32, vp, vp, i64, i32, i32, vp, vp, i64, i64, i64, vp,
+                                           vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -575,3 +579,76 @@ def decode_fixed(stream: dict, rows: int, cols: int, tile: int, lattice, seed: i
     for x in sts:
         st |= x
     return out, st
+
+
+# ---------------------------------------------------------------- int8 product
+def act_quant_i8(X, tile: int, seed: int):
+    """Rotated activations quantized per (batch row, column tile): returns
+    (Q int8 [batch, cols], S float32 [batch, cols // tile])."""
+    xa, dt = _as_bits(np.atleast_2d(X))
+    batch, cols = xa.shape
+    xf = (xa.astype(np.uint32) << 16).view(np.float32) if dt == 0 else xa.astype(np.float32)
+    xf = np.ascontiguousarray(xf)
+    tpr = cols // tile
+    Q = np.zeros((batch, cols), np.int8)
+    S = np.zeros((batch, tpr), np.float32)
+    L = lib()
+    q = np.zeros(tile, np.int8)
+    sc = ctypes.c_float(0)
+    for b in range(batch):
+        for j in range(tpr):
+            seg = np.ascontiguousarray(xf[b, j * tile:(j + 1) * tile])
+            L.hqo_act_quant_i8(_p(seg), tile, seed, j, _p(q), ctypes.byref(sc))
+            Q[b, j * tile:(j + 1) * tile] = q
+            S[b, j] = sc.value
+    return Q, S
+
+
+def tile_points_i8(words, n: int, lattice, k: int, exact: bool = True):
+    """(status, doubled lattice coordinates as int8 saturated to +-127, saturated count)."""
+    wa = np.ascontiguousarray(words, dtype=np.uint32)
+    a = np.zeros(n, np.int8)
+    sat = ctypes.c_int(0)
+    st = lib().hqo_tile_points_i8(_p(wa) if wa.size else 0, wa.size, n, _lat(lattice), k, int(exact), _p(a),
+                                  ctypes.byref(sat))
+    return st, a, sat.value
+
+
+def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X, threads: int = 1):
+    """The integer tensor-core product in binary64 (see hq_oracle.c): returns
+    (Y [batch, rows], status, saturated coordinates)."""
+    Q, S = act_quant_i8(X, tile, seed)
+    batch = Q.shape[0]
+    pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
+    cap = pay.size
+    if pay.size == 0:
+        pay = np.zeros(1, np.uint32)
+    ntiles = rows * (cols // tile)
+    if "slot" in stream:
+        off, slot, kk = None, int(stream["slot"]), np.ascontiguousarray(unpack_k(stream["kpack"], ntiles))
+    else:
+        off, slot, kk = np.ascontiguousarray(stream["off"], np.uint32), 0, np.ascontiguousarray(stream["k"], np.uint8)
+    sc = np.ascontiguousarray(stream["scale"], dtype=np.uint16)
+    L = lib()
+
+    def run(rg):
+        r0, r1 = rg
+        Y = np.zeros((batch, r1 - r0), np.float64)
+        sat = ctypes.c_int(0)
+        st = L.hqo_gemm_i8_rows(_p(pay), cap, _p(off) if off is not None else 0, slot, _p(sc), _p(kk), cols, tile,
+                                _lat(lattice), _p(Q), _p(S), batch, r0, r1, _p(Y), ctypes.byref(sat))
+        return r0, r1, Y, st, sat.value
+
+    ranges = _ranges(rows, threads * 4)
+    if threads > 1 and len(ranges) > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            parts = list(ex.map(run, ranges))
+    else:
+        parts = [run(rg) for rg in ranges]
+    Y = np.zeros((batch, rows), np.float64)
+    st = sat = 0
+    for r0, r1, y, s_, n_ in parts:
+        Y[:, r0:r1] = y
+        st |= s_
+        sat += n_
+    return Y, st, sat

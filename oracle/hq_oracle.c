@@ -882,6 +882,114 @@ int hqo_gemv_rows(const uint32_t *payload, uint64_t cap, const uint32_t *off, co
     return status;
 }
 
+/* ------------------------------------------------------------------ */
+/* Integer tensor-core product ([V1] abstract: the 8-bit MMA paths, int8
+ * ahead of fp8 on the lattice output after the rotation).  Reading: the
+ * doubled lattice coordinates 2y are integers for E8 (y in Z or Z + 1/2),
+ * D4 and Z, so A = 2y is exact in int8 while |2y| <= 127; A2's second
+ * coordinate carries sqrt3 and has no integer form.  The activations are
+ * rotated like the weights, x~ = H (s_j . x_bj) in binary32, and quantized
+ * per (batch row, column tile) to q = rint(x~ 127 / max|x~|) with scale
+ * s = max|x~| / 127 (all binary32, so q is decided exactly).  Then
+ *   Y[b][r] = sum_j Delta_rj s_bj / (2 n) sum_i A_rji q_bji.
+ * Coordinates with |2y| > 127 are saturated to +-127 and flagged. */
+
+/* q and s for one activation tile x (n binary32 values, column tile j). */
+void hqo_act_quant_i8(const float *x, int n, uint64_t seed, uint64_t j, int8_t *q, float *scale)
+{
+    float v[HQO_MAX_TILE];
+    float amax = 0.0f;
+    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * x[i];
+    hqo_fwht_f32(v, n);
+    for (int i = 0; i < n; i++)
+        if (fabsf(v[i]) > amax || isnan(v[i])) amax = isnan(v[i]) ? v[i] : fabsf(v[i]);
+    if (amax == 0.0f || !isfinite(amax)) {
+        for (int i = 0; i < n; i++) q[i] = 0;
+        *scale = amax;  /* 0, or the non-finite value, which then propagates */
+        return;
+    }
+    float inv = 127.0f / amax;
+    for (int i = 0; i < n; i++) q[i] = (int8_t)rintf(v[i] * inv);
+    *scale = amax / 127.0f;
+}
+
+/* Doubled lattice coordinates of one tile's points (E8, D4, Z): a[i] = 2 y_i
+ * saturated to [-127, 127]; *sat counts the saturated coordinates.  Returns
+ * the parse status (HQO_CORRUPT: a is zero). */
+int hqo_tile_points_i8(const uint32_t *words, int nwords, int n, int lattice, int k, int exact, int8_t *a,
+                       int *sat)
+{
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    int32_t z[8];
+    int d = lattice, nv = n / lattice;
+    int st = unpack_words(lattice, n, k, words, nwords, coset, u, exact);
+    if (st || lattice == 2) {
+        for (int i = 0; i < n; i++) a[i] = 0;
+        return st ? st : HQO_CORRUPT;
+    }
+    for (int q = 0; q < nv; q++) {
+        hqo_unsymbols(lattice, &u[q * d], z);
+        for (int m = 0; m < d; m++) {
+            int32_t v2 = 2 * z[m] + coset[q];
+            if (v2 > 127 || v2 < -127) {
+                (*sat)++;
+                v2 = v2 > 0 ? 127 : -127;
+            }
+            a[q * d + m] = (int8_t)v2;
+        }
+    }
+    return 0;
+}
+
+/* Y for rows [r0, r1) and all `batch` rows of X: Q (batch x cols int8) and
+ * S (batch x cols/n scales) from hqo_act_quant_i8; the stream is
+ * variable-rate (off != NULL) or fixed-rate (slot words, off == NULL) with
+ * one k per tile in kk.  Y is batch x (r1 - r0), binary64.  Returns the OR
+ * of the tile statuses; *sat gets the saturated coordinates. */
+int hqo_gemm_i8_rows(const uint32_t *payload, uint64_t cap, const uint32_t *off, int slot_words,
+                     const uint16_t *scale, const uint8_t *kk, int64_t cols, int n, int lattice, const int8_t *Q,
+                     const float *S, int64_t batch, int64_t r0, int64_t r1, double *Y, int *sat)
+{
+    int8_t a[HQO_MAX_TILE];
+    int64_t tpr = cols / n;
+    int status = 0;
+    for (int64_t r = r0; r < r1; r++) {
+        for (int64_t b = 0; b < batch; b++) Y[b * (r1 - r0) + (r - r0)] = 0.0;
+        for (int64_t j = 0; j < tpr; j++) {
+            int64_t t = r * tpr + j;
+            const uint32_t *w;
+            int nw;
+            if (off) {
+                if (off[t + 1] < off[t] || off[t + 1] > cap) {
+                    status |= HQO_CORRUPT;
+                    continue;
+                }
+                w = payload + off[t];
+                nw = (int)(off[t + 1] - off[t]);
+            } else {
+                if ((uint64_t)(t + 1) * (uint64_t)slot_words > cap) {
+                    status |= HQO_CORRUPT;
+                    continue;
+                }
+                w = payload + t * (int64_t)slot_words;
+                nw = slot_words;
+            }
+            int st = hqo_tile_points_i8(w, nw, n, lattice, kk[t], off != NULL, a, sat);
+            status |= st;
+            if (st) continue;
+            double delta = (double)bf16_to_float(scale[t]);
+            for (int64_t b = 0; b < batch; b++) {
+                int64_t dot = 0;
+                const int8_t *q = Q + b * cols + j * n;
+                for (int i = 0; i < n; i++) dot += (int64_t)a[i] * (int64_t)q[i];
+                Y[b * (r1 - r0) + (r - r0)] += delta * (double)S[b * tpr + j] / (2.0 * n) * (double)dot;
+            }
+        }
+    }
+    return status;
+}
+
 /* Nearest points of `count` vectors stored back to back (d floats each). */
 void hqo_nearest_batch(int lattice, const float *x, int64_t count, int32_t *c, int32_t *z,
                        float *pt)
