@@ -673,7 +673,27 @@ def fixed_leg(dev, peak):
     del ctx
     k, v = workloads.kv_layer(dev)
     ctx = run([k, v], 128, True, "kv_layer_e8")
-    del ctx, k, v
+    # attention of 32 query heads (4 per KV head) over the fixed-rate K and V streams
+    group, heads = 4, workloads.KV_HEADS
+    tokens = k.shape[0] // heads
+    q = torch.randn(heads * group, 128, generator=torch.Generator(device=dev).manual_seed(5), device=dev).to(torch.bfloat16)
+    out = torch.empty(heads * group, 128, dtype=torch.float32, device=dev)
+    aws = hq.alloc_attention_workspace(heads, tokens, 128, group, dev)
+    (_, ksf, _), (_, vsf, _) = ctx
+
+    def attend():
+        hq.hq_kv_attention(ksf, vsf, heads, tokens, 128, LAT, BPS, BPS, SEED, SEED, q, 128 ** -0.5, out, aws,
+                           group=group, status=st)
+
+    for _ in range(3):
+        attend()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    t = time_launches(attend, lambda: flush_l2(flushbuf))
+    nb = ksf.nbytes() + vsf.nbytes()
+    res["kv_attention_group4"] = {"us": round(t * 1e3, 2), "alg_gbs": round(nb / t / 1e6, 1),
+                                  "frac": round(nb / t / 1e6 / peak, 4), "compressed_bytes": nb}
+    del ctx, k, v, ksf, vsf
     w1, _, x1, _ = workloads.gemv_case(dev)
     r, c = w1.shape
     slot = hq.hq_fixed_slot_words(TILE, LAT, BPS)

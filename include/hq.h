@@ -48,7 +48,8 @@
  * too small: words past the capacity are not written), HQ_ST_CORRUPT (a
  * decoded tile is not a canonical tile: its output is zero), HQ_ST_TIMEOUT
  * (a bounded wait between thread blocks gave up: the call's output is
- * invalid).
+ * invalid), HQ_ST_RANGE (the integer product saturated a doubled lattice
+ * coordinate to +-127).
  *
  * The same seed must be given to encode and decode: signs and dither are
  * regenerated from it, not stored.
@@ -80,7 +81,7 @@ enum {
 };
 
 /* device status bits OR-ed into *d_status */
-enum { HQ_ST_NONFINITE = 1, HQ_ST_CAPACITY = 2, HQ_ST_CORRUPT = 4, HQ_ST_TIMEOUT = 8 };
+enum { HQ_ST_NONFINITE = 1, HQ_ST_CAPACITY = 2, HQ_ST_CORRUPT = 4, HQ_ST_TIMEOUT = 8, HQ_ST_RANGE = 16 };
 
 /* A compressed matrix.  Host struct; all pointers are device memory owned by
  * the caller.
@@ -257,6 +258,29 @@ int hq_decode_gemm_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, ui
 int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                    uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
                    uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
+/* Bytes of device workspace hq_decode_gemm_int8 needs: the quantized
+ * activations (int8, batch rounded up to the block's batch rows (at most 64)
+ * x cols, 256-byte rounded), their scales (fp32, padded batch x cols / 256),
+ * then fp32 split-K partials.  Host only; as hq_decode_gemm_workspace_bytes. */
+int hq_decode_gemm_int8_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, uint64_t *out);
+
+/* Batched decode + integer tensor-core product ([V1] abstract: 8-bit MMA
+ * paths, int8 ahead of fp8 on the lattice output after the rotation):
+ *   y[b][r] = sum_j Delta_rj s_bj / (2 n) sum_i A_rji q_bji
+ * with A = 2y, the doubled lattice coordinates (exact integers for E8, D4
+ * and Z; saturated to +-127 with HQ_ST_RANGE raised where they leave int8),
+ * and q_bj = rint(x~_bj 127 / max|x~_bj|), s_bj = max|x~_bj| / 127 the
+ * rotated activations x~_bj = H (s_j . x_bj) quantized per (batch row,
+ * column tile) in binary32.  The int32 sums over each column tile are exact
+ * (tcgen05.mma kind::i8, TMEM accumulator); scaling and the sum over column
+ * tiles are fp32.  The activation rounding makes this an approximation of
+ * X W_hat^T (each term moves by at most s_bj / 2).  Arguments as
+ * hq_decode_gemm; lattice HQ_A2 returns HQ_ERR_UNSUPPORTED (its points carry
+ * sqrt 3).  Non-finite activations give non-finite outputs. */
+int hq_decode_gemm_int8(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                        uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                        uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
 /* Testing hook for failure detection (no counterpart on the pages):
  * hq_decode_gemm in which column tile `stalled_tile` never issues or commits

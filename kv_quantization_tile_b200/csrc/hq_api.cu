@@ -445,13 +445,15 @@ namespace {
 
 int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                      uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
-                     uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stall_tile)
+                     uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stall_tile,
+                     bool int8 = false)
 {
     GemmArgs a{};
     int64_t ntiles = 0;
     int rc = decode_common(w, rows, cols, tile, lattice, bps, seed, a.w, &ntiles);
     if (rc) return rc;
     if (tile != 256) return HQ_ERR_UNSUPPORTED;
+    if (int8 && lattice == HQ_A2) return HQ_ERR_UNSUPPORTED;  // A2 points have no integer form
     if (batch < 0) return HQ_ERR_ARG;
     if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
     if (batch == 0 || rows == 0) return HQ_OK;
@@ -461,11 +463,17 @@ int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, i
         return cudaMemsetAsync(y, 0, sizeof(float) * (size_t)(batch * rows), s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     if (!x || !aligned(x, 16)) return HQ_ERR_ARG;
     GemmPlan p{};
-    gemm_plan(rows, cols, batch, 2, &p);  // workspace bound; the launch re-plans
+    if (int8) gemm_plan_i8(rows, cols, batch, 2, &p);  // workspace bound; the launch re-plans
+    else gemm_plan(rows, cols, batch, 2, &p);
     const uint64_t xt_span = (p.xt_bytes + 255) / 256 * 256;
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < xt_span + p.part_bytes) return HQ_ERR_WORKSPACE;
     a.x = static_cast<const uint16_t *>(x);
     a.xt = static_cast<uint16_t *>(workspace);
+    if (int8) {  // Q (batch_pad x cols int8, 256-byte rounded), then the scales
+        a.xq = static_cast<int8_t *>(workspace);
+        a.sx = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                         ((uint64_t)p.batch_pad * (uint64_t)cols + 255) / 256 * 256);
+    }
     a.y = y;
     a.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + xt_span);
     a.rows = rows;
@@ -479,6 +487,7 @@ int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, i
     a.sign_key = hash_key(seed, 1);
     a.status = d_status;
     a.stall_tile = stall_tile;
+    if (int8) return launch_gemm_i8(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     return launch_gemm(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -492,6 +501,24 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
 {
     return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
                             d_status, -1);
+}
+
+int hq_decode_gemm_int8_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, uint64_t *out)
+{
+    if (!out || rows < 0 || cols < 0 || batch < 0 || cols % 256) return HQ_ERR_ARG;
+    if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
+    GemmPlan p{};
+    gemm_plan_i8(rows, cols, batch, 2, &p);  // the most splits any launch picks
+    *out = (p.xt_bytes + 255) / 256 * 256 + p.part_bytes;
+    return HQ_OK;
+}
+
+int hq_decode_gemm_int8(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                        uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                        uint64_t workspace_bytes, void *stream, int32_t *d_status)
+{
+    return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
+                            d_status, -1, true);
 }
 
 int hq_test_gemm_stalled(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,

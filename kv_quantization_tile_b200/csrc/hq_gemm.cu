@@ -70,6 +70,28 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
         : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// kind::i8 instruction descriptor: s32 accumulator, signed 8-bit A and B,
+// both K-major, M x N.
+__host__ __device__ constexpr uint32_t make_idesc_i8(int m, int n)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// 8-bit operands: a 256-element row is 16 chunks of 16 bytes (same chunk
+// layout as the bf16 operands, half the chunks).
+__host__ __device__ constexpr uint32_t gemm_operand_bytes_i8(int rows) { return 16u * gemm_lbo(rows) * 16u; }
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t mbar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
@@ -332,6 +354,236 @@ __global__ void splitk_reduce_kernel(const GemmArgs a)
     }
 }
 
+// ------------------------------------------------------------ int8 product
+// The integer variant ([V1]: 8-bit MMA paths, int8 ahead of fp8 on the
+// lattice output after the rotation).  The doubled lattice coordinates 2y are
+// exact integers for E8 (y in Z or Z + 1/2), D4 and Z, so A = 2y in int8
+// (saturated to +-127, flagged); the activations, rotated like the weights,
+// are quantized per (batch row, column tile) to q = rint(x~ 127 / max|x~|)
+// with scale s = max|x~| / 127.  Per column tile the tensor cores form the
+// exact int32 sums A q; the epilogue scales them by Delta_rj s_bj / (2 n) and
+// accumulates in fp32:  Y[b][r] = sum_j Delta_rj s_bj / (2 n) sum_i A_rji q_bji.
+
+// Q[b][j n + i] and S[b][j] for b < batch_pad (zero for the padding rows).
+__global__ void __launch_bounds__(256) rotate_quant_x_kernel(const GemmArgs a)
+{
+    constexpr int N = kGemmN, EPL = 16, LPT = 16, GPB = 16;
+    const int lane = threadIdx.x & 31, l = lane % LPT;
+    const unsigned mask = group_mask<LPT>(lane);
+    const int64_t ntiles = (int64_t)a.batch_pad * a.tiles_per_row;
+    for (int64_t t = (int64_t)blockIdx.x * GPB + threadIdx.x / LPT; t < ntiles; t += (int64_t)gridDim.x * GPB) {
+        const int64_t b = t / a.tiles_per_row, j = t % a.tiles_per_row;
+        float v[EPL];
+        if (b < a.batch) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(a.x + b * a.cols + j * N + l * EPL);
+#pragma unroll
+            for (int i = 0; i < EPL / 8; i++) {
+                const uint4 q = __ldg(p + i);
+                const uint32_t qq[4] = { q.x, q.y, q.z, q.w };
+#pragma unroll
+                for (int h = 0; h < 4; h++) {
+                    v[8 * i + 2 * h] = __uint_as_float(qq[h] << 16);
+                    v[8 * i + 2 * h + 1] = __uint_as_float(qq[h] & 0xffff0000u);
+                }
+            }
+            const uint32_t i0 = (uint32_t)l * EPL;
+            const uint64_t w = mix64(mix64(a.sign_key ^ (uint64_t)j) ^ (uint64_t)(i0 >> 6));
+            const uint32_t sb = (uint32_t)(w >> (i0 & 63));
+#pragma unroll
+            for (int r = 0; r < EPL; r++) v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sb << (31 - r)) & 0x80000000u));
+            fwht<EPL, LPT>(v, mask, l);
+        } else {
+#pragma unroll
+            for (int r = 0; r < EPL; r++) v[r] = 0.0f;
+        }
+        // max |x~|: bit patterns of non-negative floats order like the values
+        // (a NaN above infinity, which then propagates through the scale)
+        uint32_t mb = 0;
+#pragma unroll
+        for (int r = 0; r < EPL; r++) mb = max(mb, __float_as_uint(fabsf(v[r])));
+        mb = __reduce_max_sync(mask, mb);
+        const float amax = __uint_as_float(mb);
+        uint32_t wq[4] = { 0u, 0u, 0u, 0u };
+        float scale = amax;
+        if (mb != 0u && mb < 0x7f800000u) {
+            const float inv = __fdiv_rn(127.0f, amax);
+#pragma unroll
+            for (int r = 0; r < EPL; r++) {
+                const int q = __float2int_rn(__fmul_rn(v[r], inv));  // |q| <= 127
+                wq[r >> 2] |= ((uint32_t)q & 0xffu) << (8 * (r & 3));
+            }
+            scale = __fdiv_rn(amax, 127.0f);
+        }
+        *reinterpret_cast<uint4 *>(a.xq + b * a.cols + j * N + l * EPL) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+        if (l == 0) a.sx[b * a.tiles_per_row + j] = scale;
+    }
+}
+
+// Work items as in gemm_tc_kernel.  Per column tile: every 16-lane group
+// parses rows into A (int8 2y, K-major) and keeps each row's Delta, all
+// threads copy Q into B and its scales, one thread issues 8 MMAs (K = 32
+// each) into an s32 TMEM accumulator.  After the MMAs of tile j complete,
+// warps 0-3 read the accumulator (row = TMEM lane), scale each sum by
+// Delta s / (2 n) and add it to the item's fp32 sums in shared memory while
+// the other warps parse tile j + 1 (the row and batch scales are double
+// buffered); the item's sums are stored after its last tile.
+template <int D, int NB, bool FIXED>
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs a)
+{
+    constexpr int N = kGemmN, EPL = 16, LPT = 16, TPW = 2, GPB = kGemmWarps * TPW;
+    constexpr uint32_t LBO_A = gemm_lbo(kGemmM) * 16u, LBO_B = gemm_lbo(NB) * 16u;
+    constexpr uint32_t NCOLS = NB < 32 ? 32u : (uint32_t)NB;
+    constexpr uint32_t IDESC = make_idesc_i8(kGemmM, NB);
+    static_assert(NB == 16 || NB == 32 || NB == 64, "int8 batch block");
+    extern __shared__ __align__(128) uint8_t smraw[];
+    uint8_t *sA = smraw;
+    uint8_t *sB = sA + gemm_operand_bytes_i8(kGemmM);
+    float *acc = reinterpret_cast<float *>(sB + gemm_operand_bytes_i8(NB));  // [NB][128] fp32 sums
+    float *dlt = acc + NB * kGemmM;                                          // [2][128] Delta per row
+    float *sxs = dlt + 2 * kGemmM;                                           // [2][NB] scale per batch row
+    uint32_t *wbase = reinterpret_cast<uint32_t *>(sxs + 2 * NB);
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int l = lane % LPT, gid = warp * TPW + lane / LPT;
+    const unsigned mask = group_mask<LPT>(lane);
+    uint32_t *wbuf = wbase + gid * group_words(a.w.wmax);
+    const uint32_t bar = smem_u32(&mbar);
+
+    if (warp == 0) tmem_alloc(smem_u32(&tmem_base), NCOLS);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t aA = smem_u32(sA), aB = smem_u32(sB);
+    const int64_t row_blocks = (a.rows + kGemmM - 1) / kGemmM, batch_blocks = a.batch_pad / NB;
+    const int64_t items = row_blocks * batch_blocks * a.ksplit;
+    constexpr float kInv2N = 1.0f / (2.0f * N);  // a power of two: exact
+
+    // warps 0-3: add tile buffer pb's scaled int32 sums to row `warp * 32 + lane`'s fp32 sums
+    auto epilogue = [&](int pb) {
+        const int row = warp * 32 + lane;
+        const float d = dlt[pb * kGemmM + row];
+#pragma unroll
+        for (int c = 0; c < NB; c += 16) {
+            float v[16];
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const float term = __fmul_rn(__fmul_rn(d, sxs[pb * NB + c + i]), (float)__float_as_int(v[i]));
+                acc[(c + i) * kGemmM + row] = __fadd_rn(acc[(c + i) * kGemmM + row], __fmul_rn(term, kInv2N));
+            }
+        }
+    };
+
+    uint32_t parity = 0;
+    bool fail = false, pending = false;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int ks = (int)(it % a.ksplit);
+        const int64_t rb = (it / a.ksplit) % row_blocks, bb = it / (a.ksplit * row_blocks);
+        const int64_t r0 = rb * kGemmM;
+        const int b0 = (int)bb * NB;
+        const int64_t j0 = (int64_t)ks * a.tiles_per_split;
+        const int64_t j1 = j0 + a.tiles_per_split < a.tiles_per_row ? j0 + a.tiles_per_split : a.tiles_per_row;
+        for (int e = tid; e < NB * kGemmM; e += kGemmThreads) acc[e] = 0.0f;
+        for (int64_t j = j0; j < j1; j++) {
+            const int pb = (int)((j - j0) & 1);
+            if (pending) {  // the previous tile's MMAs are complete: A and B are free, its sums readable
+                const bool ok = mbar_wait(bar, parity);
+                parity ^= 1u;
+                pending = false;
+                if (__syncthreads_or(!ok)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                if (warp < 4) epilogue(pb ^ 1);
+            }
+            // A: rows r0 .. r0 + 127 of column tile j; lane l holds K bytes 16 l .. 16 l + 15 (chunk l)
+            for (int m = gid; m < kGemmM; m += GPB) {
+                const int64_t r = r0 + m;
+                float pt[EPL];
+                uint32_t sb = 0;
+                bool bad = false;
+                if (r < a.rows) {
+                    bad = parse_tile<N, D, EPL, FIXED>(a.w, r * a.tiles_per_row + j, wbuf, mask, l, pt, sb);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < EPL; i++) pt[i] = 0.0f;
+                }
+                uint32_t wa[4] = { 0u, 0u, 0u, 0u };
+                bool sat = false;
+#pragma unroll
+                for (int i = 0; i < EPL; i++) {
+                    int v2 = __float2int_rn(2.0f * pt[i]);  // exact: 2y is an integer
+                    if (v2 > 127 || v2 < -127) {
+                        sat = true;
+                        v2 = v2 > 0 ? 127 : -127;
+                    }
+                    wa[i >> 2] |= ((uint32_t)v2 & 0xffu) << (8 * (i & 3));
+                }
+                *reinterpret_cast<uint4 *>(sA + (uint32_t)((m & 7) + 8 * (m >> 3)) * 16u + (uint32_t)l * LBO_A) =
+                    make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                if (l == 0) dlt[pb * kGemmM + m] = bf16_bits_to_float(sb);
+                if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
+                if (__any_sync(mask, sat) && l == 0 && a.status) atomicOr(a.status, kStatusRange);
+            }
+            // B: Q rows b0 .. b0 + NB - 1 of tile j, and their scales
+            for (int e = tid; e < NB * 16; e += kGemmThreads) {
+                const int n = e % NB, kc = e / NB;
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.xq + (int64_t)(b0 + n) * a.cols + j * N + kc * 16));
+                *reinterpret_cast<uint4 *>(sB + (uint32_t)((n & 7) + 8 * (n >> 3)) * 16u + (uint32_t)kc * LBO_B) = v;
+            }
+            for (int n = tid; n < NB; n += kGemmThreads) sxs[pb * NB + n] = a.sx[(int64_t)(b0 + n) * a.tiles_per_row + j];
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0 && j != a.stall_tile) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < N / 32; s++) {
+                    const uint64_t ad = make_smem_desc(aA + 2u * s * LBO_A, LBO_A, 128u);
+                    const uint64_t bd = make_smem_desc(aB + 2u * s * LBO_B, LBO_B, 128u);
+                    umma_i8(tmem, ad, bd, IDESC, s > 0 ? 1u : 0u);
+                }
+                umma_commit(bar);
+            }
+            pending = true;
+        }
+        if (pending) {
+            const bool ok = mbar_wait(bar, parity);
+            parity ^= 1u;
+            pending = false;
+            if (__syncthreads_or(!ok)) fail = true;
+            tc_fence_after();
+            if (!fail && warp < 4) epilogue((int)((j1 - 1 - j0) & 1));
+        }
+        // warps 0-3 store the sums of their rows (the threads that accumulated them)
+        if (warp < 4) {
+            const int64_t r = r0 + warp * 32 + lane;
+            for (int c = 0; c < NB; c++) {
+                const int b = b0 + c;
+                if (r < a.rows && b < a.batch) {
+                    const float val = fail ? 0.0f : acc[c * kGemmM + warp * 32 + lane];
+                    if (a.ksplit == 1) a.y[(int64_t)b * a.rows + r] = val;
+                    else a.part[((int64_t)ks * a.batch_pad + b) * a.rows + r] = val;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();  // sums stored and the accumulator read before the next item
+        tc_fence_after();
+        if (fail) break;
+    }
+    if (fail && tid == 0 && a.status) atomicOr(a.status, kStatusTimeout);
+    if (warp == 0) tmem_dealloc(tmem, NCOLS);
+}
+
 // ------------------------------------------------------------------ launch
 int gemm_block_batch(int64_t batch)
 {
@@ -357,6 +609,16 @@ void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, Gem
     p->tiles_per_split = (int)tps;
     p->ksplit = (int)(tpr > 0 ? (tpr + tps - 1) / tps : 1);
     p->xt_bytes = (uint64_t)p->batch_pad * (uint64_t)cols * 2;
+    p->part_bytes = p->ksplit > 1 ? (uint64_t)p->ksplit * (uint64_t)p->batch_pad * (uint64_t)rows * 4 : 0;
+}
+
+void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p)
+{
+    gemm_plan(rows, cols, batch < 64 ? batch : 64, blocks_per_sm, p);  // splits for one batch block of <= 64
+    p->batch_pad = (int)(((batch + p->nb - 1) / p->nb) * p->nb);
+    const int64_t tpr = cols / kGemmN;
+    const uint64_t q_bytes = ((uint64_t)p->batch_pad * (uint64_t)cols + 255) / 256 * 256;
+    p->xt_bytes = q_bytes + (uint64_t)p->batch_pad * (uint64_t)tpr * 4;
     p->part_bytes = p->ksplit > 1 ? (uint64_t)p->ksplit * (uint64_t)p->batch_pad * (uint64_t)rows * 4 : 0;
 }
 
@@ -426,6 +688,68 @@ cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s)
     case 2: return launch_gemm_d<2>(a, s);
     case 4: return launch_gemm_d<4>(a, s);
     default: return launch_gemm_d<8>(a, s);
+    }
+}
+
+namespace {
+
+template <int D, int NB>
+cudaError_t launch_gemm_i8_t(GemmArgs a, cudaStream_t s)
+{
+    const size_t smem = gemm_operand_bytes_i8(kGemmM) + gemm_operand_bytes_i8(NB) +
+                        ((size_t)NB * kGemmM + 2 * kGemmM + 2 * NB) * 4 +
+                        (size_t)kGemmWarps * 2 * group_words(a.w.wmax) * 4;
+    auto kern = a.w.slot ? gemm_i8_kernel<D, NB, true> : gemm_i8_kernel<D, NB, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    int dev = 0, smem_sm = 0, reserved = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+    int per_sm = (int)((size_t)smem_sm / (smem + 256 + (size_t)reserved));
+    if (per_sm > 2) per_sm = 2;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    GemmPlan p{};
+    gemm_plan_i8(a.rows, a.cols, a.batch, per_sm, &p);  // never more splits than the workspace holds
+    a.ksplit = p.ksplit;
+    a.tiles_per_split = p.tiles_per_split;
+    const int64_t items = ((a.rows + kGemmM - 1) / kGemmM) * (a.batch_pad / NB) * a.ksplit;
+    if (items >= ((int64_t)1 << 31)) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)(items > 0 ? items : 1), kGemmThreads, smem, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.ksplit == 1) return e;
+    int64_t n = (int64_t)a.batch * a.rows, blocks = (n + 255) / 256;
+    if (blocks > 8 * (int64_t)sm_count()) blocks = 8 * (int64_t)sm_count();
+    splitk_reduce_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_gemm_i8_d(const GemmArgs &a, cudaStream_t s)
+{
+    switch (a.nb) {
+    case 16: return launch_gemm_i8_t<D, 16>(a, s);
+    case 32: return launch_gemm_i8_t<D, 32>(a, s);
+    default: return launch_gemm_i8_t<D, 64>(a, s);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s)
+{
+    const int64_t xtiles = (int64_t)a.batch_pad * a.tiles_per_row;
+    int64_t rb = (xtiles + 15) / 16;
+    if (rb > 4 * (int64_t)sm_count()) rb = 4 * (int64_t)sm_count();
+    rotate_quant_x_kernel<<<(unsigned)(rb > 0 ? rb : 1), 256, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    switch (lattice) {
+    case 1: return launch_gemm_i8_d<1>(a, s);
+    case 4: return launch_gemm_i8_d<4>(a, s);
+    default: return launch_gemm_i8_d<8>(a, s);  // A2 has no integer form: refused by the host API
     }
 }
 

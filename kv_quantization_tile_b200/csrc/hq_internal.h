@@ -9,7 +9,7 @@
 
 namespace hq {
 
-constexpr int kStatusNonfinite = 1, kStatusCapacity = 2, kStatusCorrupt = 4, kStatusTimeout = 8;
+constexpr int kStatusNonfinite = 1, kStatusCapacity = 2, kStatusCorrupt = 4, kStatusTimeout = 8, kStatusRange = 16;
 
 // Look-back slot: bits 62..63 flag (1 = chunk aggregate, 2 = inclusive
 // prefix), bits 0..61 the word count.
@@ -94,6 +94,8 @@ struct GemmArgs {
     DecodeArgs w;               // weight stream, rows x cols
     const uint16_t *x;          // bf16 [batch][cols]
     uint16_t *xt;               // bf16 [batch_pad][cols]: rotated activations (workspace)
+    int8_t *xq;                 // int8 product: quantized rotated activations [batch_pad][cols] (workspace)
+    float *sx;                  // int8 product: their scales [batch_pad][tiles_per_row] (workspace)
     float *y;                   // fp32 [batch][rows]
     float *part;                // fp32 [ksplit][batch_pad][rows] split-K partials (workspace)
     int64_t rows, cols, tiles_per_row;
@@ -106,7 +108,7 @@ struct GemmArgs {
 
 struct GemmPlan {
     int nb, batch_pad, ksplit, tiles_per_split;
-    uint64_t xt_bytes, part_bytes;  // workspace: X~, then the partials
+    uint64_t xt_bytes, part_bytes;  // workspace: X~ (int8 product: Q, then the scales), then the partials
 };
 
 // Launch helpers; return a cudaError_t.
@@ -121,6 +123,10 @@ cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s);
 // Plan for blocks_per_sm resident blocks; the launch re-plans from the
 // kernel's occupancy (never more splits than for two blocks per SM).
 void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
+// The integer product (A = 2y in int8, activations quantized to int8):
+// batch blocks of at most 64 rows; same splitting rule.
+void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
+cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s);
 // Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
 cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 

@@ -23,7 +23,7 @@ if not os.path.exists(_LIB_PATH):
 HQ_Z, HQ_A2, HQ_D4, HQ_E8 = 1, 2, 4, 8
 HQ_BF16, HQ_F32 = 0, 1
 HQ_OK, HQ_ERR_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_CAPACITY, HQ_ERR_WORKSPACE, HQ_ERR_CUDA, HQ_ERR_FORMAT = range(7)
-HQ_ST_NONFINITE, HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT = 1, 2, 4, 8
+HQ_ST_NONFINITE, HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT, HQ_ST_RANGE = 1, 2, 4, 8, 16
 LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 
 EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_words",
@@ -31,7 +31,8 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_decode", "hq_kv_decode", "hq_decode_gemv", "hq_encode_noalloc", "hq_test_encode_stalled",
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
            "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled",
-           "hq_min_slot_words", "hq_fixed_slot_words", "hq_encode_fixed", "hq_kv_encode_fixed"]
+           "hq_min_slot_words", "hq_fixed_slot_words", "hq_encode_fixed", "hq_kv_encode_fixed",
+           "hq_decode_gemm_int8_workspace_bytes", "hq_decode_gemm_int8"]
 
 
 class hq_file_info(ctypes.Structure):
@@ -82,6 +83,9 @@ _SIGS = {
     "hq_fixed_slot_words": (_i32, [_i32, _i32, _f32, ctypes.POINTER(ctypes.c_uint32)]),
     "hq_encode_fixed": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _u64, ctypes.POINTER(hq_stream), _vp, _vp]),
     "hq_kv_encode_fixed": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _u64, ctypes.POINTER(hq_stream), _vp, _vp]),
+    "hq_decode_gemm_int8_workspace_bytes": (_i32, [_i64, _i64, _i64, ctypes.POINTER(_u64)]),
+    "hq_decode_gemm_int8": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
+                                   _u64, _vp, _vp]),
     "hq_decode_gemm": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
                               _u64, _vp, _vp]),
     "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
@@ -322,6 +326,31 @@ def hq_decode_gemm(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, worksp
     _check(_lib.hq_decode_gemm(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch, _ptr(y),
                                _ptr(workspace), workspace.numel(), _stream_handle(stream), _ptr(status)),
            "hq_decode_gemm")
+    return y
+
+
+def hq_decode_gemm_int8_workspace_bytes(rows: int, cols: int, batch: int) -> int:
+    out = _u64(0)
+    _check(_lib.hq_decode_gemm_int8_workspace_bytes(rows, cols, batch, ctypes.byref(out)),
+           "hq_decode_gemm_int8_workspace_bytes")
+    return out.value
+
+
+def alloc_gemm_int8_workspace(rows: int, cols: int, batch: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(hq_decode_gemm_int8_workspace_bytes(rows, cols, batch), 16), dtype=torch.uint8,
+                       device=device)
+
+
+def hq_decode_gemm_int8(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, workspace, status=None, stream=None):
+    """Y = X W_hat^T on the integer tensor cores: A = 2y in int8, the rotated
+    activations quantized to int8 per (row, column tile); y is fp32 [batch, rows]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == cols
+    batch = x.shape[0]
+    assert y.dtype == torch.float32 and y.is_contiguous() and y.numel() == batch * rows
+    st = s.struct()
+    _check(_lib.hq_decode_gemm_int8(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch,
+                                    _ptr(y), _ptr(workspace), workspace.numel(), _stream_handle(stream),
+                                    _ptr(status)), "hq_decode_gemm_int8")
     return y
 
 

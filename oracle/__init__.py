@@ -614,9 +614,12 @@ def tile_points_i8(words, n: int, lattice, k: int, exact: bool = True):
     return st, a, sat.value
 
 
-def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X, threads: int = 1):
-    """The integer tensor-core product in binary64 (see hq_oracle.c): returns
-    (Y [batch, rows], status, saturated coordinates)."""
+def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X, threads: int = 1,
+            r0: int = 0, r1: int | None = None):
+    """The integer tensor-core product in binary64 (see hq_oracle.c) for
+    weight rows [r0, r1): returns (Y [batch, r1 - r0], status, saturated
+    coordinates)."""
+    r1 = rows if r1 is None else r1
     Q, S = act_quant_i8(X, tile, seed)
     batch = Q.shape[0]
     pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
@@ -639,16 +642,16 @@ def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X
                                 _lat(lattice), _p(Q), _p(S), batch, r0, r1, _p(Y), ctypes.byref(sat))
         return r0, r1, Y, st, sat.value
 
-    ranges = _ranges(rows, threads * 4)
+    ranges = [(a + r0, b + r0) for a, b in _ranges(r1 - r0, threads * 4)]
     if threads > 1 and len(ranges) > 1:
         with ThreadPoolExecutor(threads) as ex:
             parts = list(ex.map(run, ranges))
     else:
         parts = [run(rg) for rg in ranges]
-    Y = np.zeros((batch, rows), np.float64)
+    Y = np.zeros((batch, r1 - r0), np.float64)
     st = sat = 0
-    for r0, r1, y, s_, n_ in parts:
-        Y[:, r0:r1] = y
+    for a, b, y, s_, n_ in parts:
+        Y[:, a - r0:b - r0] = y
         st |= s_
         sat += n_
     return Y, st, sat

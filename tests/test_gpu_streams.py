@@ -74,3 +74,42 @@ def test_two_streams_at_once():
             g = fetch(s)
             for key in ("off", "scale", "k", "payload"):
                 assert np.array_equal(g[key], r[key]), key
+
+
+def test_fixed_rate_graph_capture_and_replay():
+    """Fixed-rate KV encode + attention over the fixed-rate streams, captured
+    in a CUDA graph: replays reproduce the eager results bit for bit."""
+    heads, tokens, d, lat, group = 2, 640, 128, "E8", 4
+    g = torch.Generator().manual_seed(4)
+    k = torch.randn(heads * tokens, d, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(heads * tokens, d, generator=g).to(torch.bfloat16).to(DEV)
+    q = torch.randn(heads * group, d, generator=g).to(torch.bfloat16).to(DEV)
+    slot = hq.hq_fixed_slot_words(d, lat, 4.0)
+    ks = hq.alloc_fixed_stream(heads * tokens, d, d, slot, DEV)
+    vs = hq.alloc_fixed_stream(heads * tokens, d, d, slot, DEV)
+    ws = hq.alloc_attention_workspace(heads, tokens, d, group, DEV)
+    out = torch.empty(heads * group, d, dtype=torch.float32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+
+    def step():
+        hq.hq_kv_encode_fixed(k, d, lat, 7, ks, st)
+        hq.hq_kv_encode_fixed(v, d, lat, 8, vs, st)
+        hq.hq_kv_attention(ks, vs, heads, tokens, d, lat, 4.0, 4.0, 7, 8, q, 0.1, out, ws, group=group, status=st)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    eager = (ks.payload.clone(), ks.tile_k.clone(), vs.payload.clone(), out.clone())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(2):
+        ks.payload.zero_(); vs.payload.zero_(); ks.tile_k.zero_(); out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(ks.payload, eager[0]) and torch.equal(ks.tile_k, eager[1])
+        assert torch.equal(vs.payload, eager[2]) and torch.equal(out, eager[3])
+    assert int(st.item()) == 0
