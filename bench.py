@@ -519,9 +519,14 @@ def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
         x = torch.randn(batch, c, generator=g, device=dev).to(torch.bfloat16)
         y = torch.empty(batch, r, dtype=torch.float32, device=dev)
         ws = hq.alloc_gemm_workspace(r, c, batch, dev)
+        ws8 = hq.alloc_gemm_int8_workspace(r, c, batch, dev)
+        y8 = torch.empty(batch, r, dtype=torch.float32, device=dev)
 
         def ours():
             hq.hq_decode_gemm(s, r, c, TILE, LAT, BPS, SEED, x, y, ws, st)
+
+        def ours_int8():
+            hq.hq_decode_gemm_int8(s, r, c, TILE, LAT, BPS, SEED, x, y8, ws8, st)
 
         def dense():
             torch.matmul(x, w1.t())
@@ -531,16 +536,22 @@ def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
             torch.matmul(x, wd.t())
 
         for _ in range(3):
-            ours(); dense(); decode_then_dense()
+            ours(); ours_int8(); dense(); decode_then_dense()
         torch.cuda.synchronize()
         assert int(st.item()) == 0
+        ref = (x.float() @ wd.float().t())  # the bf16 decode's product, for the int8 path's error
+        rel8 = float((y8 - ref).norm() / ref.norm())
+        rel16 = float((y - ref).norm() / ref.norm())
+        t8 = time_launches(ours_int8, lambda: flush_l2(flushbuf))
         t = time_launches(ours, lambda: flush_l2(flushbuf))
         td = time_launches(dense, lambda: flush_l2(flushbuf))
         tdd = time_launches(decode_then_dense, lambda: flush_l2(flushbuf))
         flops = 2.0 * batch * r * c
         res[f"batch{batch}"] = {"us": round(t * 1e3, 2), "tflops": round(flops / t / 1e9, 2),
                                 "weights_per_us": round(r * c / t / 1e3, 1),
-                                "bf16_cublas_us": round(td * 1e3, 2), "decode_then_cublas_us": round(tdd * 1e3, 2)}
+                                "bf16_cublas_us": round(td * 1e3, 2), "decode_then_cublas_us": round(tdd * 1e3, 2),
+                                "int8_us": round(t8 * 1e3, 2), "int8_rel_err": round(rel8, 5),
+                                "bf16_rel_err": round(rel16, 5)}
     return res
 
 
