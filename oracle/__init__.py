@@ -98,6 +98,11 @@ def lib() -> ctypes.CDLL:
                 "hqo_tile_points_i8": (i32, [vp, i32, i32, i32, i32, i32, vp, vp]),
                 "hqo_gemm_i8_rows": (i32, [vp, u64, vp, i32, vp, vp, i64, i32, i32, vp, vp, i64, i64, i64, vp,
                                            vp]),
+                "hqo_e4m3": (ctypes.c_uint8, [f32]),
+                "hqo_e4m3_value": (f32, [ctypes.c_uint8]),
+                "hqo_act_quant_e4m3": (None, [vp, i32, u64, u64, vp, vp]),
+                "hqo_gemm_e4m3_rows": (i32, [vp, u64, vp, i32, vp, vp, i64, i32, i32, vp, vp, i64, i64, i64, vp,
+                                             vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -619,8 +624,53 @@ def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X
     """The integer tensor-core product in binary64 (see hq_oracle.c) for
     weight rows [r0, r1): returns (Y [batch, r1 - r0], status, saturated
     coordinates)."""
-    r1 = rows if r1 is None else r1
     Q, S = act_quant_i8(X, tile, seed)
+    return _lowbit_product("hqo_gemm_i8_rows", Q, S, stream, rows, cols, tile, lattice, threads, r0, r1)
+
+
+def e4m3(x) -> np.ndarray:
+    """OCP FP8 E4M3 bits of binary32 values (round to nearest even, saturating)."""
+    xa = np.asarray(x, np.float32).ravel()
+    L = lib()
+    return np.array([L.hqo_e4m3(float(v)) for v in xa], np.uint8).reshape(np.shape(x))
+
+
+def e4m3_value(b) -> np.ndarray:
+    ba = np.asarray(b, np.uint8).ravel()
+    L = lib()
+    return np.array([L.hqo_e4m3_value(int(v)) for v in ba], np.float32).reshape(np.shape(b))
+
+
+def act_quant_e4m3(X, tile: int, seed: int):
+    """Rotated activations scaled per (batch row, column tile) to +-448 and
+    rounded to E4M3: (Q bits uint8 [batch, cols], S float32 [batch, cols // tile])."""
+    xa, dt = _as_bits(np.atleast_2d(X))
+    batch, cols = xa.shape
+    xf = np.ascontiguousarray((xa.astype(np.uint32) << 16).view(np.float32) if dt == 0 else xa.astype(np.float32))
+    tpr = cols // tile
+    Q = np.zeros((batch, cols), np.uint8)
+    S = np.zeros((batch, tpr), np.float32)
+    L = lib()
+    q = np.zeros(tile, np.uint8)
+    sc = ctypes.c_float(0)
+    for b in range(batch):
+        for j in range(tpr):
+            seg = np.ascontiguousarray(xf[b, j * tile:(j + 1) * tile])
+            L.hqo_act_quant_e4m3(_p(seg), tile, seed, j, _p(q), ctypes.byref(sc))
+            Q[b, j * tile:(j + 1) * tile] = q
+            S[b, j] = sc.value
+    return Q, S
+
+
+def gemm_e4m3(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X, threads: int = 1,
+              r0: int = 0, r1: int | None = None):
+    """The fp8 (E4M3) tensor-core product in binary64 (see hq_oracle.c)."""
+    Q, S = act_quant_e4m3(X, tile, seed)
+    return _lowbit_product("hqo_gemm_e4m3_rows", Q, S, stream, rows, cols, tile, lattice, threads, r0, r1)
+
+
+def _lowbit_product(fn_name, Q, S, stream, rows, cols, tile, lattice, threads, r0, r1):
+    r1 = rows if r1 is None else r1
     batch = Q.shape[0]
     pay = np.ascontiguousarray(stream["payload"], dtype=np.uint32)
     cap = pay.size
@@ -638,8 +688,8 @@ def gemm_i8(stream: dict, rows: int, cols: int, tile: int, lattice, seed: int, X
         r0, r1 = rg
         Y = np.zeros((batch, r1 - r0), np.float64)
         sat = ctypes.c_int(0)
-        st = L.hqo_gemm_i8_rows(_p(pay), cap, _p(off) if off is not None else 0, slot, _p(sc), _p(kk), cols, tile,
-                                _lat(lattice), _p(Q), _p(S), batch, r0, r1, _p(Y), ctypes.byref(sat))
+        st = getattr(L, fn_name)(_p(pay), cap, _p(off) if off is not None else 0, slot, _p(sc), _p(kk), cols, tile,
+                                 _lat(lattice), _p(Q), _p(S), batch, r0, r1, _p(Y), ctypes.byref(sat))
         return r0, r1, Y, st, sat.value
 
     ranges = [(a + r0, b + r0) for a, b in _ranges(r1 - r0, threads * 4)]

@@ -990,6 +990,130 @@ int hqo_gemm_i8_rows(const uint32_t *payload, uint64_t cap, const uint32_t *off,
     return status;
 }
 
+/* ------------------------------------------------------------------ */
+/* fp8 tensor-core product ([V1] abstract: the fp8-e4m3 MMA path, which the
+ * pages find behind int8 on the lattice output).  Same construction as the
+ * integer product with both operands in OCP FP8 E4M3 (1 sign, 4 exponent
+ * bits with bias 7, 3 mantissa bits, subnormals, no infinity, largest
+ * finite 448, NaN = S.1111.111): A = e4m3(2y) -- exact only while |2y| <= 16
+ * or on the format's coarser grid beyond -- and q = e4m3(x~ 448 / max|x~|),
+ * s = max|x~| / 448.  Conversion rounds to nearest, ties to even, and
+ * saturates finite values to +-448. */
+
+/* binary32 -> E4M3 bits, round to nearest even, saturating (NaN -> 0x7F). */
+uint8_t hqo_e4m3(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;  /* 448 or above (ties at 464 would round up past the largest) */
+    int e;
+    if (a < 0x1p-6) {
+        e = -6;  /* subnormal range: quantum 2^-9 */
+    } else {
+        e = (int)floor(log2(a));
+        if (ldexp(1.0, e) > a) e--;  /* guard the log against rounding */
+        if (ldexp(1.0, e + 1) <= a) e++;
+    }
+    double quantum = ldexp(1.0, e - 3);
+    double m = a / quantum;  /* exact: a power-of-two scale */
+    double r = floor(m);
+    double frac = m - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double v = r * quantum;  /* the rounded magnitude */
+    if (v >= 448.0) return sign | 0x7E;
+    if (v < 0x1p-6) return sign | (uint8_t)(v / 0x1p-9);  /* subnormal: exponent field 0 */
+    int ev;
+    double mant = frexp(v, &ev);  /* v = mant 2^ev, mant in [0.5, 1) */
+    int E = ev - 1;               /* v = 1.f 2^E */
+    int f = (int)((mant * 2.0 - 1.0) * 8.0);
+    return sign | (uint8_t)(((E + 7) << 3) | f);
+}
+
+float hqo_e4m3_value(uint8_t b)
+{
+    int s = b >> 7, E = (b >> 3) & 15, f = b & 7;
+    if (E == 15 && f == 7) return NAN;
+    double v = E == 0 ? ldexp((double)f, -9) : ldexp(1.0 + f / 8.0, E - 7);
+    return (float)(s ? -v : v);
+}
+
+/* q (E4M3 bits) and s for one activation tile x (column tile j). */
+void hqo_act_quant_e4m3(const float *x, int n, uint64_t seed, uint64_t j, uint8_t *q, float *scale)
+{
+    float v[HQO_MAX_TILE];
+    float amax = 0.0f;
+    for (int i = 0; i < n; i++) v[i] = (float)hqo_sign(seed, j, (uint32_t)i) * x[i];
+    hqo_fwht_f32(v, n);
+    for (int i = 0; i < n; i++)
+        if (fabsf(v[i]) > amax || isnan(v[i])) amax = isnan(v[i]) ? v[i] : fabsf(v[i]);
+    if (amax == 0.0f || !isfinite(amax)) {
+        for (int i = 0; i < n; i++) q[i] = 0;
+        *scale = amax;
+        return;
+    }
+    float inv = 448.0f / amax;
+    for (int i = 0; i < n; i++) q[i] = hqo_e4m3(v[i] * inv);
+    *scale = amax / 448.0f;
+}
+
+/* Y for rows [r0, r1): as hqo_gemm_i8_rows with A = e4m3(2y) (saturated to
+ * +-448 and counted in *sat) and Q holding E4M3 bits; the products of E4M3
+ * values are summed exactly in binary64. */
+int hqo_gemm_e4m3_rows(const uint32_t *payload, uint64_t cap, const uint32_t *off, int slot_words,
+                       const uint16_t *scale, const uint8_t *kk, int64_t cols, int n, int lattice,
+                       const uint8_t *Q, const float *S, int64_t batch, int64_t r0, int64_t r1, double *Y, int *sat)
+{
+    uint32_t u[HQO_MAX_TILE];
+    uint8_t coset[HQO_MAX_TILE];
+    double a[HQO_MAX_TILE];
+    int32_t z[8];
+    int64_t tpr = cols / n;
+    int status = 0, d = lattice, nv = n / lattice;
+    for (int64_t r = r0; r < r1; r++) {
+        for (int64_t b = 0; b < batch; b++) Y[b * (r1 - r0) + (r - r0)] = 0.0;
+        for (int64_t j = 0; j < tpr; j++) {
+            int64_t t = r * tpr + j;
+            const uint32_t *w;
+            int nw;
+            if (off) {
+                if (off[t + 1] < off[t] || off[t + 1] > cap) {
+                    status |= HQO_CORRUPT;
+                    continue;
+                }
+                w = payload + off[t];
+                nw = (int)(off[t + 1] - off[t]);
+            } else {
+                if ((uint64_t)(t + 1) * (uint64_t)slot_words > cap) {
+                    status |= HQO_CORRUPT;
+                    continue;
+                }
+                w = payload + t * (int64_t)slot_words;
+                nw = slot_words;
+            }
+            int st = lattice == 2 ? HQO_CORRUPT : unpack_words(lattice, n, kk[t], w, nw, coset, u, off != NULL);
+            status |= st;
+            if (st) continue;
+            for (int q = 0; q < nv; q++) {
+                hqo_unsymbols(lattice, &u[q * d], z);
+                for (int m = 0; m < d; m++) {
+                    float v2 = (float)(2 * z[m] + coset[q]);
+                    if (fabsf(v2) > 448.0f) (*sat)++;
+                    a[q * d + m] = (double)hqo_e4m3_value(hqo_e4m3(v2));
+                }
+            }
+            double delta = (double)bf16_to_float(scale[t]);
+            for (int64_t b = 0; b < batch; b++) {
+                double dot = 0.0;
+                const uint8_t *qq = Q + b * cols + j * n;
+                for (int i = 0; i < n; i++) dot += a[i] * (double)hqo_e4m3_value(qq[i]);
+                Y[b * (r1 - r0) + (r - r0)] += delta * (double)S[b * tpr + j] / (2.0 * n) * dot;
+            }
+        }
+    }
+    return status;
+}
+
 /* Nearest points of `count` vectors stored back to back (d floats each). */
 void hqo_nearest_batch(int lattice, const float *x, int64_t count, int32_t *c, int32_t *z,
                        float *pt)
