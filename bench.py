@@ -528,6 +528,11 @@ def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
         def ours_int8():
             hq.hq_decode_gemm_int8(s, r, c, TILE, LAT, BPS, SEED, x, y8, ws8, st)
 
+        yf8 = torch.empty(batch, r, dtype=torch.float32, device=dev)
+
+        def ours_fp8():
+            hq.hq_decode_gemm_fp8(s, r, c, TILE, LAT, BPS, SEED, x, yf8, ws8, st)
+
         def dense():
             torch.matmul(x, w1.t())
 
@@ -536,11 +541,13 @@ def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
             torch.matmul(x, wd.t())
 
         for _ in range(3):
-            ours(); ours_int8(); dense(); decode_then_dense()
+            ours(); ours_int8(); ours_fp8(); dense(); decode_then_dense()
         torch.cuda.synchronize()
         assert int(st.item()) == 0
         ref = (x.float() @ wd.float().t())  # the bf16 decode's product, for the int8 path's error
         rel8 = float((y8 - ref).norm() / ref.norm())
+        relf8 = float((yf8 - ref).norm() / ref.norm())
+        tf8 = time_launches(ours_fp8, lambda: flush_l2(flushbuf))
         rel16 = float((y - ref).norm() / ref.norm())
         t8 = time_launches(ours_int8, lambda: flush_l2(flushbuf))
         t = time_launches(ours, lambda: flush_l2(flushbuf))
@@ -551,6 +558,7 @@ def gemm_leg(dev, peak, batches=(1, 16, 64, 256)):
                                 "weights_per_us": round(r * c / t / 1e3, 1),
                                 "bf16_cublas_us": round(td * 1e3, 2), "decode_then_cublas_us": round(tdd * 1e3, 2),
                                 "int8_us": round(t8 * 1e3, 2), "int8_rel_err": round(rel8, 5),
+                                "fp8_us": round(tf8 * 1e3, 2), "fp8_rel_err": round(relf8, 5),
                                 "bf16_rel_err": round(rel16, 5)}
     return res
 

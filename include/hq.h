@@ -259,7 +259,7 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
                    uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
-/* Bytes of device workspace hq_decode_gemm_int8 needs: the quantized
+/* Bytes of device workspace hq_decode_gemm_int8 (and hq_decode_gemm_fp8) needs: the quantized
  * activations (int8, batch rounded up to the block's batch rows (at most 64)
  * x cols, 256-byte rounded), their scales (fp32, padded batch x cols / 256),
  * then fp32 split-K partials.  Host only; as hq_decode_gemm_workspace_bytes. */
@@ -281,6 +281,19 @@ int hq_decode_gemm_int8_workspace_bytes(int64_t rows, int64_t cols, int64_t batc
 int hq_decode_gemm_int8(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                         uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
                         uint64_t workspace_bytes, void *stream, int32_t *d_status);
+
+/* Batched decode + fp8 tensor-core product ([V1] abstract: the fp8-e4m3
+ * MMA path, which the pages find behind int8 on the lattice output): as
+ * hq_decode_gemm_int8 with both operands in OCP FP8 E4M3 (largest finite
+ * 448): A = e4m3(2y), exact while |2y| <= 16 and rounded to nearest even on
+ * the format's coarser grid beyond (HQ_ST_RANGE where |2y| > 448, saturated),
+ * and q_bj = e4m3(x~_bj 448 / max|x~_bj|), s_bj = max|x~_bj| / 448.  Products
+ * accumulate in fp32 on the tensor cores (tcgen05.mma kind::f8f6f4).
+ * Workspace: hq_decode_gemm_int8_workspace_bytes.  A2 returns
+ * HQ_ERR_UNSUPPORTED. */
+int hq_decode_gemm_fp8(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                       uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                       uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
 /* Testing hook for failure detection (no counterpart on the pages):
  * hq_decode_gemm in which column tile `stalled_tile` never issues or commits

@@ -446,13 +446,14 @@ namespace {
 int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                      uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
                      uint64_t workspace_bytes, void *stream, int32_t *d_status, int64_t stall_tile,
-                     bool int8 = false)
+                     int lowbit = 0)  // 0: bf16 operands, 1: int8, 2: fp8 (E4M3)
 {
     GemmArgs a{};
     int64_t ntiles = 0;
     int rc = decode_common(w, rows, cols, tile, lattice, bps, seed, a.w, &ntiles);
     if (rc) return rc;
     if (tile != 256) return HQ_ERR_UNSUPPORTED;
+    const bool int8 = lowbit != 0;  // both 8-bit products share the workspace layout and plan
     if (int8 && lattice == HQ_A2) return HQ_ERR_UNSUPPORTED;  // A2 points have no integer form
     if (batch < 0) return HQ_ERR_ARG;
     if (batch > (int64_t)1 << 24) return HQ_ERR_UNSUPPORTED;
@@ -487,7 +488,8 @@ int decode_gemm_impl(const hq_stream *w, int64_t rows, int64_t cols, int tile, i
     a.sign_key = hash_key(seed, 1);
     a.status = d_status;
     a.stall_tile = stall_tile;
-    if (int8) return launch_gemm_i8(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    if (lowbit == 2) return launch_gemm_e4m3(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    if (lowbit == 1) return launch_gemm_i8(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     return launch_gemm(lattice, a, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -518,7 +520,15 @@ int hq_decode_gemm_int8(const hq_stream *w, int64_t rows, int64_t cols, int tile
                         uint64_t workspace_bytes, void *stream, int32_t *d_status)
 {
     return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
-                            d_status, -1, true);
+                            d_status, -1, 1);
+}
+
+int hq_decode_gemm_fp8(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                       uint64_t seed, const void *x, int64_t batch, float *y, void *workspace,
+                       uint64_t workspace_bytes, void *stream, int32_t *d_status)
+{
+    return decode_gemm_impl(w, rows, cols, tile, lattice, bps, seed, x, batch, y, workspace, workspace_bytes, stream,
+                            d_status, -1, 2);
 }
 
 int hq_test_gemm_stalled(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,

@@ -19,6 +19,7 @@
 // "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline for Large
 // Language and Diffusion Models", abstract (low-bit MMA decode paths).
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "hq_parse.cuh"
 
@@ -90,6 +91,30 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// kind::f8f6f4 instruction descriptor: fp32 accumulator, E4M3 A and B (type
+// code 0), both K-major, M x N.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int m, int n)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// E4M3 bits of x, round to nearest even, saturating to +-448 (NaN stays NaN)
+__device__ __forceinline__ uint32_t e4m3_bits(float x)
+{
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
 }
 
 __device__ __forceinline__ void umma_commit(uint32_t mbar)
@@ -364,9 +389,12 @@ __global__ void splitk_reduce_kernel(const GemmArgs a)
 // exact int32 sums A q; the epilogue scales them by Delta_rj s_bj / (2 n) and
 // accumulates in fp32:  Y[b][r] = sum_j Delta_rj s_bj / (2 n) sum_i A_rji q_bji.
 
-// Q[b][j n + i] and S[b][j] for b < batch_pad (zero for the padding rows).
+// Q[b][j n + i] and S[b][j] for b < batch_pad (zero for the padding rows);
+// FP8: q = e4m3(x~ 448 / max|x~|), s = max|x~| / 448 (the fp8 variant).
+template <bool FP8>
 __global__ void __launch_bounds__(256) rotate_quant_x_kernel(const GemmArgs a)
 {
+    constexpr float kQmax = FP8 ? 448.0f : 127.0f;
     constexpr int N = kGemmN, EPL = 16, LPT = 16, GPB = 16;
     const int lane = threadIdx.x & 31, l = lane % LPT;
     const unsigned mask = group_mask<LPT>(lane);
@@ -406,13 +434,14 @@ __global__ void __launch_bounds__(256) rotate_quant_x_kernel(const GemmArgs a)
         uint32_t wq[4] = { 0u, 0u, 0u, 0u };
         float scale = amax;
         if (mb != 0u && mb < 0x7f800000u) {
-            const float inv = __fdiv_rn(127.0f, amax);
+            const float inv = __fdiv_rn(kQmax, amax);
 #pragma unroll
             for (int r = 0; r < EPL; r++) {
-                const int q = __float2int_rn(__fmul_rn(v[r], inv));  // |q| <= 127
-                wq[r >> 2] |= ((uint32_t)q & 0xffu) << (8 * (r & 3));
+                const float xs = __fmul_rn(v[r], inv);
+                const uint32_t q = FP8 ? e4m3_bits(xs) : ((uint32_t)__float2int_rn(xs) & 0xffu);  // |q| <= 127
+                wq[r >> 2] |= q << (8 * (r & 3));
             }
-            scale = __fdiv_rn(amax, 127.0f);
+            scale = __fdiv_rn(amax, kQmax);
         }
         *reinterpret_cast<uint4 *>(a.xq + b * a.cols + j * N + l * EPL) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
         if (l == 0) a.sx[b * a.tiles_per_row + j] = scale;
@@ -427,13 +456,13 @@ __global__ void __launch_bounds__(256) rotate_quant_x_kernel(const GemmArgs a)
 // Delta s / (2 n) and add it to the item's fp32 sums in shared memory while
 // the other warps parse tile j + 1 (the row and batch scales are double
 // buffered); the item's sums are stored after its last tile.
-template <int D, int NB, bool FIXED>
+template <int D, int NB, bool FIXED, bool FP8>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs a)
 {
     constexpr int N = kGemmN, EPL = 16, LPT = 16, TPW = 2, GPB = kGemmWarps * TPW;
     constexpr uint32_t LBO_A = gemm_lbo(kGemmM) * 16u, LBO_B = gemm_lbo(NB) * 16u;
     constexpr uint32_t NCOLS = NB < 32 ? 32u : (uint32_t)NB;
-    constexpr uint32_t IDESC = make_idesc_i8(kGemmM, NB);
+    constexpr uint32_t IDESC = FP8 ? make_idesc_e4m3(kGemmM, NB) : make_idesc_i8(kGemmM, NB);
     static_assert(NB == 16 || NB == 32 || NB == 64, "int8 batch block");
     extern __shared__ __align__(128) uint8_t smraw[];
     uint8_t *sA = smraw;
@@ -475,7 +504,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs
             tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
 #pragma unroll
             for (int i = 0; i < 16; i++) {
-                const float term = __fmul_rn(__fmul_rn(d, sxs[pb * NB + c + i]), (float)__float_as_int(v[i]));
+                const float sum = FP8 ? v[i] : (float)__float_as_int(v[i]);  // fp32 (fp8) or s32 (int8) accumulator
+                const float term = __fmul_rn(__fmul_rn(d, sxs[pb * NB + c + i]), sum);
                 acc[(c + i) * kGemmM + row] = __fadd_rn(acc[(c + i) * kGemmM + row], __fmul_rn(term, kInv2N));
             }
         }
@@ -520,12 +550,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs
                 bool sat = false;
 #pragma unroll
                 for (int i = 0; i < EPL; i++) {
-                    int v2 = __float2int_rn(2.0f * pt[i]);  // exact: 2y is an integer
-                    if (v2 > 127 || v2 < -127) {
-                        sat = true;
-                        v2 = v2 > 0 ? 127 : -127;
+                    const float y2 = 2.0f * pt[i];  // exact: 2y is an integer
+                    uint32_t b8;
+                    if constexpr (FP8) {
+                        sat |= fabsf(y2) > 448.0f;
+                        b8 = e4m3_bits(y2);
+                    } else {
+                        int v2 = __float2int_rn(y2);
+                        if (v2 > 127 || v2 < -127) {
+                            sat = true;
+                            v2 = v2 > 0 ? 127 : -127;
+                        }
+                        b8 = (uint32_t)v2 & 0xffu;
                     }
-                    wa[i >> 2] |= ((uint32_t)v2 & 0xffu) << (8 * (i & 3));
+                    wa[i >> 2] |= b8 << (8 * (i & 3));
                 }
                 *reinterpret_cast<uint4 *>(sA + (uint32_t)((m & 7) + 8 * (m >> 3)) * 16u + (uint32_t)l * LBO_A) =
                     make_uint4(wa[0], wa[1], wa[2], wa[3]);
@@ -549,7 +587,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs
                 for (int s = 0; s < N / 32; s++) {
                     const uint64_t ad = make_smem_desc(aA + 2u * s * LBO_A, LBO_A, 128u);
                     const uint64_t bd = make_smem_desc(aB + 2u * s * LBO_B, LBO_B, 128u);
-                    umma_i8(tmem, ad, bd, IDESC, s > 0 ? 1u : 0u);
+                    if constexpr (FP8) umma_e4m3(tmem, ad, bd, IDESC, s > 0 ? 1u : 0u);
+                    else umma_i8(tmem, ad, bd, IDESC, s > 0 ? 1u : 0u);
                 }
                 umma_commit(bar);
             }
@@ -693,13 +732,13 @@ cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s)
 
 namespace {
 
-template <int D, int NB>
+template <int D, int NB, bool FP8>
 cudaError_t launch_gemm_i8_t(GemmArgs a, cudaStream_t s)
 {
     const size_t smem = gemm_operand_bytes_i8(kGemmM) + gemm_operand_bytes_i8(NB) +
                         ((size_t)NB * kGemmM + 2 * kGemmM + 2 * NB) * 4 +
                         (size_t)kGemmWarps * 2 * group_words(a.w.wmax) * 4;
-    auto kern = a.w.slot ? gemm_i8_kernel<D, NB, true> : gemm_i8_kernel<D, NB, false>;
+    auto kern = a.w.slot ? gemm_i8_kernel<D, NB, true, FP8> : gemm_i8_kernel<D, NB, false, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -726,31 +765,36 @@ cudaError_t launch_gemm_i8_t(GemmArgs a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_gemm_i8_d(const GemmArgs &a, cudaStream_t s)
 {
     switch (a.nb) {
-    case 16: return launch_gemm_i8_t<D, 16>(a, s);
-    case 32: return launch_gemm_i8_t<D, 32>(a, s);
-    default: return launch_gemm_i8_t<D, 64>(a, s);
+    case 16: return launch_gemm_i8_t<D, 16, FP8>(a, s);
+    case 32: return launch_gemm_i8_t<D, 32, FP8>(a, s);
+    default: return launch_gemm_i8_t<D, 64, FP8>(a, s);
+    }
+}
+
+template <bool FP8>
+cudaError_t launch_lowbit(int lattice, const GemmArgs &a, cudaStream_t s)
+{
+    const int64_t xtiles = (int64_t)a.batch_pad * a.tiles_per_row;
+    int64_t rb = (xtiles + 15) / 16;
+    if (rb > 4 * (int64_t)sm_count()) rb = 4 * (int64_t)sm_count();
+    rotate_quant_x_kernel<FP8><<<(unsigned)(rb > 0 ? rb : 1), 256, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    switch (lattice) {
+    case 1: return launch_gemm_i8_d<1, FP8>(a, s);
+    case 4: return launch_gemm_i8_d<4, FP8>(a, s);
+    default: return launch_gemm_i8_d<8, FP8>(a, s);  // A2 has no integer form: refused by the host API
     }
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s)
-{
-    const int64_t xtiles = (int64_t)a.batch_pad * a.tiles_per_row;
-    int64_t rb = (xtiles + 15) / 16;
-    if (rb > 4 * (int64_t)sm_count()) rb = 4 * (int64_t)sm_count();
-    rotate_quant_x_kernel<<<(unsigned)(rb > 0 ? rb : 1), 256, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    switch (lattice) {
-    case 1: return launch_gemm_i8_d<1>(a, s);
-    case 4: return launch_gemm_i8_d<4>(a, s);
-    default: return launch_gemm_i8_d<8>(a, s);  // A2 has no integer form: refused by the host API
-    }
-}
+cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s) { return launch_lowbit<false>(lattice, a, s); }
+
+cudaError_t launch_gemm_e4m3(int lattice, const GemmArgs &a, cudaStream_t s) { return launch_lowbit<true>(lattice, a, s); }
 
 }  // namespace hq

@@ -94,8 +94,9 @@ struct GemmArgs {
     DecodeArgs w;               // weight stream, rows x cols
     const uint16_t *x;          // bf16 [batch][cols]
     uint16_t *xt;               // bf16 [batch_pad][cols]: rotated activations (workspace)
-    int8_t *xq;                 // int8 product: quantized rotated activations [batch_pad][cols] (workspace)
-    float *sx;                  // int8 product: their scales [batch_pad][tiles_per_row] (workspace)
+    int8_t *xq;                 // 8-bit products: quantized rotated activations [batch_pad][cols]
+                                // (int8, or E4M3 bits for the fp8 variant; workspace)
+    float *sx;                  // 8-bit products: their scales [batch_pad][tiles_per_row] (workspace)
     float *y;                   // fp32 [batch][rows]
     float *part;                // fp32 [ksplit][batch_pad][rows] split-K partials (workspace)
     int64_t rows, cols, tiles_per_row;
@@ -127,6 +128,8 @@ void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, Gem
 // batch blocks of at most 64 rows; same splitting rule.
 void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
 cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s);
+// The fp8 variant: A = e4m3(2y), activations in E4M3 scaled to +-448 (same workspace).
+cudaError_t launch_gemm_e4m3(int lattice, const GemmArgs &a, cudaStream_t s);
 // Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
 cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 

@@ -32,7 +32,7 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
            "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled",
            "hq_min_slot_words", "hq_fixed_slot_words", "hq_encode_fixed", "hq_kv_encode_fixed",
-           "hq_decode_gemm_int8_workspace_bytes", "hq_decode_gemm_int8"]
+           "hq_decode_gemm_int8_workspace_bytes", "hq_decode_gemm_int8", "hq_decode_gemm_fp8"]
 
 
 class hq_file_info(ctypes.Structure):
@@ -86,6 +86,8 @@ _SIGS = {
     "hq_decode_gemm_int8_workspace_bytes": (_i32, [_i64, _i64, _i64, ctypes.POINTER(_u64)]),
     "hq_decode_gemm_int8": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
                                    _u64, _vp, _vp]),
+    "hq_decode_gemm_fp8": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
+                                  _u64, _vp, _vp]),
     "hq_decode_gemm": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _i64, _vp, _vp,
                               _u64, _vp, _vp]),
     "hq_kv_attention": (_i32, [ctypes.POINTER(hq_stream), ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32,
@@ -351,6 +353,20 @@ def hq_decode_gemm_int8(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, w
     _check(_lib.hq_decode_gemm_int8(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch,
                                     _ptr(y), _ptr(workspace), workspace.numel(), _stream_handle(stream),
                                     _ptr(status)), "hq_decode_gemm_int8")
+    return y
+
+
+def hq_decode_gemm_fp8(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, workspace, status=None, stream=None):
+    """Y = X W_hat^T on the fp8 tensor cores: A = e4m3(2y), the rotated
+    activations in E4M3 per (row, column tile); workspace from
+    alloc_gemm_int8_workspace; y is fp32 [batch, rows]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == cols
+    batch = x.shape[0]
+    assert y.dtype == torch.float32 and y.is_contiguous() and y.numel() == batch * rows
+    st = s.struct()
+    _check(_lib.hq_decode_gemm_fp8(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), batch,
+                                   _ptr(y), _ptr(workspace), workspace.numel(), _stream_handle(stream),
+                                   _ptr(status)), "hq_decode_gemm_fp8")
     return y
 
 
