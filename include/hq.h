@@ -35,6 +35,8 @@
  *               tile_off[ntiles] = total payload words
  *   tile_scale  ntiles bf16 bit patterns of Delta (0 = all-zero tile)
  *   tile_k      ntiles Rice parameters, 0..15
+ * (A fixed-rate stream, hq_stream.slot_words > 0, has no offsets and packs k
+ * in 4 bits: see hq_stream and hq_encode_fixed.)
  * Tile layout, bits LSB-first in little-endian words: the n/d coset bits
  * (E8 and A2 only), then k low bits of each of the n codes in coordinate
  * order, then for each code q = u >> k zero bits and a one bit, then zero
