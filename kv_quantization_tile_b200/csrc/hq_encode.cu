@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 // the byte of packed 4-bit Rice parameters, into a zeroed shared-memory slot
 // image and stores it whole.
 
-constexpr int kFixedWarps = 8;
+constexpr int kFixedWarps = 8, kFixedThreads = kFixedWarps * 32;
 // Resident blocks the registers are budgeted for: the rotated tile, the
 // next tile's raw words and a probe's symbols are live together.  At 80
 // registers (3 blocks per SM) E8 spills a few words, yet measured faster
@@ -521,6 +521,7 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
     extern __shared__ __align__(16) uint32_t smem[];
     unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);
     uint32_t *images = smem + 2 * ((a.sign_words + 1) & ~1);
+    uint32_t *sym = images + (size_t)GPB * istride;  // [EPL + 3][threads]: the last fitting probe's symbols
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < a.sign_words; i += kFixedWarps * 32) {
@@ -568,10 +569,11 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             if (nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
             const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
 
-            // ---- scale search: one probe site (quantize + Rice parameter) serves
-            // every probe and the final pass; a state machine picks the next
-            // pattern.  When the search ends on the pattern just probed, that
-            // probe's symbols are the tile's and no final pass runs.
+            // ---- scale search: one probe site (quantize + Rice parameter), a
+            // state machine picking the next pattern.  Every fitting probe's
+            // symbols are kept in shared memory, so the answer (the last
+            // fitting probe) never needs a final pass; only the all-zero tile
+            // runs one, on zeros.
             const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
             const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
             int phase = c0 ? kPredict : kFinal, lo = 0, hi = (int)c0, step = 1, c = (int)c0;
@@ -583,6 +585,13 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
                 if (phase == kFinal) break;
                 const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part);
                 const bool f = bits <= budget;
+                if (f) {  // keep a fitting probe's symbols: the search's answer is its last fitting probe
+#pragma unroll
+                    for (int r = 0; r < EPL; r++) sym[r * kFixedThreads + tid] = u[r];
+                    sym[(EPL + 0) * kFixedThreads + tid] = cbits;
+                    sym[(EPL + 1) * kFixedThreads + tid] = (uint32_t)k;
+                    sym[(EPL + 2) * kFixedThreads + tid] = part;
+                }
                 if (phase == kPredict) {
                     // a pattern step moves the size by about N / 128 bits: start
                     // from c0 + floor(128 (bits - budget) / N), clamped
@@ -622,7 +631,15 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
                 } else {
                     if (answer == c && f) break;  // the last probe is the answer
                     c = answer;
-                    phase = kFinal;
+                    if (answer != 0) {  // an earlier fitting probe: its kept symbols
+#pragma unroll
+                        for (int r = 0; r < EPL; r++) u[r] = sym[r * kFixedThreads + tid];
+                        cbits = sym[(EPL + 0) * kFixedThreads + tid];
+                        k = (int)sym[(EPL + 1) * kFixedThreads + tid];
+                        part = sym[(EPL + 2) * kFixedThreads + tid];
+                        break;
+                    }
+                    phase = kFinal;  // the all-zero tile
                 }
             }
             const uint32_t sb = (uint32_t)c;
@@ -698,7 +715,8 @@ cudaError_t launch_encode_fixed_t(const EncodeArgs &a, cudaStream_t s)
 {
     constexpr int EPL = epl_for<N>(), GPB = kFixedWarps * (32 / (N / EPL));
     const size_t istride = (a.slot_words + 1 + 3) & ~(size_t)3;
-    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + (size_t)GPB * istride * 4;
+    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + (size_t)GPB * istride * 4 +
+                        (size_t)(EPL + 3) * kFixedThreads * 4;
     auto kern = encode_fixed_kernel<N, D, EPL, DITHER, F32IN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
