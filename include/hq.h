@@ -262,7 +262,7 @@ int hq_decode_gemm(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    uint64_t workspace_bytes, void *stream, int32_t *d_status);
 
 /* Bytes of device workspace hq_decode_gemm_int8 (and hq_decode_gemm_fp8) needs: the quantized
- * activations (int8, batch rounded up to the block's batch rows (at most 64)
+ * activations (int8, batch rounded up to the block's batch rows (at most 128)
  * x cols, 256-byte rounded), their scales (fp32, padded batch x cols / 256),
  * then fp32 split-K partials.  Host only; as hq_decode_gemm_workspace_bytes. */
 int hq_decode_gemm_int8_workspace_bytes(int64_t rows, int64_t cols, int64_t batch, uint64_t *out);

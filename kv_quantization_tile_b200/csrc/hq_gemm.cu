@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_i8_kernel(const GemmArgs
     constexpr uint32_t LBO_A = gemm_lbo(kGemmM) * 16u, LBO_B = gemm_lbo(NB) * 16u;
     constexpr uint32_t NCOLS = NB < 32 ? 32u : (uint32_t)NB;
     constexpr uint32_t IDESC = FP8 ? make_idesc_e4m3(kGemmM, NB) : make_idesc_i8(kGemmM, NB);
-    static_assert(NB == 16 || NB == 32 || NB == 64, "int8 batch block");
+    static_assert(NB == 16 || NB == 32 || NB == 64 || NB == 128, "8-bit batch block");
     extern __shared__ __align__(128) uint8_t smraw[];
     uint8_t *sA = smraw;
     uint8_t *sB = sA + gemm_operand_bytes_i8(kGemmM);
@@ -653,7 +653,7 @@ void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, Gem
 
 void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p)
 {
-    gemm_plan(rows, cols, batch < 64 ? batch : 64, blocks_per_sm, p);  // splits for one batch block of <= 64
+    gemm_plan(rows, cols, batch < 128 ? batch : 128, blocks_per_sm, p);  // splits for one batch block of <= 128
     p->batch_pad = (int)(((batch + p->nb - 1) / p->nb) * p->nb);
     const int64_t tpr = cols / kGemmN;
     const uint64_t q_bytes = ((uint64_t)p->batch_pad * (uint64_t)cols + 255) / 256 * 256;
@@ -771,7 +771,8 @@ cudaError_t launch_gemm_i8_d(const GemmArgs &a, cudaStream_t s)
     switch (a.nb) {
     case 16: return launch_gemm_i8_t<D, 16, FP8>(a, s);
     case 32: return launch_gemm_i8_t<D, 32, FP8>(a, s);
-    default: return launch_gemm_i8_t<D, 64, FP8>(a, s);
+    case 64: return launch_gemm_i8_t<D, 64, FP8>(a, s);
+    default: return launch_gemm_i8_t<D, 128, FP8>(a, s);
     }
 }
 

@@ -82,7 +82,7 @@ def check(s, ref, rows, cols, lat, seed, X, bps=4.0, want_status=0, fmt="int8"):
     wsn = ws.cpu().numpy()
     q = wsn[: batch * cols].view(Q.dtype).reshape(batch, cols)
     assert np.array_equal(q, Q)
-    nb = 16 if batch <= 16 else 32 if batch <= 32 else 64
+    nb = 16 if batch <= 16 else 32 if batch <= 32 else 64 if batch <= 64 else 128
     pad = (batch + nb - 1) // nb * nb
     so = (pad * cols + 255) // 256 * 256
     sx = wsn[so: so + pad * (cols // N) * 4].view(np.float32).reshape(pad, cols // N)[:batch]
@@ -90,7 +90,7 @@ def check(s, ref, rows, cols, lat, seed, X, bps=4.0, want_status=0, fmt="int8"):
 
 
 @pytest.mark.parametrize("lat", ["E8", "D4", "Z"])
-@pytest.mark.parametrize("batch", [1, 16, 37, 100])
+@pytest.mark.parametrize("batch", [1, 16, 37, 100, 150])
 @pytest.mark.parametrize("fmt", ["int8", "fp8"])
 def test_int8_product(lat, batch, fmt):
     rows, cols, seed = 203, 1024, 5
