@@ -124,8 +124,7 @@ cudaError_t launch_gemm(int lattice, const GemmArgs &a, cudaStream_t s);
 // Plan for blocks_per_sm resident blocks; the launch re-plans from the
 // kernel's occupancy (never more splits than for two blocks per SM).
 void gemm_plan(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
-// The 8-bit products (A = 2y in int8 or E4M3, activations quantized alike):
-// batch blocks of at most 128 rows; same splitting rule.
+// The 8-bit products (int8 or E4M3 operands); see gemm_plan_i8 in hq_gemm.cu.
 void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, GemmPlan *p);
 cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s);
 // The fp8 variant: A = e4m3(2y), activations in E4M3 scaled to +-448 (same workspace).
