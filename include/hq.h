@@ -373,9 +373,11 @@ int hq_test_encode_stalled(const void *x, int dtype, int64_t rows, int64_t cols,
  * exits; a call may use at most 65536 encode chunks (that is,
  * hq_encode_workspace_bytes(rows, cols, tile) <= 256 + 8 * 65536), larger
  * shapes return HQ_ERR_UNSUPPORTED with nothing launched.  The call allocates
- * nothing.  The first call on a device looks up that device's scratch
- * address (cudaGetSymbolAddress, with the device current); make that first
- * call before any stream capture.  Every call on a device shares the one
+ * nothing.  Every call looks up the current device's scratch address
+ * (cudaGetSymbolAddress, with that device current), so the address is right
+ * again after a cudaDeviceReset; the first call on a device may load the
+ * library's device code, so make that first call before any stream capture.
+ * Every call on a device shares the one
  * array and clears the part it uses on `stream` before its kernel runs, so
  * calls whose work overlaps on the GPU (different streams, no ordering)
  * race on it and must be serialised by the caller. */

@@ -366,7 +366,9 @@ int hq_kv_encode_fixed(const void *x, int dtype, int64_t rows, int64_t cols, int
 int hq_encode_workspace_bytes(int64_t rows, int64_t cols, int tile, uint64_t *out)
 {
     if (!out || rows < 0 || cols < 0 || !valid_tile(tile) || cols % tile) return HQ_ERR_ARG;
-    const int64_t ntiles = rows * (cols / tile);
+    const int64_t tpr = cols / tile;
+    if (tpr && rows > (int64_t)(INT64_MAX / 2) / tpr) return HQ_ERR_UNSUPPORTED;  // rows * tpr would overflow
+    const int64_t ntiles = rows * tpr;
     *out = 256 + 8 * (uint64_t)nchunks_for(ntiles, tile);
     return HQ_OK;
 }

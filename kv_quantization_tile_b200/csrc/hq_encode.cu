@@ -61,7 +61,10 @@ __device__ __forceinline__ void named_arrive(int id, int threads)
 
 // Decoupled look-back run by one whole warp: publish this chunk's aggregate,
 // then sum predecessors 32 at a time until an inclusive prefix is found.
-// Returns the exclusive prefix (same value in every lane).
+// Returns the exclusive prefix (same value in every lane).  A chunk that gives
+// up waiting, or meets a poisoned predecessor before any inclusive prefix,
+// publishes poison instead of a prefix and reports timed_out, so every later
+// chunk also gives up without writing rather than using a wrong offset.
 
 __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, uint64_t agg, int lane,
                                         bool publish, bool &timed_out)
@@ -80,9 +83,9 @@ __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, 
         const int64_t p = top - lane;
         unsigned long long s = p >= 0 ? ld_acquire(&lb[p]) : (kFlagInclusive | 0ull);
         const uint64_t flag = s & ~kValueMask;
-        const unsigned incl = __ballot_sync(FULL, flag == kFlagInclusive);
+        const unsigned incl = __ballot_sync(FULL, flag == kFlagInclusive || flag == kFlagPoison);
         const unsigned none = __ballot_sync(FULL, flag == 0);
-        // lanes up to and including the nearest inclusive prefix
+        // lanes up to and including the nearest inclusive (or poisoned) slot
         const unsigned upto = incl ? ((incl & -incl) << 1) - 1u : FULL;
         if (none & upto) {  // a needed predecessor has not published yet
             if (++polls > kSpinLimit || global_ns() - t0 > kWaitLimitNs) {
@@ -92,6 +95,10 @@ __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, 
             __nanosleep(64);
             continue;
         }
+        if (incl && __shfl_sync(FULL, flag, __ffs(incl) - 1) == kFlagPoison) {
+            timed_out = true;  // an earlier chunk gave up: no valid prefix exists
+            break;
+        }
         uint64_t v = ((1u << lane) & upto) ? (s & kValueMask) : 0;
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(FULL, v, m);
@@ -99,7 +106,8 @@ __device__ uint64_t chunk_lookback_warp(unsigned long long *lb, uint32_t chunk, 
         if (incl) break;
         top -= 32;
     }
-    if (lane == 0 && publish) st_release(&lb[chunk], kFlagInclusive | ((excl + agg) & kValueMask));
+    if (lane == 0 && publish)
+        st_release(&lb[chunk], timed_out ? kFlagPoison : (kFlagInclusive | ((excl + agg) & kValueMask)));
     return excl;
 }
 

@@ -283,7 +283,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
                 const bool ok = mbar_wait(bar, parity);
                 parity ^= 1u;
                 pending = false;
-                if (__syncthreads_or(!ok)) {  // every thread leaves together; nothing is in flight
+                // Every thread leaves together.  The wait gives up only when a
+                // tile's MMAs were never issued and committed (the stall hook
+                // withholds them); committed MMAs finish in microseconds, so no
+                // tensor-core work is in flight when the block then frees TMEM.
+                if (__syncthreads_or(!ok)) {
                     fail = true;
                     break;
                 }
@@ -340,13 +344,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
             if (__syncthreads_or(!ok)) fail = true;
         }
         tc_fence_after();
-        // epilogue: warp w < 4 owns TMEM lanes (rows) 32 w .. 32 w + 31
+        // epilogue: warp w < 4 owns TMEM lanes (rows) 32 w .. 32 w + 31; after
+        // a wait that gave up the accumulator is not read (zeros are stored)
         if (warp < 4) {
             const int64_t r = r0 + warp * 32 + lane;
 #pragma unroll
             for (int c = 0; c < NB; c += 16) {
                 float v[16];
-                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+                if (!fail) {
+                    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) v[i] = 0.0f;
+                }
 #pragma unroll
                 for (int i = 0; i < 16; i++) {
                     const int b = b0 + c + i;

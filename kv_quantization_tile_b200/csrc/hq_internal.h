@@ -12,8 +12,9 @@ namespace hq {
 constexpr int kStatusNonfinite = 1, kStatusCapacity = 2, kStatusCorrupt = 4, kStatusTimeout = 8, kStatusRange = 16;
 
 // Look-back slot: bits 62..63 flag (1 = chunk aggregate, 2 = inclusive
-// prefix), bits 0..61 the word count.
-constexpr uint64_t kFlagAggregate = 1ull << 62, kFlagInclusive = 2ull << 62;
+// prefix, 3 = poisoned: the chunk gave up waiting, so no prefix from it on is
+// valid), bits 0..61 the word count.
+constexpr uint64_t kFlagAggregate = 1ull << 62, kFlagInclusive = 2ull << 62, kFlagPoison = 3ull << 62;
 constexpr uint64_t kValueMask = (1ull << 62) - 1;
 constexpr uint32_t kSpinLimit = 1u << 24;          // polls before a wait gives up ...
 constexpr uint64_t kWaitLimitNs = 500ull * 1000000;  // ... or 0.5 s of waiting, whichever first

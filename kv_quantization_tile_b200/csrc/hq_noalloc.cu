@@ -14,7 +14,6 @@
 // The kernel launched is the same encoder hq_encode launches; only where its
 // scratch comes from differs.
 #include <cstdint>
-#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -32,23 +31,15 @@ constexpr uint64_t kNoallocScratchBytes = 256 + 8 * kNoallocChunks;
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void *g_scratch_ptr[kMaxDevices] = { nullptr };
-
-// Device address of the scratch array on the current device, looked up once
-// per device (under a lock) and cached.
+// Device address of the scratch array on the current device.  It is looked
+// up on every call (a host-side table lookup once the module is loaded, no
+// allocation), so the address stays right after a device reset reloads the
+// module at a new place.
 int scratch_address(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HQ_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HQ_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HQ_ERR_CUDA;
+    *out = p;
     return HQ_OK;
 }
 

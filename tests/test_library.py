@@ -81,6 +81,14 @@ def test_sizing_functions():
     with pytest.raises(hq.HQError) as e:
         hq.hq_max_payload_words(1 << 30, 1 << 14, 256, "E8", 8.0)
     assert e.value.code == hq.HQ_ERR_UNSUPPORTED
+    # a row count whose tile count overflows int64 is refused, not wrapped
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_encode_workspace_bytes((1 << 62) + 1, 1024, 256)
+    assert e.value.code == hq.HQ_ERR_UNSUPPORTED
+    # the no-workspace encoder refuses it too, before any device call
+    out = hq.hq_stream()
+    assert hq.library().hq_encode_noalloc(None, hq.HQ_BF16, (1 << 62) + 1, 1024, 256, hq.HQ_E8, 4.0, 0,
+                                          ctypes.byref(out), None, None) == hq.HQ_ERR_UNSUPPORTED
 
 
 def _raw_encode(x, dtype, rows, cols, tile, lat, bps, stream_struct, ws=1, wsb=1 << 20):
