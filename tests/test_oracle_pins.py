@@ -47,6 +47,20 @@ def test_signs_and_uniforms_are_balanced():
         assert abs(rk.mean() - 0.5) < 4 * math.sqrt(1 / 12 / rk.size)
 
 
+def test_signs_and_uniforms_match_worked_examples():
+    """Worked examples of the sign vector and the dither uniforms, derived step
+    by step from their definition with only the published-vector-pinned mix64
+    (tests/golden/make_hash_bits.py): a swapped hash argument or a mirrored bit
+    index in the oracle would change them."""
+    g = json.load(open(os.path.join(GOLD, "hash_bits.json")))
+    for e in g["signs"]:
+        want = np.array([-1 if ch == "-" else 1 for ch in e["signs"]])
+        assert np.array_equal(oracle.signs(e["seed"], e["j"], e["n"]), want), (e["seed"], e["j"])
+    for e in g["uniforms"]:
+        got = [oracle.uniform(e["seed"], e["t"], i) * 65536.0 for i in range(len(e["r_times_2^16"]))]
+        assert got == [float(v) for v in e["r_times_2^16"]], (e["seed"], e["t"])
+
+
 # ------------------------------------------------------------ Hadamard
 @pytest.mark.parametrize("n", [2, 8, 64, 128, 256, 1024])
 def test_fwht_is_sylvester_hadamard(n):
@@ -167,6 +181,18 @@ def test_tie_rules():
     assert c == 0 and list(z) == [0] * 8
     c, z, _ = oracle.nearest("E8", np.full(8, 0.2500001))
     assert c == 1
+    # an integer vector with an odd sum: every |e| is 0, so the first
+    # coordinate moves, and it moves up (the "towards x" rule when x is exact)
+    c, z, _ = oracle.nearest("D4", [1.0, 0.0, 0.0, 0.0])
+    assert list(z) == [2, 0, 0, 0]
+    c, z, _ = oracle.nearest("E8", [0.0, -3.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0])
+    assert c == 0 and list(z) == [1, -3, 0, 0, 0, 0, 0, 0]
+    # the half-integer coset: x all half-integers with an odd floor sum is not in
+    # E8; its nearest point moves one coordinate of the nearest half-integer
+    # vector by 1 (every |e| ties at 1/2, so the first), and at x - floor(x) =
+    # 1/2 exactly the move is up: z = floor(x) + e_0
+    c, z, pt = oracle.nearest("E8", [0.5] * 7 + [1.5])
+    assert c == 1 and list(z) == [1, 0, 0, 0, 0, 0, 0, 1] and list(pt) == [1.5] + [0.5] * 6 + [1.5]
 
 
 @pytest.mark.parametrize("lat", LATS)
@@ -239,6 +265,105 @@ def test_rate_constant_hits_target_entropy(lat, R):
     cc, z, _ = oracle.nearest_batch(lat, X)
     H = entropy_bits(np.concatenate([z, cc[:, None]], 1)) / d
     assert abs(H - R) < 0.03, H
+
+
+@pytest.mark.parametrize("R", [3.0, 4.0, 5.0])
+def test_e8_rate_constant_hits_target_entropy(R):
+    """E8's index at step c(R) on unit Gaussian coordinates carries ~R bits per
+    dimension.  The per-vector entropy E[-log2 P(Q(X))] is estimated without any
+    rate formula: P(y) is the Gaussian mass of y's Voronoi cell (volume 1),
+    i.e. phi(y) times the mean of phi(y + u) / phi(y) over points u uniform on
+    the cell, drawn as z - Q(z) for z uniform on [0, 2)^8 (a fundamental box
+    of the sublattice 2Z^8)."""
+    c = oracle.rate_constant("E8", R)
+    var = 1.0 / (c * c)
+    rng = np.random.default_rng(int(100 * R))
+    X = (rng.standard_normal((8000, 8)) / c).astype(np.float32)
+    _, _, Y = oracle.nearest_batch("E8", X)
+    Y = Y.astype(np.float64)
+    Zb = rng.uniform(0.0, 2.0, (2048, 8)).astype(np.float32)
+    _, _, QZ = oracle.nearest_batch("E8", Zb)
+    U = Zb.astype(np.float64) - QZ.astype(np.float64)
+    a = -(Y @ U.T) / var - (U * U).sum(1)[None, :] / (2 * var)
+    am = a.max(1, keepdims=True)
+    log_mean = (am[:, 0] + np.log(np.exp(a - am).mean(1)))
+    log_phi = -(Y * Y).sum(1) / (2 * var) - 4.0 * math.log(2 * math.pi * var)
+    H = float(-(log_phi + log_mean).mean() / math.log(2.0)) / 8
+    assert abs(H - R) < 0.03, H
+
+
+# ------------------------------------------------------------ E8 decision
+def _d8_plain(y):
+    """Conway & Sloane's D8 decoder in binary64: round every coordinate; if the
+    sum is odd, round the coordinate farthest from its integer (first such
+    index) the other way."""
+    f = np.rint(y)
+    e = y - f
+    rows = np.nonzero(np.mod(f.sum(1), 2) != 0)[0]
+    b = np.argmax(np.abs(e[rows]), 1)
+    f[rows, b] += np.where(e[rows, b] >= 0, 1.0, -1.0)
+    return f
+
+
+def _plain_e8(X):
+    """The plain two-candidate E8 decision in binary64: D8(x) against
+    D8(x - 1/2) + 1/2, by their squared distances."""
+    X64 = X.astype(np.float64)
+    y0, y1 = _d8_plain(X64), _d8_plain(X64 - 0.5) + 0.5
+    return ((X64 - y0) ** 2).sum(1), ((X64 - y1) ** 2).sum(1)
+
+
+# The oracle decides E8's coset from an exact identity for d0 - d1 evaluated in
+# binary32 (each |e| <= 1/2, at most a dozen roundings of terms below 4):
+# its decision can differ from the binary64 one only within this band.
+E8_BAND = 4e-6
+
+
+def _check_e8_against_plain(X):
+    c, _, pt = oracle.nearest_batch("E8", X)
+    d0, d1 = _plain_e8(X)
+    P = pt.astype(np.float64)
+    # the oracle's point is in E8: all-integer or all-half-integer, even sum
+    twice = 2 * P
+    assert np.all(twice == np.rint(twice))
+    par = np.mod(twice, 2)
+    assert np.all(par == par[:, :1]) and np.all(np.mod(P.sum(1), 2) == 0)
+    assert np.array_equal(c, par[:, 0].astype(np.int32))
+    # outside the band the decisions agree and the oracle's point is nearest
+    gap = np.abs(d0 - d1)
+    plain = (d1 < d0).astype(np.int32)
+    assert np.all((c == plain) | (gap <= E8_BAND))
+    dor = ((X.astype(np.float64) - P) ** 2).sum(1)
+    assert np.all(dor <= np.minimum(d0, d1) + E8_BAND)
+    return int(np.sum(c != plain))
+
+
+def test_e8_decision_agrees_with_the_plain_binary64_rule_on_random_inputs():
+    """A million random vectors at several scales: every decision matches the
+    plain binary64 rule (tie flips below 1e-6 of vectors)."""
+    rng = np.random.default_rng(88)
+    flips, total = 0, 0
+    for scale in (0.3, 1.0, 3.0, 10.0, 60.0):
+        X = (rng.standard_normal((200000, 8)) * scale).astype(np.float32)
+        flips += _check_e8_against_plain(X)
+        total += X.shape[0]
+    assert flips <= 1e-6 * total, flips
+
+
+def test_e8_decision_agrees_with_the_plain_binary64_rule_near_ties():
+    """Points within a few binary32 ulps of the boundary between the two
+    cosets (the midpoint (1/4)^8 of 0 and (1/2)^8, moved by lattice vectors
+    and sign changes that keep it on the boundary, plus tiny noise): any
+    disagreement with the binary64 rule lies inside the rounding band."""
+    rng = np.random.default_rng(89)
+    n = 100000
+    base = np.full((n, 8), 0.25)
+    flip = rng.integers(0, 2, (n, 8)) * 2 - 1
+    flip[:, 7] = flip[:, :7].prod(1)  # an even number of minus signs keeps (1/2)^8 * signs in E8
+    lam = _d8_plain(rng.normal(0, 4, (n, 8)))
+    lam[:, 0] += np.mod(lam.sum(1), 2)  # an even sum: a D8 point
+    X = (lam + base * flip + rng.normal(0, 1, (n, 8)) * 2.0**-21).astype(np.float32)
+    _check_e8_against_plain(X)
 
 
 # ------------------------------------------------------------ strip + zigzag
@@ -332,6 +457,22 @@ def test_unpack_rejects_corrupt_tiles():
 
 
 # ------------------------------------------------------------ whole tiles
+def test_tile_scale_rounds_to_bf16_like_torch():
+    """Delta = bf16_rn(c sqrt(S)): with S = 1 the oracle's rounding of c to bf16
+    equals torch's float32 -> bfloat16 conversion (round to nearest even),
+    including values exactly halfway between two bf16 numbers."""
+    import torch
+    rng = np.random.default_rng(12)
+    v = rng.uniform(-30, 30, 20000).astype(np.float32)
+    v = np.exp2(v).astype(np.float32)
+    bits = v.view(np.uint32)
+    mids = (bits & 0xFFFF0000) | rng.choice(np.array([0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF], np.uint32), bits.size)
+    v = np.concatenate([v, mids.view(np.float32)])
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.tile_scale(1.0, float(x))[0] for x in v], np.uint16)
+    assert np.array_equal(got, want)
+
+
 def test_zero_and_nonfinite_tiles():
     z = oracle.encode_tile(np.zeros(256, np.float32), "E8", 4.0, 1)
     assert z["scale"] == 0 and z["k"] == 0 and z["status"] == 0
