@@ -15,6 +15,7 @@
 // decoding; batch-1 decode against bf16 GEMV; subtractive dither).
 #include <cuda_bf16.h>
 
+#include "hq_fast.cuh"
 #include "hq_parse.cuh"
 
 namespace hq {
@@ -25,51 +26,108 @@ constexpr int kDecodeWarps = 8;
 
 }  // namespace
 
+// Output sign word of lane l of column tile j after the half-exchange transform
+// (see sign_word): pair m < EPL/4 holds tile coordinates RL l + 2m, + 1 (run
+// A), pair m >= EPL/4 coordinates N/2 + RL l + 2(m - EPL/4), + 1 (run B), RL =
+// EPL / 2; the transform's own signs on each run are folded in.
+template <int N, int EPL>
+__device__ __forceinline__ uint32_t decode_sign_word(uint64_t sign_key, uint64_t j, int l)
+{
+    constexpr int LPT = N / EPL, RL = EPL / 2, HP = EPL / 4;
+    const uint32_t sig = hx_sigma_bits<LPT>(l);
+    const uint32_t a0 = (uint32_t)l * RL, b0 = (uint32_t)N / 2 + (uint32_t)l * RL;
+    const uint64_t wa = mix64(mix64(sign_key ^ j) ^ (uint64_t)(a0 >> 6));
+    const uint64_t wb = mix64(mix64(sign_key ^ j) ^ (uint64_t)(b0 >> 6));
+    const uint32_t sa = (uint32_t)(wa >> (a0 & 63)), sbb = (uint32_t)(wb >> (b0 & 63));
+    return sign_word<EPL>([&](int i) {
+        const int m = i >> 1;
+        return m < HP ? (((sa >> i) & 1u) ^ (sig & 1u)) : (((sbb >> (i - 2 * HP)) & 1u) ^ (sig >> 1));
+    });
+}
+
 template <int N, int D, int EPL, bool DITHER, bool F32OUT, bool FIXED>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeArgs a)
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kDecodeWarps * TPW;
+    constexpr int NP = EPL / 2, HP = NP / 2, RL = EPL / 2;
     extern __shared__ __align__(16) uint32_t sm[];
-    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(sm);
+    const int ywords = a.sign_words ? (int)a.tiles_per_row * LPT : 0;  // sign words cached per block
+    uint32_t *ytab = sm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane % LPT, gid = warp * TPW + lane / LPT;
     const unsigned mask = group_mask<LPT>(lane);
-    uint32_t *wbuf = sm + 2 * a.sign_words + gid * group_words(a.wmax);
-    build_sign_table<N>(sign_tab, a.sign_words, a.sign_key);
+    uint32_t *wbuf = sm + ((ywords + 3) & ~3) + gid * group_words(a.wmax);
+    for (int i = threadIdx.x; i < ywords; i += blockDim.x)
+        ytab[i] = decode_sign_word<N, EPL>(a.sign_key, (uint64_t)(i / LPT), i % LPT);
     __syncthreads();
 
     for (int64_t t = (int64_t)blockIdx.x * GPB + gid; t < a.ntiles; t += (int64_t)gridDim.x * GPB) {
-        float pt[EPL];
-        uint32_t sb;
-        const bool bad = parse_tile<N, D, EPL, FIXED>(a, t, wbuf, mask, l, pt, sb);
-        if constexpr (DITHER) {
-            if (!bad && sb) sub_dither<D, EPL>(mix64(a.dither_key ^ (uint64_t)t), l, pt, a.a2);
-        }
-        const float scale = bf16_bits_to_float(sb) * (1.0f / N);  // exact: a power-of-two step
-        float v[EPL];
+        uint32_t u[EPL], cb, sb;
+        bool small;
+        const bool bad = parse_symbols<N, D, EPL, FIXED>(a, t, wbuf, mask, l, u, cb, sb, small);
+        float2 v[NP];
+        if constexpr (D != 2 && !DITHER) {
+            // v = (Delta / n) y = (Delta / 2n) t with t = 2y an integer: t + 1.5 2^23
+            // read as a float, times Delta / 2n, minus 1.5 2^23 Delta / 2n (exact:
+            // 9 significant bits) in one fma -- the single rounding of t Delta / 2n.
+            // Exact while |t| < 2^22, which a lane whose codes all have unary
+            // parts under 32 bits guarantees (u < 2^20); otherwise convert.
+            int32_t tt[EPL];
+            doubled_from_symbols<D, EPL>(u, cb, tt);
+            const float s2 = bf16_bits_to_float(sb) * (0.5f / N);  // exact: a power-of-two step
+            if (small) {
+                const float2 sc = splat2(s2), off = splat2(-12582912.0f * s2);
 #pragma unroll
-        for (int r = 0; r < EPL; r++) v[r] = pt[r] * scale;
-        fwht<EPL, LPT>(v, mask, l);
-        const uint64_t j = (uint32_t)t - fast_div((uint32_t)t, a.tpr_div) * (uint32_t)a.tiles_per_row;
-        const uint32_t sbits = sign_bits<N, EPL>(sign_tab, a.sign_words, a.sign_key, j, l);
+                for (int m = 0; m < NP; m++)
+                    v[m] = fma2(make_float2(__int_as_float(tt[2 * m] + kMagicBias), __int_as_float(tt[2 * m + 1] + kMagicBias)),
+                                sc, off);
+            } else {
 #pragma unroll
-        for (int r = 0; r < EPL; r++) v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
-        const int64_t e0 = t * N + (int64_t)l * EPL;
-        if constexpr (F32OUT) {
-            float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(a.y) + e0);
-#pragma unroll
-            for (int i = 0; i < EPL / 4; i++) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int m = 0; m < NP; m++) v[m] = make_float2((float)tt[2 * m] * s2, (float)tt[2 * m + 1] * s2);
+            }
         } else {
-            uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.y) + e0);
+            float pt[EPL];
+            points_from_symbols<D, EPL>(u, cb, a.a2, pt);
+            if constexpr (DITHER) {
+                if (!bad && sb) sub_dither<D, EPL>(mix64(a.dither_key ^ (uint64_t)t), l, pt, a.a2);
+            }
+            const float2 scale = splat2(bf16_bits_to_float(sb) * (1.0f / N));  // exact: a power-of-two step
 #pragma unroll
-            for (int i = 0; i < EPL / 8; i++) {
-                uint32_t qq[4];
+            for (int m = 0; m < NP; m++) v[m] = mul2(make_float2(pt[2 * m], pt[2 * m + 1]), scale);
+        }
+        fwht_hx<EPL, LPT>(v, mask, l);
+        const uint64_t j = (uint32_t)t - fast_div((uint32_t)t, a.tpr_div) * (uint32_t)a.tiles_per_row;
+        const uint32_t Y = ywords ? ytab[j * LPT + l] : decode_sign_word<N, EPL>(a.sign_key, j, l);
+        const int64_t eA = t * N + (int64_t)l * RL, eB = eA + N / 2;
+        if constexpr (F32OUT) {
 #pragma unroll
-                for (int h = 0; h < 4; h++) {
-                    const __nv_bfloat162 p2 = __floats2bfloat162_rn(v[8 * i + 2 * h], v[8 * i + 2 * h + 1]);
-                    qq[h] = *reinterpret_cast<const uint32_t *>(&p2);
+            for (int run = 0; run < 2; run++) {
+                float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(a.y) + (run ? eB : eA));
+#pragma unroll
+                for (int i = 0; i < RL / 4; i++) {
+                    const int m0 = run * HP + 2 * i;
+                    const uint32_t s0 = Y << m0, s1 = Y << (m0 + 1);
+                    o[i] = make_float4(__uint_as_float(__float_as_uint(v[m0].x) ^ ((s0 << 16) & 0x80000000u)),
+                                       __uint_as_float(__float_as_uint(v[m0].y) ^ (s0 & 0x80000000u)),
+                                       __uint_as_float(__float_as_uint(v[m0 + 1].x) ^ ((s1 << 16) & 0x80000000u)),
+                                       __uint_as_float(__float_as_uint(v[m0 + 1].y) ^ (s1 & 0x80000000u)));
                 }
-                o[i] = make_uint4(qq[0], qq[1], qq[2], qq[3]);
+            }
+        } else {
+#pragma unroll
+            for (int run = 0; run < 2; run++) {
+                uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.y) + (run ? eB : eA));
+#pragma unroll
+                for (int i = 0; i < RL / 8; i++) {
+                    uint32_t qq[4];
+#pragma unroll
+                    for (int h = 0; h < 4; h++) {
+                        const int m = run * HP + 4 * i + h;
+                        const __nv_bfloat162 p2 = __floats2bfloat162_rn(v[m].x, v[m].y);
+                        qq[h] = *reinterpret_cast<const uint32_t *>(&p2) ^ ((Y << m) & 0x80008000u);
+                    }
+                    o[i] = make_uint4(qq[0], qq[1], qq[2], qq[3]);
+                }
             }
         }
         if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
@@ -122,20 +180,45 @@ __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(con
         float acc = 0.0f;
         for (int64_t j = lane / LPT; j < tpr; j += TPW) {
             const int64_t t = row * tpr + j;
-            float pt[EPL];
-            uint32_t sb;
-            const bool bad = parse_tile<N, D, EPL, FIXED>(a, t, wbuf, mask, l, pt, sb);
+            uint32_t u[EPL], cb, sb;
+            bool small;
+            const bool bad = parse_symbols<N, D, EPL, FIXED>(a, t, wbuf, mask, l, u, cb, sb, small);
             const float4 *src = reinterpret_cast<const float4 *>(xt + j * N + l * EPL);
-            float dot = 0.0f;
+            float2 d2 = make_float2(0.0f, 0.0f);
+            float step;  // the tile's weight on the dot: Delta / n for points, Delta / 2n for doubled points
+            if constexpr (D != 2) {
+                // t = 2y: t + 1.5 2^23 read as a float minus 1.5 2^23 is exact while
+                // |t| < 2^22 (every unary part under 32 bits); otherwise convert
+                int32_t tt[EPL];
+                doubled_from_symbols<D, EPL>(u, cb, tt);
+                const float2 moff = splat2(-12582912.0f);
 #pragma unroll
-            for (int c = 0; c < EPL / 4; c++) {
-                const float4 xv = src[c ^ (l & SW)];
-                dot = fmaf(pt[4 * c], xv.x, dot);
-                dot = fmaf(pt[4 * c + 1], xv.y, dot);
-                dot = fmaf(pt[4 * c + 2], xv.z, dot);
-                dot = fmaf(pt[4 * c + 3], xv.w, dot);
+                for (int c = 0; c < EPL / 4; c++) {
+                    const float4 xv = src[c ^ (l & SW)];
+                    float2 p0, p1;
+                    if (small) {
+                        p0 = add2(make_float2(__int_as_float(tt[4 * c] + kMagicBias), __int_as_float(tt[4 * c + 1] + kMagicBias)), moff);
+                        p1 = add2(make_float2(__int_as_float(tt[4 * c + 2] + kMagicBias), __int_as_float(tt[4 * c + 3] + kMagicBias)), moff);
+                    } else {
+                        p0 = make_float2((float)tt[4 * c], (float)tt[4 * c + 1]);
+                        p1 = make_float2((float)tt[4 * c + 2], (float)tt[4 * c + 3]);
+                    }
+                    d2 = fma2(p0, make_float2(xv.x, xv.y), d2);
+                    d2 = fma2(p1, make_float2(xv.z, xv.w), d2);
+                }
+                step = bf16_bits_to_float(sb) * (0.5f / N);
+            } else {
+                float pt[EPL];
+                points_from_symbols<D, EPL>(u, cb, a.a2, pt);
+#pragma unroll
+                for (int c = 0; c < EPL / 4; c++) {
+                    const float4 xv = src[c ^ (l & SW)];
+                    d2 = fma2(make_float2(pt[4 * c], pt[4 * c + 1]), make_float2(xv.x, xv.y), d2);
+                    d2 = fma2(make_float2(pt[4 * c + 2], pt[4 * c + 3]), make_float2(xv.z, xv.w), d2);
+                }
+                step = bf16_bits_to_float(sb) * (1.0f / N);
             }
-            acc = fmaf(bf16_bits_to_float(sb) * (1.0f / N), dot, acc);
+            acc = fmaf(step, __fadd_rn(d2.x, d2.y), acc);
             if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
         }
         __syncwarp();
@@ -153,6 +236,10 @@ constexpr int epl_for() { return N == 64 ? 8 : (N <= 256 ? 16 : 32); }
 
 template <int N>
 constexpr int groups_per_block() { return kDecodeWarps * (32 / (N / epl_for<N>())); }
+// the decoder: at least 16 per lane (the half-exchange transform's two runs
+// then hold whole vectors and 16-byte stores)
+template <int N>
+constexpr int epl_dec() { return N <= 256 ? 16 : 32; }
 
 template <typename K>
 cudaError_t grid_for(K kern, size_t smem, int64_t work_blocks, unsigned &blocks)
@@ -173,8 +260,9 @@ cudaError_t grid_for(K kern, size_t smem, int64_t work_blocks, unsigned &blocks)
 template <int N, int D, bool DITHER, bool F32OUT>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
-    constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
-    const size_t smem = (size_t)a.sign_words * 8 + (size_t)GPB * group_words(a.wmax) * 4;
+    constexpr int EPL = epl_dec<N>(), GPB = kDecodeWarps * (32 / (N / EPL));
+    const size_t ywords = a.sign_words ? (size_t)a.tiles_per_row * (N / EPL) : 0;
+    const size_t smem = ((ywords + 3) & ~(size_t)3) * 4 + (size_t)GPB * group_words(a.wmax) * 4;
     auto kern = a.slot ? decode_kernel<N, D, EPL, DITHER, F32OUT, true> : decode_kernel<N, D, EPL, DITHER, F32OUT, false>;
     unsigned blocks = 0;
     cudaError_t e = grid_for(kern, smem, (a.ntiles + GPB - 1) / GPB, blocks);

@@ -369,6 +369,16 @@ __device__ __forceinline__ void or_bits32(uint32_t *buf, uint32_t pos, uint32_t 
     if (sh && (int)sh + len > 32) atomicOr(&buf[w + 1], v >> (32 - sh));
 }
 
+// or_bits32 confined to the buffer's first `limit` words: a write past them
+// is dropped (the caller's lengths already keep every write inside; this
+// only guards the buffer against an inconsistent length).
+__device__ __forceinline__ void or_bits32_lim(uint32_t *buf, uint32_t pos, uint32_t v, int len, uint32_t limit)
+{
+    const uint32_t w = pos >> 5, sh = pos & 31;
+    if (w < limit) atomicOr(&buf[w], v << sh);
+    if (sh && (int)sh + len > 32 && w + 1 < limit) atomicOr(&buf[w + 1], v >> (32 - sh));
+}
+
 // `len` (<= 32) bits at bit `pos` of a word buffer (buf[pos/32 + 1] must be
 // readable).
 __device__ __forceinline__ uint32_t get_bits(const uint32_t *buf, uint32_t pos, int len)

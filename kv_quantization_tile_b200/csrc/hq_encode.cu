@@ -25,6 +25,7 @@
 // subtractive dither).
 #include <cuda_bf16.h>
 
+#include "hq_fast.cuh"
 #include "hq_internal.h"
 
 namespace hq {
@@ -306,6 +307,473 @@ __device__ __forceinline__ void pack_lane(uint32_t *tbuf, int l, int k, uint32_t
     }
 }
 
+// ---------------------------------------------------------------- packed path
+// Unpack lane l's EPL raw coordinates into pairs and apply the random signs of
+// the sign word Y (pair m's mask is (Y << m) & 0x80008000, see sign_word).
+template <int EPL, bool F32IN>
+__device__ __forceinline__ void unpack_signed(const RawTile<EPL, F32IN> &r, uint32_t Y, float2 (&P)[EPL / 2])
+{
+    if constexpr (F32IN) {
+#pragma unroll
+        for (int i = 0; i < EPL / 4; i++) {
+            const uint32_t qq[4] = { r.q[i].x, r.q[i].y, r.q[i].z, r.q[i].w };
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int m = 2 * i + h;
+                const uint32_t sm = Y << m;
+                P[m] = make_float2(__uint_as_float(qq[2 * h] ^ ((sm << 16) & 0x80000000u)),
+                                   __uint_as_float(qq[2 * h + 1] ^ (sm & 0x80000000u)));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL / 8; i++) {
+            const uint32_t qq[4] = { r.q[i].x, r.q[i].y, r.q[i].z, r.q[i].w };
+#pragma unroll
+            for (int h = 0; h < 4; h++) {
+                const int m = 4 * i + h;
+                const uint32_t w = qq[h] ^ ((Y << m) & 0x80008000u);
+                P[m] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+            }
+        }
+    }
+}
+
+// The sign word of lane l of column tile j (see sign_word): the lane's
+// coordinates l EPL .. l EPL + EPL - 1 in pair order.
+template <int N, int EPL>
+__device__ __forceinline__ uint32_t encode_sign_word(uint64_t sign_key, uint64_t j, int l)
+{
+    const uint32_t i0 = (uint32_t)l * EPL;
+    const uint64_t w = mix64(mix64(sign_key ^ j) ^ (uint64_t)(i0 >> 6));
+    const uint32_t sb = (uint32_t)(w >> (i0 & 63));
+    return sign_word<EPL>([&](int i) { return (sb >> i) & 1u; });
+}
+
+// Dither of the D-vector whose first coordinate is tile coordinate c0 (c0 a
+// multiple of D); for D < 4, r4 carries one hash over the vectors of a group
+// of four coordinates (call with consecutive vectors in order).
+template <int D>
+__device__ __forceinline__ void dither_at(uint64_t tile_key, uint32_t c0, float (&r4)[4], float (&delta)[D],
+                                          const A2Consts &a2)
+{
+    if constexpr (D >= 4) {
+#pragma unroll
+        for (int b = 0; b < D / 4; b++) {
+            uniform4(tile_key, c0 / 4 + b, r4);
+#pragma unroll
+            for (int k = 0; k < 4; k++) delta[4 * b + k] = box_dither<D>(r4[k], 4 * b + k, a2);
+        }
+    } else {
+        if ((c0 & 3) == 0) uniform4(tile_key, c0 / 4, r4);
+#pragma unroll
+        for (int m = 0; m < D; m++) delta[m] = box_dither<D>(r4[(c0 & 3) + m], m, a2);
+    }
+}
+
+// Nearest points of lane l's two runs after the half-exchange transform (run
+// A: tile coordinates RL l .., run B: N/2 + RL l .., RL = EPL / 2) of
+// v / Delta [+ dither], stripped and zigzagged into u (run A's symbols, then
+// run B's, each in coordinate order).  sig: the transform's signs (bit 0: run
+// A negated, bit 1: run B).  Returns the coset bits (bit q: run A's vector q,
+// bit RL / D + q: run B's).  sb = 0: the all-zero tile.
+template <int N, int D, int EPL, bool DITHER>
+__device__ __forceinline__ uint32_t quantize_hx(const float2 (&P)[EPL / 2], uint32_t sb, uint32_t sig, uint64_t tkey,
+                                                int l, const A2Consts &a2, uint32_t (&u)[EPL])
+{
+    constexpr int NP = EPL / 2, HP = NP / 2, RL = EPL / 2, VPR = RL / D;
+    uint32_t cbits = 0;
+#pragma unroll
+    for (int r = 0; r < EPL; r++) u[r] = 0;
+    if (sb == 0) return 0;
+    const float inv = __frcp_rn(bf16_bits_to_float(sb));
+    const float2 ia = splat2((sig & 1u) ? -inv : inv), ib = splat2((sig & 2u) ? -inv : inv);
+    float2 X[NP];
+#pragma unroll
+    for (int m = 0; m < NP; m++) X[m] = mul2(P[m], m < HP ? ia : ib);
+    float r4[4];
+#pragma unroll
+    for (int run = 0; run < 2; run++) {
+        const uint32_t cbase = (run ? (uint32_t)N / 2 : 0u) + (uint32_t)l * RL;
+#pragma unroll
+        for (int q = 0; q < VPR; q++) {
+            float2 V[D > 1 ? D / 2 : 1];
+            float x[D];
+#pragma unroll
+            for (int m = 0; m < D; m++) {
+                const int i = q * D + m;  // coordinate within the run: pair i / 2, element i & 1
+                x[m] = (i & 1) ? X[run * HP + i / 2].y : X[run * HP + i / 2].x;
+            }
+            if constexpr (DITHER) {
+                float dl[D];
+                dither_at<D>(tkey, cbase + (uint32_t)(q * D), r4, dl, a2);
+#pragma unroll
+                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+            }
+            uint32_t *uu = u + run * RL + q * D;
+            int c = 0;
+            if constexpr (D == 8) {
+#pragma unroll
+                for (int i = 0; i < 4; i++) V[i] = make_float2(x[2 * i], x[2 * i + 1]);
+                int32_t zb[8];
+                bool tie;
+                c = e8_fast(V, zb, tie);
+                if (tie) {  // several coordinates tie for the parity fix: the sequential rule
+                    int zz[8];
+                    float pp[8];
+                    nearest<8>(x, c, zz, pp, a2);
+#pragma unroll
+                    for (int i = 0; i < 8; i++) zb[i] = zz[i] + kMagicBias;
+                }
+#pragma unroll
+                for (int i = 0; i < 7; i++) {
+                    const int32_t t2 = (int32_t)(((uint32_t)zb[i] << 1) - ((uint32_t)kMagicBias << 1));  // 2 z
+                    uu[i] = (uint32_t)t2 ^ (uint32_t)(t2 >> 31);
+                }
+                const int32_t t7 = (zb[7] - kMagicBias) & ~1;  // 2 floor(z / 2)
+                uu[7] = (uint32_t)t7 ^ (uint32_t)(t7 >> 31);
+            } else {
+                int z[D];
+                float p[D];
+                nearest<D>(x, c, z, p, a2);
+#pragma unroll
+                for (int m = 0; m < D; m++) {
+                    int sv = z[m];
+                    if constexpr (D == 4) {
+                        if (m == D - 1) sv >>= 1;
+                    }
+                    uu[m] = zigzag(sv);
+                }
+            }
+            cbits |= (uint32_t)c << (run * VPR + q);
+        }
+    }
+    return cbits;
+}
+
+// OR `cnt` codes' k low bits (code i at bit pos + i k) into a zeroed image.
+template <int CNT>
+__device__ __forceinline__ void pack_low_run(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u)
+{
+    const uint32_t lowmask = (1u << k) - 1u;
+    if (k <= 4) {  // 8 codes per 32-bit word
+#pragma unroll
+        for (int r0 = 0; r0 < CNT; r0 += 8) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+            or_bits32(tbuf, pos + (uint32_t)r0 * k, acc, 8 * k);
+        }
+    } else {
+#pragma unroll
+        for (int r0 = 0; r0 < CNT; r0 += 4) {
+            uint64_t acc = 0;
+#pragma unroll
+            for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+            or_bits(tbuf, pos + (uint32_t)r0 * k, acc, 4 * k);
+        }
+    }
+}
+
+// OR `cnt` codes' unary parts (q = u >> k zeros, then a one), starting at bit
+// pos, into a zeroed image, eight codes at a time.
+template <int CNT>
+__device__ __forceinline__ void pack_unary_run(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u)
+{
+#pragma unroll
+    for (int r0 = 0; r0 < CNT; r0 += 8) {
+        uint32_t bm = 0, rel = 0;
+#pragma unroll
+        for (int m = 0; m < 8; m++) {
+            const uint32_t pbit = rel + (u[r0 + m] >> k);
+            bm |= shl32(1u, pbit);
+            rel = pbit + 1;
+        }
+        if (rel <= 32) {
+            or_bits32(tbuf, pos, bm, (int)rel);
+        } else {  // a long code: set the terminators one by one
+            uint32_t pr = pos;
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                pr += u[r0 + m] >> k;
+                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
+                ++pr;
+            }
+        }
+        pos += rel;
+    }
+}
+
+// Pack lane l's two runs into a zeroed shared-memory image: coset bits, low
+// parts, and unary parts starting uoffA / uoffB bits into the unary section.
+template <int N, int D, int EPL>
+__device__ __forceinline__ void pack_hx(uint32_t *tbuf, int l, int k, uint32_t cbits, const uint32_t (&u)[EPL],
+                                        uint32_t uoffA, uint32_t uoffB)
+{
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
+    constexpr int RL = EPL / 2, VPR = RL / D;
+    if constexpr (C > 0) {
+        or_bits32(tbuf, (uint32_t)l * VPR, cbits & ((1u << VPR) - 1u), VPR);
+        or_bits32(tbuf, (uint32_t)(N / (2 * D)) + (uint32_t)l * VPR, cbits >> VPR, VPR);
+    }
+    if (k) {
+        pack_low_run<RL>(tbuf, (uint32_t)C + (uint32_t)l * RL * (uint32_t)k, k, u);
+        pack_low_run<RL>(tbuf, (uint32_t)C + ((uint32_t)N / 2 + (uint32_t)l * RL) * (uint32_t)k, k, u + RL);
+    }
+    const uint32_t ubase = (uint32_t)C + (uint32_t)N * (uint32_t)k;
+    pack_unary_run<RL>(tbuf, ubase + uoffA, k, u);
+    pack_unary_run<RL>(tbuf, ubase + uoffB, k, u + RL);
+}
+
+// The same as quantize_hx with the symbols as exact binary32 integers in
+// pairs (U[m]: symbols 2m, 2m + 1 of the lane's run-A-then-run-B order).  E8
+// uses e8_symbols (the fma pipe); a vector whose parity fix ties between
+// coordinates, and the other lattices, take the scalar nearest point.
+template <int N, int D, int EPL, bool DITHER>
+__device__ __forceinline__ uint32_t quantize_hx_f(const float2 (&P)[EPL / 2], uint32_t sb, uint32_t sig,
+                                                  uint64_t tkey, int l, const A2Consts &a2, float2 (&U)[EPL / 2])
+{
+    constexpr int NP = EPL / 2, HP = NP / 2, RL = EPL / 2, VPR = RL / D;
+#pragma unroll
+    for (int m = 0; m < NP; m++) U[m] = make_float2(0.0f, 0.0f);
+    if (sb == 0) return 0;
+    uint32_t cbits = 0;
+    const float inv = __frcp_rn(bf16_bits_to_float(sb));
+    const float2 ia = splat2((sig & 1u) ? -inv : inv), ib = splat2((sig & 2u) ? -inv : inv);
+    float2 X[NP];
+#pragma unroll
+    for (int m = 0; m < NP; m++) X[m] = mul2(P[m], m < HP ? ia : ib);
+    float r4[4];
+#pragma unroll
+    for (int run = 0; run < 2; run++) {
+        const uint32_t cbase = (run ? (uint32_t)N / 2 : 0u) + (uint32_t)l * RL;
+#pragma unroll
+        for (int q = 0; q < VPR; q++) {
+            float x[D];
+#pragma unroll
+            for (int m = 0; m < D; m++) {
+                const int i = q * D + m;  // coordinate within the run: pair i / 2, element i & 1
+                x[m] = (i & 1) ? X[run * HP + i / 2].y : X[run * HP + i / 2].x;
+            }
+            if constexpr (DITHER) {
+                float dl[D];
+                dither_at<D>(tkey, cbase + (uint32_t)(q * D), r4, dl, a2);
+#pragma unroll
+                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
+            }
+            float us[D];
+            int c = 0;
+            bool slow = true;
+            if constexpr (D == 8) {
+                float2 V[4], W[4];
+#pragma unroll
+                for (int i = 0; i < 4; i++) V[i] = make_float2(x[2 * i], x[2 * i + 1]);
+                bool tie;
+                c = e8_symbols(V, W, tie);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    us[2 * i] = W[i].x;
+                    us[2 * i + 1] = W[i].y;
+                }
+                slow = tie;  // several coordinates tie for the parity fix: the sequential rule
+            }
+            if (slow) {
+                int z[D];
+                float p[D];
+                nearest<D>(x, c, z, p, a2);
+#pragma unroll
+                for (int m = 0; m < D; m++) {
+                    int sv = z[m];
+                    if constexpr (D == 8 || D == 4) {
+                        if (m == D - 1) sv >>= 1;  // floor(z / 2): its parity follows from the even sum
+                    }
+                    us[m] = (float)zigzag(sv);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < D; m++) {
+                const int i = q * D + m;
+                if (i & 1) U[run * HP + i / 2].y = us[m];
+                else U[run * HP + i / 2].x = us[m];
+            }
+            cbits |= (uint32_t)c << (run * VPR + q);
+        }
+    }
+    return cbits;
+}
+
+// 2^e as a binary32 (e in -126 .. 127)
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// Sums over run A and run B of floor(u / 2^k) for one k: an fma rounded down
+// against 1.5 2^23 leaves 1.5 2^23 + floor(u 2^-k), whose bit patterns are
+// added as integers (the common bias removed at the end).
+template <int EPL>
+__device__ __forceinline__ void shifted_sums(const float2 (&U)[EPL / 2], int k, uint32_t &sa, uint32_t &sbv)
+{
+    constexpr int NP = EPL / 2, HP = NP / 2;
+    const float2 sk = splat2(exp2i(-k)), M2 = splat2(12582912.0f);
+    uint32_t a = 0, b = 0;
+#pragma unroll
+    for (int m = 0; m < NP; m++) {
+        const float2 qb = __ffma2_rd(U[m], sk, M2);
+        const uint32_t pair = (uint32_t)__float_as_int(qb.x) + (uint32_t)__float_as_int(qb.y);
+        if (m < HP) a += pair;
+        else b += pair;
+    }
+    constexpr uint32_t kBiasRun = (uint32_t)kMagicBias * (uint32_t)(EPL / 2);  // EPL / 2 biases, mod 2^32
+    sa = a - kBiasRun;
+    sbv = b - kBiasRun;
+}
+
+// Rice parameter from float symbols: as rice_param (exact argmin of the
+// tile's coded length, smallest k on ties; one pass over k0-1, k0, k0+1, a
+// walk only if the optimum lies outside).  partA / partB: this lane's
+// sum(u >> k) over run A / run B at the returned k.
+template <int N, int EPL, int LPT>
+__device__ __forceinline__ int rice_param_f(const float2 (&U)[EPL / 2], unsigned mask, int k_hint, uint32_t &partA,
+                                            uint32_t &partB)
+{
+    int k = k_hint;
+    const int km = k > 0 ? k - 1 : 0;
+    uint32_t a0, b0, a1, b1, a2, b2;
+    shifted_sums<EPL>(U, km, a0, b0);
+    shifted_sums<EPL>(U, km + 1, a1, b1);
+    shifted_sums<EPL>(U, km + 2, a2, b2);
+    const uint32_t S0 = group_sum<LPT>(mask, a0 + b0), S1 = group_sum<LPT>(mask, a1 + b1),
+                   S2 = group_sum<LPT>(mask, a2 + b2);
+    bool up = false, down = false;
+    if (k == 0) {
+        if (S0 - S1 <= (uint32_t)N) {
+            partA = a0; partB = b0;          // C(1) >= C(0)
+        } else if (S1 - S2 <= (uint32_t)N) {
+            k = 1; partA = a1; partB = b1;   // C(1) < C(0), C(2) >= C(1)
+        } else {
+            k = 2; partA = a2; partB = b2; up = true;
+        }
+    } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
+        k = km; partA = a0; partB = b0; down = true;
+    } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
+        k = k + 1; partA = a2; partB = b2; up = true;
+    } else {
+        partA = a1; partB = b1;
+    }
+    while (down && k > 0) {
+        uint32_t da, db;
+        shifted_sums<EPL>(U, k - 1, da, db);
+        if (group_sum<LPT>(mask, da + db) - group_sum<LPT>(mask, partA + partB) > (uint32_t)N) break;
+        --k; partA = da; partB = db;
+    }
+    while (up && k < 15) {
+        uint32_t ua, ub;
+        shifted_sums<EPL>(U, k + 1, ua, ub);
+        if (group_sum<LPT>(mask, partA + partB) - group_sum<LPT>(mask, ua + ub) <= (uint32_t)N) break;
+        ++k; partA = ua; partB = ub;
+    }
+    return k;
+}
+
+// Low parts and unary parts of one run of 8 float symbols (4 pairs) for
+// k <= 4 and a unary span of at most 32 bits: the low word is sum_i low_i 2^(k i)
+// formed exactly in binary32 as two halves of 4 codes (16 bits at most), the
+// unary bitmap by Horner from the last code, bm = ((bm << 1) | 1) << q, with q
+// taken from the biased floor pattern (its low 5 bits are q's).
+__device__ __forceinline__ void run_words8(const float2 *U, int k, uint32_t &low, uint32_t &unary)
+{
+    const float2 sk = splat2(exp2i(-k)), M2 = splat2(12582912.0f), mpk = splat2(-exp2i(k));
+    const float pk = exp2i(k), pk2 = exp2i(2 * k);
+    float c[4];
+    uint32_t qb[8];
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        const float2 b = __ffma2_rd(U[m], sk, M2);              // 1.5 2^23 + q
+        const float2 lo = fma2(sub2(b, M2), mpk, U[m]);         // u - 2^k q
+        c[m] = __fmaf_rn(lo.y, pk, lo.x);
+        qb[2 * m] = (uint32_t)__float_as_int(b.x);
+        qb[2 * m + 1] = (uint32_t)__float_as_int(b.y);
+    }
+    const float h0 = __fmaf_rn(c[1], pk2, c[0]), h1 = __fmaf_rn(c[3], pk2, c[2]);  // < 2^16: exact
+    const uint32_t b0 = (uint32_t)__float_as_int(__fadd_rn(h0, 8388608.0f));       // 2^23 + h0
+    const uint32_t b1 = (uint32_t)__float_as_int(__fadd_rn(h1, 8388608.0f));
+    low = (b1 << (4 * k)) + b0 - (0x4B000000u << (4 * k)) - 0x4B000000u;
+    uint32_t bm = 0;
+#pragma unroll
+    for (int i = 7; i >= 0; i--) bm = __funnelshift_l(0u, bm * 2u + 1u, qb[i]);
+    unary = bm;
+}
+
+// OR `cnt` codes' k low bits into a zeroed image, writes confined to the
+// image's first `limit` words (as pack_low_run).
+template <int CNT>
+__device__ __forceinline__ void pack_low_run_lim(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u, uint32_t limit)
+{
+    const uint32_t lowmask = (1u << k) - 1u;
+#pragma unroll
+    for (int r0 = 0; r0 < CNT; r0 += 4) {  // 4 codes of up to 15 bits: at most 60 bits, as two 32-bit halves
+        uint64_t acc = 0;
+#pragma unroll
+        for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
+        const uint32_t p = pos + (uint32_t)r0 * k;
+        or_bits32_lim(tbuf, p, (uint32_t)acc, 4 * k < 32 ? 4 * k : 32, limit);
+        if (4 * k > 32) or_bits32_lim(tbuf, p + 32, (uint32_t)(acc >> 32), 4 * k - 32, limit);
+    }
+}
+
+// OR `cnt` codes' unary parts into a zeroed image one terminator at a time,
+// writes confined to the image's first `limit` words.
+template <int CNT>
+__device__ __forceinline__ void pack_unary_run_lim(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u,
+                                                   uint32_t limit)
+{
+#pragma unroll
+    for (int m = 0; m < CNT; m++) {
+        pos += u[m] >> k;
+        if ((pos >> 5) < limit) atomicOr(&tbuf[pos >> 5], 1u << (pos & 31));
+        ++pos;
+    }
+}
+
+// Pack lane l's two runs of float symbols into a zeroed shared-memory image
+// (as pack_hx).  spanA / spanB: the runs' unary bits (sum of q + 1); limit:
+// the words of the group's image from tbuf on (no write goes past them).
+template <int N, int D, int EPL>
+__device__ __forceinline__ void pack_hx_f(uint32_t *tbuf, int l, int k, uint32_t cbits, const float2 (&U)[EPL / 2],
+                                          uint32_t uoffA, uint32_t uoffB, uint32_t spanA, uint32_t spanB,
+                                          uint32_t limit)
+{
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
+    constexpr int RL = EPL / 2, VPR = RL / D, HP = EPL / 4;
+    if constexpr (C > 0) {
+        or_bits32_lim(tbuf, (uint32_t)l * VPR, cbits & ((1u << VPR) - 1u), VPR, limit);
+        or_bits32_lim(tbuf, (uint32_t)(N / (2 * D)) + (uint32_t)l * VPR, cbits >> VPR, VPR, limit);
+    }
+    const uint32_t lowA = (uint32_t)C + (uint32_t)l * RL * (uint32_t)k;
+    const uint32_t lowB = (uint32_t)C + ((uint32_t)N / 2 + (uint32_t)l * RL) * (uint32_t)k;
+    const uint32_t ubase = (uint32_t)C + (uint32_t)N * (uint32_t)k;
+    if (RL == 8 && k <= 4 && spanA <= 32 && spanB <= 32) {
+        uint32_t wl, wu;
+        run_words8(U, k, wl, wu);
+        if (k) or_bits32_lim(tbuf, lowA, wl, 8 * k, limit);
+        or_bits32_lim(tbuf, ubase + uoffA, wu, (int)spanA, limit);
+        run_words8(U + HP, k, wl, wu);
+        if (k) or_bits32_lim(tbuf, lowB, wl, 8 * k, limit);
+        or_bits32_lim(tbuf, ubase + uoffB, wu, (int)spanB, limit);
+    } else {
+        uint32_t u[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL / 2; m++) {
+            u[2 * m] = (uint32_t)U[m].x;
+            u[2 * m + 1] = (uint32_t)U[m].y;
+        }
+        if (k) {
+            pack_low_run_lim<RL>(tbuf, lowA, k, u, limit);
+            pack_low_run_lim<RL>(tbuf, lowB, k, u + RL, limit);
+        }
+        pack_unary_run_lim<RL>(tbuf, ubase + uoffA, k, u, limit);
+        pack_unary_run_lim<RL>(tbuf, ubase + uoffB, k, u + RL, limit);
+    }
+}
+
 }  // namespace
 
 // Resident blocks per SM the compiler must fit registers for: 4 (64 registers)
@@ -319,27 +787,26 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
     constexpr int NCW = kEncodeWarps - 1;  // compute warps; the last warp scans and stores
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = NCW * TPW;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;  // coset bits per tile
-    constexpr int WPT = N / 64 > 0 ? N / 64 : 1;          // sign words per tile
-    static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
+    constexpr int RL = EPL / 2;                        // coordinates per run
+    static_assert(EPL % D == 0 && RL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32 && LPT >= 2, "layout");
     constexpr int kAll = kEncodeWarps * 32, kCompute = NCW * 32;
 
     const int G = a.tiles_per_group;
     const int T = GPB * G;  // tiles per chunk
+    const int ywords = a.sign_words ? (int)a.tiles_per_row * LPT : 0;  // sign words cached per block
     extern __shared__ __align__(16) uint32_t smem[];
-    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);      // a.sign_words
-    const uint32_t gstride = ((uint32_t)G * a.wmax + 3u) & ~3u;                        // words per group image
-    uint32_t *stage0 = smem + 2 * ((a.sign_words + 1) & ~1);                           // 2 x GPB x gstride
-    uint32_t *meta0 = stage0 + (size_t)2 * GPB * gstride;                              // 2 x (2T + GPB)
+    uint32_t *ytab = smem;                                                     // [tiles_per_row][LPT]
+    const uint32_t gstride = ((uint32_t)G * a.wmax + 3u) & ~3u;                // words per group image
+    uint32_t *stage0 = smem + ((ywords + 3) & ~3);                             // 2 x GPB x gstride
+    uint32_t *meta0 = stage0 + (size_t)2 * GPB * gstride;                      // 2 x (2T + GPB)
     __shared__ uint32_t s_chunk[2];
-    __shared__ uint32_t s_goff[32];
+    __shared__ uint32_t s_goff[64];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // per-block table of sign words for every column tile
-    for (int i = tid; i < a.sign_words; i += kAll) {
-        const uint64_t j = (uint64_t)(i / WPT), m = (uint64_t)(i % WPT);
-        sign_tab[i] = mix64(mix64(a.sign_key ^ j) ^ m);
-    }
+    // per-block table of every column tile's sign words
+    for (int i = tid; i < ywords; i += kAll)
+        ytab[i] = encode_sign_word<N, EPL>(a.sign_key, (uint64_t)(i / LPT), i % LPT);
     __syncthreads();
 
     if (warp < NCW) {
@@ -347,6 +814,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
         const int l = lane % LPT;
         const int gid = warp * TPW + lane / LPT;
         const unsigned mask = group_mask<LPT>(lane);
+        const uint32_t sig = hx_sigma_bits<LPT>(l);
         for (int it = 0;; it++) {
             const int b = it & 1;
             if (it >= 2) named_sync(kBarFree0 + b, kAll);  // the store warp is done with image b
@@ -379,46 +847,40 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
             for (int gi = 0; gi < G; gi++) {
                 const int64_t t = t_first + gi;
                 const bool active = t < a.ntiles;
-                // ---- signs (v = s . w)
-                const uint64_t j = jj;
-                const uint32_t i0 = (uint32_t)l * EPL;
-                uint64_t sw;
-                if (a.sign_words) sw = sign_tab[j * WPT + (i0 >> 6)];
-                else sw = mix64(mix64(a.sign_key ^ j) ^ (uint64_t)(i0 >> 6));
-                const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
-                float v[EPL];
+                // ---- signs (v = s . w), as pairs
+                const uint32_t Y = ywords ? ytab[jj * LPT + l] : encode_sign_word<N, EPL>(a.sign_key, jj, l);
+                float2 v[EPL / 2];
                 if (active) {
-                    unpack_raw<EPL, F32IN>(raw, v);
-    #pragma unroll
-                    for (int r = 0; r < EPL; r++)
-                        v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
+                    unpack_signed<EPL, F32IN>(raw, Y, v);
                     if (gi + 1 < G && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
                 } else {
-    #pragma unroll
-                    for (int r = 0; r < EPL; r++) v[r] = 0.0f;
+#pragma unroll
+                    for (int m = 0; m < EPL / 2; m++) v[m] = make_float2(0.0f, 0.0f);
                 }
                 if (++jj == tpr) jj = 0;
 
                 // ---- scale (sum of squares is sign-blind) + rotation
-                const float S = sumsq<EPL, LPT>(v, mask);
-                fwht<EPL, LPT>(v, mask, l);
+                const float S = sumsq_pairs<EPL, LPT, !F32IN>(v, mask);
+                fwht_hx<EPL, LPT>(v, mask, l);
                 bool nonfinite;
                 const uint32_t sb = tile_scale_bits(S, a.c, nonfinite);
                 if (active && nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
 
-                // ---- nearest point, strip, zigzag
-                uint32_t u[EPL];
+                // ---- nearest point, strip, zigzag (symbols as exact binary32 integers)
+                float2 U[EPL / 2];
                 const uint64_t tkey = DITHER ? mix64(a.dither_key ^ (uint64_t)t) : 0ull;
-                const uint32_t cbits = quantize_lane<D, EPL, DITHER>(v, sb, tkey, l, a.a2, u);
+                const uint32_t cbits = quantize_hx_f<N, D, EPL, DITHER>(v, sb, sig, tkey, l, a.a2, U);
 
-                // ---- Rice parameter (exact argmin)
-                uint32_t part;  // this lane's sum(u >> k) at the chosen k
-                const int k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
+                // ---- Rice parameter (exact argmin); this lane's sum(u >> k) per run
+                uint32_t partA, partB;
+                const int k = rice_param_f<N, EPL, LPT>(U, mask, a.k_hint, partA, partB);
 
-                // ---- lengths
-                const uint32_t ul = part + EPL;  // unary bits of this lane
-                const uint32_t uoff = group_excl_scan<LPT>(mask, ul, l);
-                const uint32_t utot = group_sum<LPT>(mask, ul);
+                // ---- lengths: run A's unary parts precede run B's in the tile
+                const uint32_t ulA = partA + RL, ulB = partB + RL;
+                const uint32_t totA = group_sum<LPT>(mask, ulA);
+                const uint32_t uoffA = group_excl_scan<LPT>(mask, ulA, l);
+                const uint32_t uoffB = totA + group_excl_scan<LPT>(mask, ulB, l);
+                const uint32_t utot = totA + group_sum<LPT>(mask, ulB);
                 const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)k + utot;
                 uint32_t W = active ? (bits + 31) >> 5 : 0;
                 const bool overflow = W > a.wmax;  // excluded by the bound; guards the image
@@ -426,7 +888,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 
                 // ---- pack into the group's image (zeroed at chunk start)
                 uint32_t *tbuf = gstage + goff;
-                if (active && !overflow) pack_lane<N, D, EPL>(tbuf, l, k, cbits, u, uoff);
+                if (active && !overflow) pack_hx_f<N, D, EPL>(tbuf, l, k, cbits, U, uoffA, uoffB, ulA, ulB, gstride - goff);
                 if (overflow && l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
                 if (l == 0) {
                     tile_w[gid * G + gi] = goff;
@@ -448,15 +910,24 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
             const uint32_t *tile_w = meta0 + (size_t)b * (2 * T + GPB);
             const uint32_t *tile_hdr = tile_w + T;
             const uint32_t *grp_w = tile_hdr + T;
+            // groups lane and lane + 32 (a block has at most 64 groups): their
+            // word offsets in the chunk by one scan over the 64 counts in order
+            static_assert(GPB <= 64, "store warp scans at most 64 groups");
             const uint32_t mine = lane < GPB ? grp_w[lane] : 0u;
-            uint32_t incl = mine;
+            const uint32_t mine2 = lane + 32 < GPB ? grp_w[lane + 32] : 0u;
+            uint32_t incl = mine, incl2 = mine2;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t o = __shfl_up_sync(FULL, incl, d);
-                if (lane >= d) incl += o;
+                const uint32_t o = __shfl_up_sync(FULL, incl, d), o2 = __shfl_up_sync(FULL, incl2, d);
+                if (lane >= d) {
+                    incl += o;
+                    incl2 += o2;
+                }
             }
-            const uint32_t total = __shfl_sync(FULL, incl, 31);
-            const uint32_t gexcl = incl - mine;  // group `lane`'s word offset in the chunk
+            const uint32_t half = __shfl_sync(FULL, incl, 31);
+            const uint32_t total = half + __shfl_sync(FULL, incl2, 31);
+            const uint32_t gexcl = incl - mine;           // group `lane`'s word offset in the chunk
+            const uint32_t gexcl2 = half + incl2 - mine2;  // group `lane + 32`'s
             bool to;
             const uint64_t base = chunk_lookback_warp(a.lb, chunk, total, lane, chunk != a.stall_chunk, to);
             if (to) {
@@ -466,13 +937,15 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
                 if (!fits && lane == 0 && a.status) atomicOr(a.status, kStatusCapacity);
                 if (fits) {
                     for (int g = 0; g < GPB; g++) {
-                        const uint32_t go = __shfl_sync(FULL, gexcl, g), gw = __shfl_sync(FULL, mine, g);
+                        const uint32_t go = g < 32 ? __shfl_sync(FULL, gexcl, g) : __shfl_sync(FULL, gexcl2, g - 32);
+                        const uint32_t gw = g < 32 ? __shfl_sync(FULL, mine, g) : __shfl_sync(FULL, mine2, g - 32);
                         const uint32_t *src = stage + (size_t)g * gstride;
                         uint32_t *dst = a.payload + base + go;
                         for (uint32_t i = lane; i < gw; i += 32) dst[i] = src[i];
                     }
                 }
                 if (lane < GPB) s_goff[lane] = gexcl;
+                if (lane + 32 < GPB) s_goff[lane + 32] = gexcl2;
                 __syncwarp();
                 const int64_t t0 = (int64_t)chunk * T;
                 for (int i = lane; i < T; i += 32) {
@@ -674,18 +1147,22 @@ namespace {
 // coordinates per lane: 8 for n = 64, 16 for 128 and 256, 32 above
 template <int N>
 constexpr int epl_for() { return N == 64 ? 8 : (N <= 256 ? 16 : 32); }
+// the variable-rate encoder: at least 16 per lane, so a run holds whole E8 vectors
+template <int N>
+constexpr int epl_var() { return N <= 256 ? 16 : 32; }
 
 template <int N>
-constexpr int groups_per_block() { return (kEncodeWarps - 1) * (32 / (N / epl_for<N>())); }
+constexpr int groups_per_block() { return (kEncodeWarps - 1) * (32 / (N / epl_var<N>())); }
 
 template <int N, int D, bool DITHER, bool F32IN>
 cudaError_t launch_encode_t(const EncodeArgs &a0, cudaStream_t s)
 {
-    constexpr int EPL = epl_for<N>(), GPB = groups_per_block<N>();
+    constexpr int EPL = epl_var<N>(), GPB = groups_per_block<N>();
     EncodeArgs a = a0;
     const int T = GPB * a.tiles_per_group;
     const size_t gstride = ((size_t)a.tiles_per_group * a.wmax + 3) & ~(size_t)3;
-    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + 2 * (size_t)GPB * gstride * 4 +
+    const size_t ywords = a.sign_words ? (size_t)a.tiles_per_row * (N / EPL) : 0;
+    const size_t smem = ((ywords + 3) & ~(size_t)3) * 4 + 2 * (size_t)GPB * gstride * 4 +
                         2 * ((size_t)T * 8 + (size_t)GPB * 4);
     auto kern = encode_kernel<N, D, EPL, DITHER, F32IN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -48,11 +48,13 @@ __device__ __forceinline__ uint32_t select_bit(uint32_t v, uint32_t r)
     return pos;
 }
 
-// Parse tile t into lattice point coordinates pt (binary32).  Returns true
-// if the tile is not canonical (pt is then zero and sb is 0).
+// Parse tile t into lane l's symbols u (zigzagged stripped coordinates, code
+// order) and coset bits cb (bit q: the lane's vector q).  Returns true if the
+// tile is not canonical (u, cb and sb are then zero).  small: every code's
+// unary part is shorter than 32 bits, so u < 2^20.
 template <int N, int D, int EPL, bool FIXED>
-__device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint32_t *wbuf,
-                                           unsigned mask, int l, float (&pt)[EPL], uint32_t &sb)
+__device__ __forceinline__ bool parse_symbols(const DecodeArgs &a, int64_t t, uint32_t *wbuf, unsigned mask, int l,
+                                              uint32_t (&u)[EPL], uint32_t &cb, uint32_t &sb, bool &small)
 {
     constexpr int LPT = N / EPL;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
@@ -116,7 +118,9 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     __syncwarp(mask);
 
 #pragma unroll
-    for (int r = 0; r < EPL; r++) pt[r] = 0.0f;
+    for (int r = 0; r < EPL; r++) u[r] = 0;
+    cb = 0;
+    small = true;
     if (bad) {
         sb = 0;
         return true;
@@ -134,7 +138,6 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
     }
 
     // ---- coset bits and low parts
-    uint32_t cb = 0;
     if constexpr (C > 0) cb = get_bits(wbuf, (uint32_t)l * VPL, VPL);
     uint32_t low[EPL];
     if (k == 0) {
@@ -182,6 +185,7 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
             rl = shl32(rl, z + 1);
         }
     } else {
+        small = false;
         uint32_t p = p0;
 #pragma unroll
         for (int r = 0; r < EPL; r++) {
@@ -201,12 +205,22 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
         }
     }
 
-    // ---- symbols -> lattice point
+#pragma unroll
+    for (int r = 0; r < EPL; r++) u[r] = (q[r] << k) | low[r];
+    return false;
+}
+
+// Lattice point coordinates (binary32) of lane's vectors from their symbols.
+template <int D, int EPL>
+__device__ __forceinline__ void points_from_symbols(const uint32_t (&u)[EPL], uint32_t cb, const A2Consts &a2,
+                                                    float (&pt)[EPL])
+{
+    constexpr int VPL = EPL / D;
 #pragma unroll
     for (int qv = 0; qv < VPL; qv++) {
         int z[D];
 #pragma unroll
-        for (int m = 0; m < D; m++) z[m] = unzigzag((q[qv * D + m] << k) | low[qv * D + m]);
+        for (int m = 0; m < D; m++) z[m] = unzigzag(u[qv * D + m]);
         if constexpr (D == 8 || D == 4) {
             int s = 0;
 #pragma unroll
@@ -216,13 +230,52 @@ __device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint3
         const float half = ((cb >> qv) & 1u) ? 0.5f : 0.0f;
         if constexpr (D == 2) {
             pt[qv * 2] = (float)z[0] + half;
-            pt[qv * 2 + 1] = __fmul_rn((float)z[1] + half, a.a2.s3);
+            pt[qv * 2 + 1] = __fmul_rn((float)z[1] + half, a2.s3);
         } else {
 #pragma unroll
             for (int m = 0; m < D; m++) pt[qv * D + m] = (float)z[m] + half;
         }
     }
-    return false;
+}
+
+// Doubled lattice coordinates t = 2y of lane's vectors from their symbols
+// (D = 1, 4, 8: integer points, E8's half-integer coset odd).  With z the
+// unzigzagged symbol, 2z = u ^ -(u & 1); a stripped last coordinate s =
+// floor(z / 2) is restored as 2z = 2 (2s) + 2 parity(sum of the others), that
+// parity being bit 1 of the XOR of the others' 2z.
+template <int D, int EPL>
+__device__ __forceinline__ void doubled_from_symbols(const uint32_t (&u)[EPL], uint32_t cb, int32_t (&t)[EPL])
+{
+    static_assert(D != 2, "A2 has no integer form");
+    constexpr int VPL = EPL / D;
+#pragma unroll
+    for (int qv = 0; qv < VPL; qv++) {
+        int32_t d2[D];
+#pragma unroll
+        for (int m = 0; m < D; m++) d2[m] = (int32_t)(u[qv * D + m] ^ (0u - (u[qv * D + m] & 1u)));
+        if constexpr (D == 8 || D == 4) {
+            int32_t x = 0;
+#pragma unroll
+            for (int m = 0; m < D - 1; m++) x ^= d2[m];
+            d2[D - 1] = 2 * d2[D - 1] + (x & 2);
+        }
+        const int32_t c = (D == 8) ? (int32_t)((cb >> qv) & 1u) : 0;
+#pragma unroll
+        for (int m = 0; m < D; m++) t[qv * D + m] = d2[m] + c;
+    }
+}
+
+// Parse tile t into lattice point coordinates pt (binary32).  Returns true
+// if the tile is not canonical (pt is then zero and sb is 0).
+template <int N, int D, int EPL, bool FIXED>
+__device__ __forceinline__ bool parse_tile(const DecodeArgs &a, int64_t t, uint32_t *wbuf, unsigned mask, int l,
+                                           float (&pt)[EPL], uint32_t &sb)
+{
+    uint32_t u[EPL], cb;
+    bool small;
+    const bool bad = parse_symbols<N, D, EPL, FIXED>(a, t, wbuf, mask, l, u, cb, sb, small);
+    points_from_symbols<D, EPL>(u, cb, a.a2, pt);
+    return bad;
 }
 
 template <int N, int EPL>
