@@ -56,15 +56,40 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane % LPT, gid = warp * TPW + lane / LPT;
     const unsigned mask = group_mask<LPT>(lane);
-    uint32_t *wbuf = sm + ((ywords + 3) & ~3) + gid * group_words(a.wmax);
+    // two staging buffers per group: the next tile's words arrive (cp.async)
+    // while this one is parsed
+    uint32_t *wb0 = sm + ((ywords + 3) & ~3) + gid * 2 * group_words(a.wmax);
+    uint32_t *wb1 = wb0 + group_words(a.wmax);
     for (int i = threadIdx.x; i < ywords; i += blockDim.x)
         ytab[i] = decode_sign_word<N, EPL>(a.sign_key, (uint64_t)(i / LPT), i % LPT);
     __syncthreads();
 
-    for (int64_t t = (int64_t)blockIdx.x * GPB + gid; t < a.ntiles; t += (int64_t)gridDim.x * GPB) {
+    const int64_t stride = (int64_t)gridDim.x * GPB;
+    int64_t t = (int64_t)blockIdx.x * GPB + gid;
+    TileHdr h{};
+    if (t < a.ntiles) {
+        h = tile_header<N, D, FIXED>(a, t);
+        stage_async<LPT>(a, h, wb0, l);
+    }
+    async_commit();
+    for (; t < a.ntiles; t += stride) {
+        const int64_t tn = t + stride;
+        TileHdr hn{};
+        if (tn < a.ntiles) {
+            hn = tile_header<N, D, FIXED>(a, tn);
+            stage_async<LPT>(a, hn, wb1, l);
+        }
+        async_commit();
+        async_wait<1>();   // this tile's words have arrived
+        __syncwarp(mask);  // ... for every lane of the group
         uint32_t u[EPL], cb, sb;
         bool small;
-        const bool bad = parse_symbols<N, D, EPL, FIXED>(a, t, wbuf, mask, l, u, cb, sb, small);
+        const bool bad = parse_staged<N, D, EPL, FIXED>(a, h, wb0, mask, l, u, cb, sb, small);
+        h = hn;
+        uint32_t *tmp = wb0;
+        wb0 = wb1;
+        wb1 = tmp;
+        __syncwarp(mask);  // the group is done with the words the next prefetch overwrites
         float2 v[NP];
         if constexpr (D != 2 && !DITHER) {
             // v = (Delta / n) y = (Delta / 2n) t with t = 2y an integer: t + 1.5 2^23
@@ -146,7 +171,8 @@ __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(con
     const int64_t tpr = a.tiles_per_row;
     unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(sm);
     float *xt = reinterpret_cast<float *>(sm + 2 * a.sign_words);
-    uint32_t *wbuf = sm + 2 * a.sign_words + tpr * N + gid * group_words(a.wmax);
+    uint32_t *wb0 = sm + 2 * a.sign_words + tpr * N + gid * 2 * group_words(a.wmax);
+    uint32_t *wb1 = wb0 + group_words(a.wmax);
     build_sign_table<N>(sign_tab, a.sign_words, a.sign_key);
     __syncthreads();
 
@@ -178,11 +204,33 @@ __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(con
 
     for (int64_t row = (int64_t)blockIdx.x * W + warp; row < a.rows; row += (int64_t)gridDim.x * W) {
         float acc = 0.0f;
-        for (int64_t j = lane / LPT; j < tpr; j += TPW) {
+        // the row's tiles j = group, group + TPW, ...: the next one's words
+        // arrive (cp.async) while this one is parsed
+        int64_t j = lane / LPT;
+        TileHdr h{};
+        if (j < tpr) {
+            h = tile_header<N, D, FIXED>(a, row * tpr + j);
+            stage_async<LPT>(a, h, wb0, l);
+        }
+        async_commit();
+        for (; j < tpr; j += TPW) {
             const int64_t t = row * tpr + j;
+            TileHdr hn{};
+            if (j + TPW < tpr) {
+                hn = tile_header<N, D, FIXED>(a, t + TPW);
+                stage_async<LPT>(a, hn, wb1, l);
+            }
+            async_commit();
+            async_wait<1>();
+            __syncwarp(mask);
             uint32_t u[EPL], cb, sb;
             bool small;
-            const bool bad = parse_symbols<N, D, EPL, FIXED>(a, t, wbuf, mask, l, u, cb, sb, small);
+            const bool bad = parse_staged<N, D, EPL, FIXED>(a, h, wb0, mask, l, u, cb, sb, small);
+            h = hn;
+            uint32_t *tmp = wb0;
+            wb0 = wb1;
+            wb1 = tmp;
+            __syncwarp(mask);
             const float4 *src = reinterpret_cast<const float4 *>(xt + j * N + l * EPL);
             float2 d2 = make_float2(0.0f, 0.0f);
             float step;  // the tile's weight on the dot: Delta / n for points, Delta / 2n for doubled points
@@ -262,7 +310,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
     constexpr int EPL = epl_dec<N>(), GPB = kDecodeWarps * (32 / (N / EPL));
     const size_t ywords = a.sign_words ? (size_t)a.tiles_per_row * (N / EPL) : 0;
-    const size_t smem = ((ywords + 3) & ~(size_t)3) * 4 + (size_t)GPB * group_words(a.wmax) * 4;
+    const size_t smem = ((ywords + 3) & ~(size_t)3) * 4 + (size_t)GPB * 2 * group_words(a.wmax) * 4;
     auto kern = a.slot ? decode_kernel<N, D, EPL, DITHER, F32OUT, true> : decode_kernel<N, D, EPL, DITHER, F32OUT, false>;
     unsigned blocks = 0;
     cudaError_t e = grid_for(kern, smem, (a.ntiles + GPB - 1) / GPB, blocks);
@@ -297,7 +345,7 @@ template <int N, int D, int W>
 cudaError_t launch_gemv_w(const DecodeArgs &a, int64_t cols, cudaStream_t s)
 {
     constexpr int EPL = epl_for<N>(), GPB = W * (32 / (N / EPL));
-    const size_t smem = (size_t)a.sign_words * 8 + (size_t)cols * 4 + (size_t)GPB * group_words(a.wmax) * 4;
+    const size_t smem = (size_t)a.sign_words * 8 + (size_t)cols * 4 + (size_t)GPB * 2 * group_words(a.wmax) * 4;
     auto kern = a.slot ? gemv_kernel<N, D, EPL, W, true> : gemv_kernel<N, D, EPL, W, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

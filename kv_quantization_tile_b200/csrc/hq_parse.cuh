@@ -48,45 +48,83 @@ __device__ __forceinline__ uint32_t select_bit(uint32_t v, uint32_t r)
     return pos;
 }
 
-// Parse tile t into lane l's symbols u (zigzagged stripped coordinates, code
-// order) and coset bits cb (bit q: the lane's vector q).  Returns true if the
-// tile is not canonical (u, cb and sb are then zero).  small: every code's
-// unary part is shorter than 32 bits, so u < 2^20.
+// A tile's header as the parser reads it: word offset, words (0 if the header
+// is not canonical), Rice parameter and scale bits.
+struct TileHdr {
+    uint32_t o0, W, sb;
+    int k;
+    bool bad;
+};
+
+// Load tile t's header and check it (offsets in order and inside the
+// capacity, k <= 15, Delta zero or a positive normal finite bf16, enough
+// words for the coset bits, the low parts and n terminators).
+template <int N, int D, bool FIXED>
+__device__ __forceinline__ TileHdr tile_header(const DecodeArgs &a, int64_t t)
+{
+    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
+    TileHdr h;
+    uint32_t o1;
+    if constexpr (FIXED) {
+        h.o0 = (uint32_t)t * a.slot;  // the host keeps ntiles * slot below 2^32
+        o1 = h.o0 + a.slot;
+        h.k = (a.kk[t >> 1] >> ((t & 1) * 4)) & 15;
+    } else {
+        h.o0 = a.off[t];
+        o1 = a.off[t + 1];
+        h.k = a.kk[t];
+    }
+    h.sb = a.scale[t];
+    const uint32_t ex = h.sb & 0x7f80u;
+    h.bad = (o1 < h.o0) || (o1 - h.o0 > a.wmax) || ((uint64_t)o1 > a.cap) || (h.k > 15) || (h.sb & 0x8000u) ||
+            ex == 0x7f80u || (h.sb != 0 && ex == 0);
+    const uint32_t U0 = (uint32_t)C + (uint32_t)N * (uint32_t)h.k;
+    const uint32_t W0 = h.bad ? 0u : o1 - h.o0;
+    if (!h.bad && U0 + (uint32_t)N > 32u * W0) h.bad = true;
+    h.W = h.bad ? 0u : W0;
+    return h;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Start copying the tile's words into the group's staging buffer (cp.async,
+// no registers held; each lane copies words l, l + LPT, ...) and write the
+// four zero guard words.  The caller commits the group and waits for it.
+template <int LPT>
+__device__ __forceinline__ void stage_async(const DecodeArgs &a, const TileHdr &h, uint32_t *wbuf, int l)
+{
+    for (uint32_t i = l; i < h.W; i += LPT)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(wbuf + i)), "l"(a.payload + h.o0 + i)
+                     : "memory");
+    if (l < 4) wbuf[h.W + l] = 0u;
+}
+
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Parse a staged tile (header h, words in wbuf) into lane l's symbols u
+// (zigzagged stripped coordinates, code order) and coset bits cb (bit q: the
+// lane's vector q).  Returns true if the tile is not canonical (u, cb and sb
+// are then zero).  small: every code's unary part is shorter than 32 bits, so
+// u < 2^20.
 template <int N, int D, int EPL, bool FIXED>
-__device__ __forceinline__ bool parse_symbols(const DecodeArgs &a, int64_t t, uint32_t *wbuf, unsigned mask, int l,
-                                              uint32_t (&u)[EPL], uint32_t &cb, uint32_t &sb, bool &small)
+__device__ __forceinline__ bool parse_staged(const DecodeArgs &a, const TileHdr &h, uint32_t *wbuf, unsigned mask,
+                                             int l, uint32_t (&u)[EPL], uint32_t &cb, uint32_t &sb, bool &small)
 {
     constexpr int LPT = N / EPL;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
     constexpr int VPL = EPL / D;
+    constexpr bool fixed = FIXED;
     uint32_t *starts = wbuf + a.wmax + 4;
-
-    constexpr bool fixed = FIXED;  // the stream kind is a launch-time choice (a.slot != 0)
-    uint32_t o0, o1;
-    int k;
-    if constexpr (fixed) {
-        o0 = (uint32_t)t * a.slot;  // the host keeps ntiles * slot below 2^32
-        o1 = o0 + a.slot;
-        k = (a.kk[t >> 1] >> ((t & 1) * 4)) & 15;
-    } else {
-        o0 = a.off[t];
-        o1 = a.off[t + 1];
-        k = a.kk[t];
-    }
-    sb = a.scale[t];
-    // Delta is 0 or a positive, normal, finite bf16 in any canonical tile
-    const uint32_t ex = sb & 0x7f80u;
-    bool bad = (o1 < o0) || (o1 - o0 > a.wmax) || ((uint64_t)o1 > a.cap) || (k > 15) ||
-               (sb & 0x8000u) || ex == 0x7f80u || (sb != 0 && ex == 0);
+    const int k = h.k;
+    bool bad = h.bad;
+    const uint32_t W = h.W;
+    sb = h.sb;
     const uint32_t U0 = (uint32_t)C + (uint32_t)N * (uint32_t)k;
-    const uint32_t W0 = bad ? 0u : o1 - o0;
-    if (!bad && U0 + (uint32_t)N > 32u * W0) bad = true;
-    const uint32_t W = bad ? 0u : W0;
-
-    __syncwarp(mask);  // the group is done with the previous tile's words
-    for (uint32_t i = l; i < W; i += LPT) wbuf[i] = __ldg(a.payload + o0 + i);
-    if (l < 4) wbuf[W + l] = 0u;
-    __syncwarp(mask);
 
     // ---- unary terminators: count per word, scanned across the group; the
     // word holding terminator m*EPL - 1 yields lane m's start
@@ -205,9 +243,24 @@ __device__ __forceinline__ bool parse_symbols(const DecodeArgs &a, int64_t t, ui
         }
     }
 
+    const uint32_t p2k = 1u << k;
 #pragma unroll
-    for (int r = 0; r < EPL; r++) u[r] = (q[r] << k) | low[r];
+    for (int r = 0; r < EPL; r++) u[r] = q[r] * p2k + low[r];  // (q << k) | low: the low part is below 2^k
     return false;
+}
+
+// Load, stage and parse tile t (parse_staged with synchronous staging).
+template <int N, int D, int EPL, bool FIXED>
+__device__ __forceinline__ bool parse_symbols(const DecodeArgs &a, int64_t t, uint32_t *wbuf, unsigned mask, int l,
+                                              uint32_t (&u)[EPL], uint32_t &cb, uint32_t &sb, bool &small)
+{
+    constexpr int LPT = N / EPL;
+    const TileHdr h = tile_header<N, D, FIXED>(a, t);
+    __syncwarp(mask);  // the group is done with the previous tile's words
+    for (uint32_t i = l; i < h.W; i += LPT) wbuf[i] = __ldg(a.payload + h.o0 + i);
+    if (l < 4) wbuf[h.W + l] = 0u;
+    __syncwarp(mask);
+    return parse_staged<N, D, EPL, FIXED>(a, h, wbuf, mask, l, u, cb, sb, small);
 }
 
 // Lattice point coordinates (binary32) of lane's vectors from their symbols.
