@@ -11,9 +11,13 @@ scaling, no collective on the data path).
 
 Also reported: per-kernel roofline of the dominant kernel (algorithmic bytes
 / CUDA-event time on the launching stream), the end-to-end figure through the
-C ABI from pinned host buffers, the batch-1 decode-GEMV and KV-cache paths,
-the CPU oracle timed on a bounded sample, and SM clocks sampled during the
-timed region.
+C ABI from pinned host buffers, every workload (the tiny fp32 matrix; the
+Llama layer at 3, 4 and 5 bps; the dithered KV layer with D4 and E8 at 2, 3
+and 4 bps; the whole 72-block DiT stack as one job plus D4/A2/Z passes over
+its FFN matrices) with the itemized rate and Rice gap of each stream, the
+batch-1 decode-GEMV, batched product, attention and fixed-rate paths, the
+CPU oracle timed on a bounded sample on all cores and on one thread, and SM
+clocks sampled during the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -45,7 +49,7 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
-    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "kv", "kv_attention", "fixed"],
+    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "configs", "dit", "kv_attention", "fixed"],
                    help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
     p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
     p.add_argument("--batch", type=int, default=None, help="one batch size for --leg gemm")
@@ -137,57 +141,89 @@ class Clocks:
 
 
 # ------------------------------------------------------------------ oracle leg
-def cpu_baseline(seconds: float):
-    """The CPU oracle (as it stands) on a bounded sample of the gate matrix:
-    encode + decode of whole rows until `seconds` of wall time have passed,
-    one thread per core over disjoint row blocks."""
+def _oracle_sample():
+    """The gate matrix of the Llama layer as uint16 bf16 bits, and the built oracle."""
     import numpy as np
     import torch
 
     import oracle
     from kv_quantization_tile_b200 import workloads
 
-    cores = len(os.sched_getaffinity(0))
     gate = workloads.outlier_weight(14336, 4096, 1004, 1104, "cpu")
-    bits = gate.view(torch.int16).numpy().view(np.uint16)
     oracle.build()
-    rows_per_block = 8
-    done_rows, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < seconds and done_rows < bits.shape[0]:
-        blk = bits[done_rows: done_rows + rows_per_block * cores]
-        s = oracle.encode(blk, TILE, LAT, BPS, SEED, threads=cores)
-        oracle.decode(s, blk.shape[0], blk.shape[1], TILE, LAT, SEED, threads=cores)
-        done_rows += blk.shape[0]
-    el = time.perf_counter() - t0
-    elems = done_rows * bits.shape[1]
-    return {"value": round(4 * elems / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"encode+decode of the first {done_rows} rows x 4096 of the gate matrix "
-                      f"({elems} weights, E8 4 bps, tile 256) in {el:.1f} s on {cores} threads"}
+    return oracle, gate.view(torch.int16).numpy().view(np.uint16)
+
+
+def _oracle_rows(oracle, bits, r0: int, rows: int, threads: int) -> None:
+    blk = bits[r0: r0 + rows]
+    s = oracle.encode(blk, TILE, LAT, BPS, SEED, threads=threads)
+    oracle.decode(s, blk.shape[0], blk.shape[1], TILE, LAT, SEED, threads=threads)
+
+
+def _oracle_timed(oracle, bits, seconds: float, threads: int):
+    """Encode + decode of whole rows of the gate matrix, blocks of 8 rows per
+    thread, until `seconds` of wall time have passed: (rows, seconds)."""
+    done, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds and done < bits.shape[0]:
+        n = min(8 * threads, bits.shape[0] - done)
+        _oracle_rows(oracle, bits, done, n, threads)
+        done += n
+    return done, time.perf_counter() - t0
+
+
+def cpu_baseline(seconds: float):
+    """The CPU oracle (as it stands) on a bounded sample of the gate matrix,
+    timed on all host cores (one thread per core over disjoint row blocks)
+    and on one thread."""
+    oracle, bits = _oracle_sample()
+    cores = len(os.sched_getaffinity(0))
+    rows, el = _oracle_timed(oracle, bits, seconds, cores)
+    rows1, el1 = _oracle_timed(oracle, bits, max(1.0, seconds / 3), 1)
+    cols = bits.shape[1]
+    return {"value": round(4 * rows * cols / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"encode+decode of the first {rows} rows x {cols} of the gate matrix "
+                      f"({rows * cols} weights, E8 4 bps, tile 256) in {el:.1f} s on {cores} threads",
+            "single_thread": {"value": round(4 * rows1 * cols / el1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                              "sample": f"first {rows1} rows x {cols} of the gate matrix in {el1:.1f} s"}}
 
 
 def run_reference(args):
+    """The oracle as the reference arm: every step encodes and decodes the same
+    bounded sample of the Llama layer's gate matrix (a fixed number of whole
+    rows, sized so that warm-up plus timed steps take about a minute), on all
+    host cores; ms_per_step is the measured wall time of a step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per = max(2.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    oracle, bits = _oracle_sample()
+    cores = len(os.sched_getaffinity(0))
+    cols = bits.shape[1]
+    # calibrate the rows a step can take in its share of the minute
+    rows_c, el_c = _oracle_timed(oracle, bits, 1.0, cores)
+    per = max(0.25, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
+    rows = max(cores, min(bits.shape[0], int(rows_c / el_c * per) // cores * cores))
     for _ in range(args.warmup):
-        cpu_baseline(per / 4)
-    vals = [cpu_baseline(per) for _ in range(args.steps)]
-    v = statistics.median(x["value"] for x in vals)
-    cb = dict(vals[-1])
-    cb["value"] = v
+        _oracle_rows(oracle, bits, 0, rows, cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_rows(oracle, bits, 0, rows, cores)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    v = round(4 * rows * cols / (ms * 1e-3) / 1e9, 4)
+    sample = (f"each step: encode+decode of the first {rows} rows x {cols} of the gate matrix "
+              f"({rows * cols} weights, E8 4 bps, tile 256) on {cores} threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(4 * LAYER_ELEMENTS / (v * 1e9) * 1e3, 1),  # extrapolated from the sample
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": layer_config(1),
-        "cpu_baseline": cb, "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
-                                    "d2h_bytes_per_step": 0}}))
+        "config": dict(layer_config(1), sample=sample, elements_per_step=rows * cols),
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
 # ------------------------------------------------------------------ GPU leg
-KERNEL_HEADERS = ("hq_device.cuh", "hq_parse.cuh", "hq_internal.h")
+KERNEL_HEADERS = ("hq_device.cuh", "hq_fast.cuh", "hq_parse.cuh", "hq_internal.h")
 
 
 def kernel_source_sha(kernel_file: str) -> str:
@@ -332,7 +368,10 @@ def run_ours(args):
     if not args.no_extras:
         out["e2e"] = e2e_leg(args, ctx, dev, stream, status, n_elem, world, max_over_ranks, barrier)
         if rank == 0:
-            out["paths"] = {"gemv": gemv_leg(dev, peak), "gemm": gemm_leg(dev, peak), "kv": kv_leg(dev, peak),
+            out["configs"] = configs_leg(dev, peak, [m["x"] for m in ctx])
+            del ctx
+            out["configs"]["dit_stack"] = dit_leg(dev, peak)
+            out["paths"] = {"gemv": gemv_leg(dev, peak), "gemm": gemm_leg(dev, peak),
                             "kv_attention": attention_leg(dev, peak), "fixed_rate": fixed_leg(dev, peak)}
             out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
@@ -423,6 +462,110 @@ def time_launches(fn, flush, reps=20):
     return statistics.median(ts)
 
 
+def codec_pass(mats, tile, lat, bps, dev, peak, kv=False, reps=5, flush=None, seed=SEED, stats=True):
+    """One job over `mats`: encode every matrix, then decode every matrix back
+    to its own dtype (into one scratch output per shape), timed as two CUDA-event
+    intervals on the current stream; median over `reps` jobs after one warm-up.
+    Reports time, bytes, GB/s (algorithmic: input + stream bytes) and, when
+    `stats`, the itemized rate of the streams (rate accounting kernel)."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq
+
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws, out, streams = {}, {}, []
+    for x in mats:
+        r, c = x.shape
+        if (r, c) not in ws:
+            ws[(r, c)] = hq.alloc_workspace(r, c, tile, dev)
+        if (r, c, x.dtype) not in out:
+            out[(r, c, x.dtype)] = torch.empty_like(x)
+        streams.append(hq.alloc_stream(r, c, tile, lat, bps, dev))
+    enc_fn = hq.hq_kv_encode if kv else hq.hq_encode
+    dec_fn = hq.hq_kv_decode if kv else hq.hq_decode
+
+    def enc():
+        for x, s in zip(mats, streams):
+            enc_fn(x, tile, lat, bps, seed, s, ws[tuple(x.shape)], st)
+
+    def dec():
+        for x, s in zip(mats, streams):
+            r, c = x.shape
+            dec_fn(s, r, c, tile, lat, bps, seed, out[(r, c, x.dtype)], st)
+
+    enc(); dec()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
+    flush = flush or (lambda: None)
+    te = time_launches(enc, flush, reps=reps)
+    td = time_launches(dec, flush, reps=reps)
+    n = sum(x.numel() for x in mats)
+    nin = sum(x.numel() * x.element_size() for x in mats)
+    cb = sum(s.nbytes() for s in streams)
+    alg = nin + cb
+    res = {"matrices": len(mats), "weights": n, "input_bytes": nin, "stream_bytes": cb,
+           "bits_per_weight_total": round(8 * cb / n, 4),
+           "encode_ms": round(te, 4), "decode_ms": round(td, 4),
+           "encode_alg_gbs": round(alg / te / 1e6, 1), "decode_alg_gbs": round(alg / td / 1e6, 1),
+           "encode_frac": round(alg / te / 1e6 / peak, 4), "decode_frac": round(alg / td / 1e6 / peak, 4),
+           "job_gbs": round(2 * nin / (te + td) / 1e6, 1)}
+    if stats:
+        tot_c = tot_h = None
+        for x, s in zip(mats, streams):
+            c, h = hq.hq_stream_stats(s, x.shape[0], x.shape[1], tile, lat, bps, status=st)
+            tot_c = c if tot_c is None else tot_c + c
+            tot_h = h if tot_h is None else tot_h + h
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        res["rate"] = hq.rate_report(tot_c.cpu().tolist(), tot_h.cpu().tolist(), tile)
+    del streams, ws, out
+    return res
+
+
+def configs_leg(dev, peak, llama_mats):
+    """Every workload: the tiny fp32 matrix, the Llama layer at 3, 4 and 5 bps,
+    the KV layer (dithered, tile 128) for D4 and E8 at 2, 3 and 4 bps, each with
+    its itemized rate and Rice gap."""
+    import torch
+
+    from kv_quantization_tile_b200 import workloads
+
+    flushbuf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    res = {"tiny_fp32": dict(codec_pass([workloads.tiny(dev)], TILE, LAT, BPS, dev, peak, reps=20,
+                                        flush=lambda: flush_l2(flushbuf)),
+                             note="256 x 1024 fp32 (1 MB) E8 4 bps tile 256; L2 flushed before each timed job")}
+    res["llama_layer"] = {f"E8_{b:g}bps": codec_pass(llama_mats, TILE, LAT, float(b), dev, peak)
+                          for b in (3, 4, 5)}
+    k, v = workloads.kv_layer(dev)
+    res["kv_layer"] = {f"{lat}_{b:g}bps": codec_pass([k, v], 128, lat, float(b), dev, peak, kv=True, reps=10)
+                       for lat in ("E8", "D4") for b in (2, 3, 4)}
+    del k, v, flushbuf
+    return res
+
+
+def dit_leg(dev, peak, reps=3):
+    """The 72-block video-DiT weight stack (720 bf16 matrices, 19.3 G weights,
+    38.6 GB), all resident in HBM; one job = encode all 720 matrices at E8 4 bps
+    tile 256, then decode all 720 (median of `reps` jobs).  Then the 144 FFN
+    matrices alone with D4, A2 and Z at 4 bps."""
+    import torch
+
+    from kv_quantization_tile_b200 import workloads
+
+    mats, ffn = [], []
+    for b in range(workloads.DIT_BLOCKS):
+        for name, x in workloads.dit_block(b, dev):
+            mats.append(x)
+            if name.startswith("ffn"):
+                ffn.append(x)
+    res = {"blocks": workloads.DIT_BLOCKS, "E8_4bps": codec_pass(mats, TILE, "E8", BPS, dev, peak, reps=reps)}
+    for lat in ("D4", "A2", "Z"):
+        res[f"ffn_{lat}_4bps"] = codec_pass(ffn, TILE, lat, BPS, dev, peak, reps=reps)
+    del mats, ffn
+    torch.cuda.empty_cache()
+    return res
+
+
 def gemv_leg(dev, peak):
     """Batch-1 decode-GEMV on 14336x4096 and 4096x14336 E8 4-bps streams vs the
     bf16 GEMV (cuBLAS) on the uncompressed matrices; L2 flushed before each."""
@@ -453,47 +596,6 @@ def gemv_leg(dev, peak):
                      "compressed_bytes": s.nbytes(), "bf16_gemv_us": round(ms_bf16 * 1e3, 2),
                      "speedup_vs_bf16": round(ms_bf16 / ms, 3)}
         del s, ws
-    return res
-
-
-def kv_leg(dev, peak):
-    """KV cache, one layer: K and V (8 x 32768 x 128 bf16) encoded and decoded
-    with subtractive dither, tile 128, E8 and D4 at 4 bps."""
-    import torch
-
-    from kv_quantization_tile_b200 import hq, workloads
-
-    k, v = workloads.kv_layer(dev)
-    res = {}
-    for lat in ("E8", "D4"):
-        ctx = []
-        for x in (k, v):
-            r, c = x.shape
-            ctx.append((x, hq.alloc_stream(r, c, 128, lat, 4.0, dev), hq.alloc_workspace(r, c, 128, dev),
-                        torch.empty_like(x)))
-        st = torch.zeros(1, dtype=torch.int32, device=dev)
-
-        def enc():
-            for x, s, ws, _ in ctx:
-                hq.hq_kv_encode(x, 128, lat, 4.0, SEED, s, ws, st)
-
-        def dec():
-            for x, s, _, y in ctx:
-                hq.hq_kv_decode(s, x.shape[0], 128, 128, lat, 4.0, SEED, y, st)
-
-        for _ in range(3):
-            enc(); dec()
-        torch.cuda.synchronize()
-        assert int(st.item()) == 0
-        n = 2 * k.numel()
-        cb = sum(s.nbytes() for _, s, _, _ in ctx)
-        te = time_launches(enc, lambda: None, reps=10)
-        td = time_launches(dec, lambda: None, reps=10)
-        res[f"{lat}_4bps"] = {"encode_alg_gbs": round((2 * n + cb) / te / 1e6, 1),
-                              "decode_alg_gbs": round((2 * n + cb) / td / 1e6, 1),
-                              "encode_frac": round((2 * n + cb) / te / 1e6 / peak, 4),
-                              "decode_frac": round((2 * n + cb) / td / 1e6 / peak, 4),
-                              "bits_per_value_total": round(8 * cb / n, 4)}
     return res
 
 
@@ -736,8 +838,11 @@ def run_leg(args):
         res = gemv_leg("cuda", peak)
     elif args.leg == "gemm":
         res = gemm_leg("cuda", peak, batches=(args.batch,) if args.batch else (1, 16, 64, 256))
-    elif args.leg == "kv":
-        res = kv_leg("cuda", peak)
+    elif args.leg == "configs":
+        from kv_quantization_tile_b200 import workloads
+        res = configs_leg("cuda", peak, [m for _, m in workloads.llama_layer("cuda")])
+    elif args.leg == "dit":
+        res = dit_leg("cuda", peak)
     elif args.leg == "fixed":
         res = fixed_leg("cuda", peak)
     else:

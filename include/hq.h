@@ -233,6 +233,24 @@ int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int
                    float bps, uint64_t seed, const void *x, float *y, void *stream,
                    int32_t *d_status);
 
+/* Rate accounting of a stream ([V2] abstract: itemized rate accounting;
+ * the Rice code's distance from the lattice's rate-distortion ideal).  The
+ * stream is read, not changed; any stream kind (variable or fixed rate).
+ * counts: device uint64[8], cleared by the call, then: canonical tiles, coset
+ * bits, low-part bits (n k per tile), unary bits (sum(u >> k) + n), padding
+ * bits (the tile's words minus those), offset-header bits (32 per tile; 0 in
+ * a fixed-rate stream), scale-header bits (16), Rice-parameter bits (8; 4
+ * packed in a fixed-rate stream).  hist: device uint64[2][bins] (2 <= bins
+ * <= 4096), cleared by the call: counts of symbol values 0 .. bins - 2 and of
+ * values >= bins - 1 in the last bin; row 1 holds the stripped last
+ * coordinates of D4 / E8 vectors, row 0 every other symbol.  Both pointers
+ * 8-byte aligned, caller-owned.  Asynchronous on `stream`; tiles that are not
+ * canonical are skipped and raise HQ_ST_CORRUPT.  HQ_ERR_ARG for bad
+ * pointers or bins, the decode calls' shape errors otherwise. */
+int hq_stream_stats(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice,
+                    float bps, uint64_t *counts, uint64_t *hist, int bins, void *stream,
+                    int32_t *d_status);
+
 /* Bytes of device workspace hq_decode_gemm needs for this shape: the
  * rotated activations (bf16, batch rounded up to the block's batch rows x
  * cols), then, when column tiles are split across blocks, fp32 partial

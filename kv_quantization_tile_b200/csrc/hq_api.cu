@@ -409,6 +409,23 @@ int hq_kv_decode(const hq_stream *in, int64_t rows, int64_t cols, int tile, int 
     return decode_impl(in, rows, cols, tile, lattice, bps, seed, y, dtype, stream, d_status, true);
 }
 
+int hq_stream_stats(const hq_stream *in, int64_t rows, int64_t cols, int tile, int lattice, float bps,
+                    uint64_t *counts, uint64_t *hist, int bins, void *stream, int32_t *d_status)
+{
+    DecodeArgs a{};
+    int64_t ntiles = 0;
+    int rc = decode_common(in, rows, cols, tile, lattice, bps, 0, a, &ntiles);
+    if (rc) return rc;
+    if (!counts || !hist || bins < 2 || bins > 4096 || !aligned(counts, 8) || !aligned(hist, 8)) return HQ_ERR_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(counts, 0, 8 * sizeof(uint64_t), s) != cudaSuccess ||
+        cudaMemsetAsync(hist, 0, 2 * (size_t)bins * sizeof(uint64_t), s) != cudaSuccess)
+        return HQ_ERR_CUDA;
+    if (ntiles == 0) return HQ_OK;
+    a.status = d_status;
+    return launch_stats(tile, lattice, a, counts, hist, bins, s) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
 int hq_decode_gemv(const hq_stream *w, int64_t rows, int64_t cols, int tile, int lattice, float bps,
                    uint64_t seed, const void *x, float *y, void *stream, int32_t *d_status)
 {

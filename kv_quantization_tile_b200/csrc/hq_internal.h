@@ -130,6 +130,9 @@ void gemm_plan_i8(int64_t rows, int64_t cols, int64_t batch, int blocks_per_sm, 
 cudaError_t launch_gemm_i8(int lattice, const GemmArgs &a, cudaStream_t s);
 // The fp8 variant: A = e4m3(2y), activations in E4M3 scaled to +-448 (same workspace).
 cudaError_t launch_gemm_e4m3(int lattice, const GemmArgs &a, cudaStream_t s);
+// Rate accounting of a stream: counts[8] and hist[2][bins] (device, added to).
+cudaError_t launch_stats(int tile, int lattice, const DecodeArgs &a, uint64_t *counts, uint64_t *hist, int bins,
+                         cudaStream_t s);
 // Fills a.splits / a.tokens_per_split from the kernel's occupancy, then launches.
 cudaError_t launch_attention(int head_dim, int lattice, AttnArgs a, cudaStream_t s);
 

@@ -9,6 +9,7 @@ raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 
@@ -32,7 +33,8 @@ EXPORTS = ["hq_error_string", "hq_version", "hq_rate_constant", "hq_tile_bound_w
            "hq_kv_attention_workspace_bytes", "hq_kv_attention", "hq_decode_gemm_workspace_bytes",
            "hq_decode_gemm", "hq_file_bytes", "hq_file_write", "hq_file_read", "hq_test_gemm_stalled",
            "hq_min_slot_words", "hq_fixed_slot_words", "hq_encode_fixed", "hq_kv_encode_fixed",
-           "hq_decode_gemm_int8_workspace_bytes", "hq_decode_gemm_int8", "hq_decode_gemm_fp8"]
+           "hq_decode_gemm_int8_workspace_bytes", "hq_decode_gemm_int8", "hq_decode_gemm_fp8",
+           "hq_stream_stats"]
 
 
 class hq_file_info(ctypes.Structure):
@@ -67,6 +69,8 @@ _SIGS = {
                             _vp, _vp]),
     "hq_decode_gemv": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _u64, _vp, _vp,
                               _vp, _vp]),
+    "hq_stream_stats": (_i32, [ctypes.POINTER(hq_stream), _i64, _i64, _i32, _i32, _f32, _vp, _vp, _i32,
+                               _vp, _vp]),
     "hq_encode_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
                                  _vp, _vp]),
     "hq_test_encode_stalled": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _f32, _u64, ctypes.POINTER(hq_stream),
@@ -306,6 +310,50 @@ def hq_decode_gemv(s: Stream, rows, cols, tile, lattice, bps, seed, x, y, status
     _check(_lib.hq_decode_gemv(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, seed, _ptr(x), _ptr(y),
                                _stream_handle(stream), _ptr(status)), "hq_decode_gemv")
     return y
+
+
+STATS_KEYS = ("tiles", "coset", "low", "unary", "padding", "offset_header", "scale_header", "k_header")
+
+
+def hq_stream_stats(s: Stream, rows, cols, tile, lattice, bps, bins=1024, status=None, stream=None):
+    """Bits by kind and the symbol histogram of a stream (device tensors:
+    counts int64[8] in STATS_KEYS order, hist int64[2][bins])."""
+    dev = s.payload.device
+    counts = torch.empty(8, dtype=torch.int64, device=dev)
+    hist = torch.empty(2, bins, dtype=torch.int64, device=dev)
+    st = s.struct()
+    _check(_lib.hq_stream_stats(ctypes.byref(st), rows, cols, tile, _lat(lattice), bps, _ptr(counts), _ptr(hist),
+                                bins, _stream_handle(stream), _ptr(status)), "hq_stream_stats")
+    return counts, hist
+
+
+def _entropy_bits(counts) -> float:
+    total = sum(counts)
+    return -sum(c / total * math.log2(c / total) for c in counts if c) if total else 0.0
+
+
+def rate_report(counts, hist, tile: int) -> dict:
+    """Itemized rate of a stream from hq_stream_stats (host lists or tensors):
+    bits per coordinate by kind, the empirical entropy of the symbols per
+    coordinate (stripped last coordinates counted apart), and the Rice code's
+    excess over it (low-part + unary bits minus that entropy)."""
+    c = [int(v) for v in counts]
+    h = [[int(v) for v in row] for row in hist]
+    coords = c[0] * tile
+    if coords == 0:
+        return {"coords": 0}
+    n0, n1 = sum(h[0]), sum(h[1])
+    sym_entropy = (_entropy_bits(h[0]) * n0 + _entropy_bits(h[1]) * n1) / coords
+    per = {k: c[i] / coords for i, k in enumerate(STATS_KEYS) if i > 0}
+    rice = per["low"] + per["unary"]
+    return {"coords": coords,
+            "bits_per_coord": {k: round(v, 4) for k, v in per.items()},
+            "payload_bits_per_coord": round(per["coset"] + rice + per["padding"], 4),
+            "total_bits_per_coord": round(sum(per.values()), 4),
+            "rice_bits_per_coord": round(rice, 4),
+            "symbol_entropy_bits_per_coord": round(sym_entropy, 4),
+            "rice_gap_bits_per_coord": round(rice - sym_entropy, 4),
+            "symbols_clipped_to_last_bin": h[0][-1] + h[1][-1]}
 
 
 def hq_decode_gemm_workspace_bytes(rows: int, cols: int, batch: int) -> int:
