@@ -97,15 +97,14 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
             // 9 significant bits) in one fma -- the single rounding of t Delta / 2n.
             // Exact while |t| < 2^22, which a lane whose codes all have unary
             // parts under 32 bits guarantees (u < 2^20); otherwise convert.
-            int32_t tt[EPL];
-            doubled_from_symbols<D, EPL>(u, cb, tt);
+            int32_t tt[EPL];  // t + 1.5 2^23 (bit patterns) where small, else t
+            doubled_from_symbols<D, EPL>(u, cb, tt, small ? kMagicBias : 0);
             const float s2 = bf16_bits_to_float(sb) * (0.5f / N);  // exact: a power-of-two step
             if (small) {
                 const float2 sc = splat2(s2), off = splat2(-12582912.0f * s2);
 #pragma unroll
                 for (int m = 0; m < NP; m++)
-                    v[m] = fma2(make_float2(__int_as_float(tt[2 * m] + kMagicBias), __int_as_float(tt[2 * m + 1] + kMagicBias)),
-                                sc, off);
+                    v[m] = fma2(make_float2(__int_as_float(tt[2 * m]), __int_as_float(tt[2 * m + 1])), sc, off);
             } else {
 #pragma unroll
                 for (int m = 0; m < NP; m++) v[m] = make_float2((float)tt[2 * m] * s2, (float)tt[2 * m + 1] * s2);
@@ -237,16 +236,16 @@ __global__ void __launch_bounds__(W * 32, N <= 256 ? 32 / W : 1) gemv_kernel(con
             if constexpr (D != 2) {
                 // t = 2y: t + 1.5 2^23 read as a float minus 1.5 2^23 is exact while
                 // |t| < 2^22 (every unary part under 32 bits); otherwise convert
-                int32_t tt[EPL];
-                doubled_from_symbols<D, EPL>(u, cb, tt);
+                int32_t tt[EPL];  // t + 1.5 2^23 (bit patterns) where small, else t
+                doubled_from_symbols<D, EPL>(u, cb, tt, small ? kMagicBias : 0);
                 const float2 moff = splat2(-12582912.0f);
 #pragma unroll
                 for (int c = 0; c < EPL / 4; c++) {
                     const float4 xv = src[c ^ (l & SW)];
                     float2 p0, p1;
                     if (small) {
-                        p0 = add2(make_float2(__int_as_float(tt[4 * c] + kMagicBias), __int_as_float(tt[4 * c + 1] + kMagicBias)), moff);
-                        p1 = add2(make_float2(__int_as_float(tt[4 * c + 2] + kMagicBias), __int_as_float(tt[4 * c + 3] + kMagicBias)), moff);
+                        p0 = add2(make_float2(__int_as_float(tt[4 * c]), __int_as_float(tt[4 * c + 1])), moff);
+                        p1 = add2(make_float2(__int_as_float(tt[4 * c + 2]), __int_as_float(tt[4 * c + 3])), moff);
                     } else {
                         p0 = make_float2((float)tt[4 * c], (float)tt[4 * c + 1]);
                         p1 = make_float2((float)tt[4 * c + 2], (float)tt[4 * c + 3]);

@@ -56,6 +56,27 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b)
 }
 __device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
 
+// three-input max / min (one instruction each on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// 1.0f if a == b, else 0.0f
+__device__ __forceinline__ float eq1f(float a, float b)
+{
+    float d;
+    asm("set.eq.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
 // ------------------------------------------------------------- transform
 // Forward transform of one tile held as EPL / 2 pairs per lane (see above).
 // l is the lane's index in its group, mask the group's lanes.
@@ -266,13 +287,11 @@ __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4], 
     }
     const float ae[8] = { fabsf(E[0].x), fabsf(E[0].y), fabsf(E[1].x), fabsf(E[1].y),
                           fabsf(E[2].x), fabsf(E[2].y), fabsf(E[3].x), fabsf(E[3].y) };
-    float s = ae[0], mx = ae[0], mn = ae[0];
+    float s = ae[0];
 #pragma unroll
-    for (int i = 1; i < 8; i++) {
-        s = __fadd_rn(s, ae[i]);
-        mx = fmaxf(mx, ae[i]);
-        mn = fminf(mn, ae[i]);
-    }
+    for (int i = 1; i < 8; i++) s = __fadd_rn(s, ae[i]);  // in index order: the rounding is part of the rule
+    const float mx = max3f(max3f(ae[0], ae[1], ae[2]), max3f(ae[3], ae[4], ae[5]), fmaxf(ae[6], ae[7]));
+    const float mn = min3f(min3f(ae[0], ae[1], ae[2]), min3f(ae[3], ae[4], ae[5]), fminf(ae[6], ae[7]));
     const int32_t px = __float_as_int(R[0].x) ^ __float_as_int(R[0].y) ^ __float_as_int(R[1].x) ^
                        __float_as_int(R[1].y) ^ __float_as_int(R[2].x) ^ __float_as_int(R[2].y) ^
                        __float_as_int(R[3].x) ^ __float_as_int(R[3].y);
@@ -287,17 +306,19 @@ __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4], 
     const bool fix = one ? odd1 : odd0;
     const float T = fix ? (one ? mn : mx) : -1.0f;
     const float sc = one ? -1.0f : 1.0f;
-    float h[8];
+    // H: 1 at the coordinates whose |e| is T, else 0; more than one hit is a tie
+    float2 H[4];
 #pragma unroll
-    for (int i = 0; i < 8; i++) h[i] = ae[i] == T ? sc : 0.0f;
-    // all hits carry the same sign, so |sum| counts them
-    tie = fabsf(((h[0] + h[1]) + (h[2] + h[3])) + ((h[4] + h[5]) + (h[6] + h[7]))) > 1.5f;
-    const float2 mq0 = splat2(one ? 0.0f : -1.0f), two = splat2(2.0f), unit = splat2(1.0f), half = splat2(0.5f);
+    for (int i = 0; i < 4; i++) H[i] = make_float2(eq1f(ae[2 * i], T), eq1f(ae[2 * i + 1], T));
+    const float2 hs = add2(add2(H[0], H[1]), add2(H[2], H[3]));
+    tie = __fadd_rn(hs.x, hs.y) > 1.5f;
+    const float2 mq0 = splat2(one ? 0.0f : -1.0f), two = splat2(2.0f), half = splat2(0.5f);
+    const float2 sc2 = splat2(2.0f * sc), sc1 = splat2(sc);
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const float2 C = sub2(F[i], R[i]);
         const float2 base = fma2(C, mq0, F[i]);
-        const float2 zb = fma2(make_float2(h[2 * i], h[2 * i + 1]), fma2(C, two, unit), base);
+        const float2 zb = fma2(H[i], fma2(C, sc2, sc1), base);  // h (1 + 2C), h = sc at a hit
         const float2 z = sub2(zb, M2);
         if (i < 3) {
             const float2 t = fma2(z, two, half);

@@ -4,10 +4,11 @@
 // A group of LPT lanes parses one tile; lane l owns codes l*EPL .. l*EPL+EPL-1.
 //   * The tile's words are staged in shared memory (plus zero guard words).
 //   * Coset bits and the fixed-width low parts are read at computed offsets.
-//   * Unary parts: one pass popcounts the unary words (a lane per word) and
-//     scans the counts across the group; the lane holding the word in which
-//     terminator m*EPL - 1 lies writes lane m's start bit (the bit after that
-//     terminator), so no lane searches.  Each lane then parses its EPL codes
+//   * Unary parts: one pass popcounts the unary words (two per lane) and
+//     scans the counts across the group; lane m finds the word holding
+//     terminator m*EPL - 1 by a binary search over the scanned counts and
+//     selects the bit (its start is the bit after that terminator), all
+//     lanes in step.  Each lane then parses its EPL codes
 //     from a bit-reversed 64-bit window with one count-leading-zeros and two
 //     funnel shifts per code, once it has checked that no zero run of its
 //     span reaches 32 bits; otherwise (and for spans over 64 bits) it parses
@@ -26,9 +27,8 @@
 
 namespace hq {
 
-// words of shared memory per group: staged tile words + 4 guard words, then
-// the start bit of each lane (up to 32 lanes)
-__host__ __device__ constexpr uint32_t group_words(uint32_t wmax) { return wmax + 4 + 32; }
+// words of shared memory per group: staged tile words + 4 guard words
+__host__ __device__ constexpr uint32_t group_words(uint32_t wmax) { return wmax + 4; }
 
 // position of the r-th (0-based) set bit of v (v has more than r set bits):
 // a branch-free binary search on popcounts of halves
@@ -119,41 +119,57 @@ __device__ __forceinline__ bool parse_staged(const DecodeArgs &a, const TileHdr 
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
     constexpr int VPL = EPL / D;
     constexpr bool fixed = FIXED;
-    uint32_t *starts = wbuf + a.wmax + 4;
     const int k = h.k;
     bool bad = h.bad;
     const uint32_t W = h.W;
     sb = h.sb;
     const uint32_t U0 = (uint32_t)C + (uint32_t)N * (uint32_t)k;
 
-    // ---- unary terminators: count per word, scanned across the group; the
-    // word holding terminator m*EPL - 1 yields lane m's start
+    // ---- unary terminators: lane l counts the ones of unary words 2l, 2l + 1
+    // of each pass of 2 LPT words, the counts are scanned across the group,
+    // and lane m (m >= 1) finds the word pair holding terminator m EPL - 1
+    // by a binary search over the scanned counts (shuffles, no divergence),
+    // then the bit by a select: its start is the bit after that terminator.
     const uint32_t wu0 = U0 >> 5;
     const uint32_t nwu = W > wu0 ? W - wu0 : 0;  // unary words (the first shared with the low parts)
     uint32_t found = 0, last_nz = 0;  // last_nz: 1 + the last unary word holding a one bit
-    for (uint32_t wb = 0; wb < nwu; wb += LPT) {
-        const uint32_t wi = wb + l;
-        uint32_t v = wi < nwu ? wbuf[wu0 + wi] : 0u;
-        if (wi == 0) v &= 0xffffffffu << (U0 & 31);
-        const uint32_t c = __popc(v);
+    uint32_t start = 0;
+    const uint32_t target = (uint32_t)l * EPL - 1u;  // lane l's terminator (l >= 1)
+    for (uint32_t wb = 0; wb < nwu; wb += 2 * LPT) {
+        const uint32_t wi = wb + 2 * (uint32_t)l;
+        uint32_t v0 = wi < nwu ? wbuf[wu0 + wi] : 0u;
+        const uint32_t v1 = wi + 1 < nwu ? wbuf[wu0 + wi + 1] : 0u;
+        if (wi == 0) v0 &= 0xffffffffu << (U0 & 31);
+        const uint32_t c0 = __popc(v0), c = c0 + __popc(v1);
         uint32_t incl = c;
 #pragma unroll
         for (int d = 1; d < LPT; d <<= 1) {
             const uint32_t o = __shfl_up_sync(mask, incl, d, LPT);
             if (l >= d) incl += o;
         }
-        if (wi < nwu) {
-            const uint32_t before = found + incl - c, after = found + incl;
-            if (c) last_nz = wi + 1;
-            for (uint32_t m = (before + EPL) / EPL; m < (uint32_t)LPT && m * EPL <= after; m++)
-                starts[m] = (wu0 + wi) * 32u + select_bit(v, m * EPL - 1u - before) + 1u - U0;
+        if (v1) last_nz = wi + 2;
+        else if (v0) last_nz = wi + 1;
+        const uint32_t total = __shfl_sync(mask, incl, LPT - 1, LPT);
+        const uint32_t rel = target - found;  // wraps for a target before this pass
+        int w = 0;  // first lane whose inclusive count exceeds rel
+#pragma unroll
+        for (int sh = LPT / 2; sh >= 1; sh >>= 1) {
+            const uint32_t o = __shfl_sync(mask, incl, w + sh - 1, LPT);
+            if (o <= rel) w += sh;
         }
-        found += __shfl_sync(mask, incl, LPT - 1, LPT);
+        const uint32_t ex = __shfl_sync(mask, incl - c, w, LPT);
+        const uint32_t a0 = __shfl_sync(mask, v0, w, LPT), a1 = __shfl_sync(mask, v1, w, LPT);
+        const uint32_t ac0 = __shfl_sync(mask, c0, w, LPT);
+        if (l > 0 && rel < total) {
+            const uint32_t r = rel - ex;
+            const uint32_t bit = r < ac0 ? select_bit(a0, r) : 32u + select_bit(a1, r - ac0);
+            start = (wu0 + wb + 2u * (uint32_t)w) * 32u + bit + 1u - U0;
+        }
+        found += total;
     }
     last_nz = group_max<LPT>(mask, last_nz);
     // a variable-rate tile ends in its last word (no whole word of padding)
     if (!bad && (found != (uint32_t)N || (!fixed && last_nz != nwu))) bad = true;
-    __syncwarp(mask);
 
 #pragma unroll
     for (int r = 0; r < EPL; r++) u[r] = 0;
@@ -164,7 +180,6 @@ __device__ __forceinline__ bool parse_staged(const DecodeArgs &a, const TileHdr 
         return true;
     }
 
-    const uint32_t start = l > 0 ? starts[l] : 0u;
     // the next lane's start bounds this lane's codes
     uint32_t end = __shfl_down_sync(mask, start, 1, LPT);
     if (l == LPT - 1) {
@@ -295,9 +310,11 @@ __device__ __forceinline__ void points_from_symbols(const uint32_t (&u)[EPL], ui
 // (D = 1, 4, 8: integer points, E8's half-integer coset odd).  With z the
 // unzigzagged symbol, 2z = u ^ -(u & 1); a stripped last coordinate s =
 // floor(z / 2) is restored as 2z = 2 (2s) + 2 parity(sum of the others), that
-// parity being bit 1 of the XOR of the others' 2z.
+// parity being bit 1 of the XOR of the others' 2z.  `bias` is added to every
+// coordinate (with the coset), e.g. the bit pattern of 1.5 2^23.
 template <int D, int EPL>
-__device__ __forceinline__ void doubled_from_symbols(const uint32_t (&u)[EPL], uint32_t cb, int32_t (&t)[EPL])
+__device__ __forceinline__ void doubled_from_symbols(const uint32_t (&u)[EPL], uint32_t cb, int32_t (&t)[EPL],
+                                                     int32_t bias = 0)
 {
     static_assert(D != 2, "A2 has no integer form");
     constexpr int VPL = EPL / D;
@@ -312,7 +329,7 @@ __device__ __forceinline__ void doubled_from_symbols(const uint32_t (&u)[EPL], u
             for (int m = 0; m < D - 1; m++) x ^= d2[m];
             d2[D - 1] = 2 * d2[D - 1] + (x & 2);
         }
-        const int32_t c = (D == 8) ? (int32_t)((cb >> qv) & 1u) : 0;
+        const int32_t c = ((D == 8) ? (int32_t)((cb >> qv) & 1u) : 0) + bias;
 #pragma unroll
         for (int m = 0; m < D; m++) t[qv * D + m] = d2[m] + c;
     }
