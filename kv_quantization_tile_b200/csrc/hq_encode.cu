@@ -126,187 +126,6 @@ __device__ __forceinline__ void load_raw(const void *x, int64_t e0, RawTile<EPL,
     for (int i = 0; i < (F32IN ? EPL / 4 : EPL / 8); i++) r.q[i] = __ldg(p + i);
 }
 
-template <int EPL, bool F32IN>
-__device__ __forceinline__ void unpack_raw(const RawTile<EPL, F32IN> &r, float (&w)[EPL])
-{
-#pragma unroll
-    for (int i = 0; i < (F32IN ? EPL / 4 : EPL / 8); i++) {
-        const uint32_t qq[4] = { r.q[i].x, r.q[i].y, r.q[i].z, r.q[i].w };
-#pragma unroll
-        for (int h = 0; h < 4; h++) {
-            if constexpr (F32IN) {
-                w[4 * i + h] = __uint_as_float(qq[h]);
-            } else {
-                w[8 * i + 2 * h] = __uint_as_float(qq[h] << 16);
-                w[8 * i + 2 * h + 1] = __uint_as_float(qq[h] & 0xffff0000u);
-            }
-        }
-    }
-}
-
-// Nearest lattice points of this lane's EPL / D vectors of v / Delta
-// (+ dither), stripped and zigzagged into u; returns the lane's coset bits
-// (bit q for vector q).  sb = 0: the all-zero tile.
-template <int D, int EPL, bool DITHER>
-__device__ __forceinline__ uint32_t quantize_lane(const float (&v)[EPL], uint32_t sb, uint64_t tkey, int l,
-                                                  const A2Consts &a2, uint32_t (&u)[EPL])
-{
-    constexpr int VPL = EPL / D;
-    uint32_t cbits = 0;
-#pragma unroll
-    for (int r = 0; r < EPL; r++) u[r] = 0;
-    if (sb != 0) {
-        const float inv = __frcp_rn(bf16_bits_to_float(sb));
-        float r4[4];
-#pragma unroll
-        for (int q = 0; q < VPL; q++) {
-            float x[D], p[D];
-            int z[D], c;
-#pragma unroll
-            for (int m = 0; m < D; m++) x[m] = __fmul_rn(v[q * D + m], inv);
-            if constexpr (DITHER) {
-                float dl[D];
-                dither_vec<D, EPL>(tkey, l, q, r4, dl, a2);
-#pragma unroll
-                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
-            }
-            nearest<D>(x, c, z, p, a2);
-            cbits |= (uint32_t)c << q;
-#pragma unroll
-            for (int m = 0; m < D; m++) {
-                int s = z[m];
-                if constexpr (D == 8 || D == 4) {
-                    if (m == D - 1) s >>= 1;  // floor(z / 2): its parity follows from the even sum
-                }
-                u[q * D + m] = zigzag(s);
-            }
-        }
-    }
-    return cbits;
-}
-
-// Rice parameter: smallest k minimising sum(u >> k) + N (1 + k) over the
-// group's symbols.  One pass gives the sums at k0-1, k0, k0+1 (k0 = the
-// rate's typical k); the cost is convex in k, so k0 is optimal iff
-// C(k0-1) > C(k0) <= C(k0+1), and only otherwise does the search walk on.
-// `part` gets this lane's sum(u >> k) at the returned k.
-template <int N, int EPL, int LPT>
-__device__ __forceinline__ int rice_param(const uint32_t (&u)[EPL], unsigned mask, int k_hint, uint32_t &part)
-{
-    int k = k_hint;
-    part = 0;
-    const int km = k > 0 ? k - 1 : 0;
-    uint32_t s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-    for (int r = 0; r < EPL; r++) {
-        const uint32_t aa = u[r] >> km;
-        s0 += aa;
-        s1 += aa >> 1;
-        s2 += aa >> 2;
-    }
-    const uint32_t S0 = group_sum<LPT>(mask, s0), S1 = group_sum<LPT>(mask, s1),
-                   S2 = group_sum<LPT>(mask, s2);
-    // sums at km (S0), km + 1 (S1), km + 2 (S2); C(k + 1) < C(k) iff
-    // sum(k) - sum(k + 1) > N
-    bool up = false, down = false;
-    if (k == 0) {
-        if (S0 - S1 <= (uint32_t)N) {
-            part = s0;                       // C(1) >= C(0)
-        } else if (S1 - S2 <= (uint32_t)N) {
-            k = 1;                           // C(1) < C(0), C(2) >= C(1)
-            part = s1;
-        } else {
-            k = 2;
-            part = s2;
-            up = true;
-        }
-    } else if (S0 - S1 <= (uint32_t)N) {     // C(k0 - 1) <= C(k0)
-        k = km;
-        part = s0;
-        down = true;
-    } else if (S1 - S2 > (uint32_t)N && k < 15) {  // C(k0 + 1) < C(k0)
-        k = k + 1;
-        part = s2;
-        up = true;
-    } else {
-        part = s1;
-    }
-    while (down && k > 0) {
-        uint32_t sd = 0;
-#pragma unroll
-        for (int r = 0; r < EPL; r++) sd += u[r] >> (k - 1);
-        if (group_sum<LPT>(mask, sd) - group_sum<LPT>(mask, part) > (uint32_t)N) break;
-        --k;
-        part = sd;
-    }
-    while (up && k < 15) {
-        uint32_t su = 0;
-#pragma unroll
-        for (int r = 0; r < EPL; r++) su += u[r] >> (k + 1);
-        if (group_sum<LPT>(mask, part) - group_sum<LPT>(mask, su) <= (uint32_t)N) break;
-        ++k;
-        part = su;
-    }
-    return k;
-}
-
-// Pack this lane's share of a tile into a zeroed shared-memory image: its
-// coset bits, the k low bits of its symbols, and its unary parts starting
-// uoff bits into the tile's unary section.
-template <int N, int D, int EPL>
-__device__ __forceinline__ void pack_lane(uint32_t *tbuf, int l, int k, uint32_t cbits, const uint32_t (&u)[EPL],
-                                          uint32_t uoff)
-{
-    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
-    constexpr int VPL = EPL / D;
-    if constexpr (C > 0) or_bits32(tbuf, (uint32_t)l * VPL, cbits, VPL);
-    if (k) {
-        const uint32_t lowmask = (1u << k) - 1u;
-        const uint32_t base = (uint32_t)C + (uint32_t)l * EPL * (uint32_t)k;
-        if (k <= 4) {  // 8 codes fit one 32-bit word
-#pragma unroll
-            for (int r0 = 0; r0 < EPL; r0 += 8) {
-                uint32_t acc = 0;
-#pragma unroll
-                for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                or_bits32(tbuf, base + (uint32_t)r0 * k, acc, 8 * k);
-            }
-        } else {
-#pragma unroll
-            for (int r0 = 0; r0 < EPL; r0 += 4) {
-                uint64_t acc = 0;
-#pragma unroll
-                for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-                or_bits(tbuf, base + (uint32_t)r0 * k, acc, 4 * k);
-            }
-        }
-    }
-    // unary parts: eight codes at a time into a 32-bit bitmap
-    uint32_t upos = (uint32_t)C + (uint32_t)N * (uint32_t)k + uoff;
-#pragma unroll
-    for (int r0 = 0; r0 < EPL; r0 += 8) {
-        uint32_t bm = 0, rel = 0;
-#pragma unroll
-        for (int m = 0; m < 8; m++) {
-            const uint32_t pbit = rel + (u[r0 + m] >> k);
-            bm |= shl32(1u, pbit);
-            rel = pbit + 1;
-        }
-        if (rel <= 32) {
-            or_bits32(tbuf, upos, bm, (int)rel);
-        } else {  // a long code: set the terminators one by one
-            uint32_t pr = upos;
-#pragma unroll
-            for (int m = 0; m < 8; m++) {
-                pr += u[r0 + m] >> k;
-                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
-                ++pr;
-            }
-        }
-        upos += rel;
-    }
-}
-
 // ---------------------------------------------------------------- packed path
 // Unpack lane l's EPL raw coordinates into pairs and apply the random signs of
 // the sign word Y (pair m's mask is (Y << m) & 0x80008000, see sign_word).
@@ -373,162 +192,13 @@ __device__ __forceinline__ void dither_at(uint64_t tile_key, uint32_t c0, float 
 
 // Nearest points of lane l's two runs after the half-exchange transform (run
 // A: tile coordinates RL l .., run B: N/2 + RL l .., RL = EPL / 2) of
-// v / Delta [+ dither], stripped and zigzagged into u (run A's symbols, then
-// run B's, each in coordinate order).  sig: the transform's signs (bit 0: run
-// A negated, bit 1: run B).  Returns the coset bits (bit q: run A's vector q,
-// bit RL / D + q: run B's).  sb = 0: the all-zero tile.
-template <int N, int D, int EPL, bool DITHER>
-__device__ __forceinline__ uint32_t quantize_hx(const float2 (&P)[EPL / 2], uint32_t sb, uint32_t sig, uint64_t tkey,
-                                                int l, const A2Consts &a2, uint32_t (&u)[EPL])
-{
-    constexpr int NP = EPL / 2, HP = NP / 2, RL = EPL / 2, VPR = RL / D;
-    uint32_t cbits = 0;
-#pragma unroll
-    for (int r = 0; r < EPL; r++) u[r] = 0;
-    if (sb == 0) return 0;
-    const float inv = __frcp_rn(bf16_bits_to_float(sb));
-    const float2 ia = splat2((sig & 1u) ? -inv : inv), ib = splat2((sig & 2u) ? -inv : inv);
-    float2 X[NP];
-#pragma unroll
-    for (int m = 0; m < NP; m++) X[m] = mul2(P[m], m < HP ? ia : ib);
-    float r4[4];
-#pragma unroll
-    for (int run = 0; run < 2; run++) {
-        const uint32_t cbase = (run ? (uint32_t)N / 2 : 0u) + (uint32_t)l * RL;
-#pragma unroll
-        for (int q = 0; q < VPR; q++) {
-            float2 V[D > 1 ? D / 2 : 1];
-            float x[D];
-#pragma unroll
-            for (int m = 0; m < D; m++) {
-                const int i = q * D + m;  // coordinate within the run: pair i / 2, element i & 1
-                x[m] = (i & 1) ? X[run * HP + i / 2].y : X[run * HP + i / 2].x;
-            }
-            if constexpr (DITHER) {
-                float dl[D];
-                dither_at<D>(tkey, cbase + (uint32_t)(q * D), r4, dl, a2);
-#pragma unroll
-                for (int m = 0; m < D; m++) x[m] = __fadd_rn(x[m], dl[m]);
-            }
-            uint32_t *uu = u + run * RL + q * D;
-            int c = 0;
-            if constexpr (D == 8) {
-#pragma unroll
-                for (int i = 0; i < 4; i++) V[i] = make_float2(x[2 * i], x[2 * i + 1]);
-                int32_t zb[8];
-                bool tie;
-                c = e8_fast(V, zb, tie);
-                if (tie) {  // several coordinates tie for the parity fix: the sequential rule
-                    int zz[8];
-                    float pp[8];
-                    nearest<8>(x, c, zz, pp, a2);
-#pragma unroll
-                    for (int i = 0; i < 8; i++) zb[i] = zz[i] + kMagicBias;
-                }
-#pragma unroll
-                for (int i = 0; i < 7; i++) {
-                    const int32_t t2 = (int32_t)(((uint32_t)zb[i] << 1) - ((uint32_t)kMagicBias << 1));  // 2 z
-                    uu[i] = (uint32_t)t2 ^ (uint32_t)(t2 >> 31);
-                }
-                const int32_t t7 = (zb[7] - kMagicBias) & ~1;  // 2 floor(z / 2)
-                uu[7] = (uint32_t)t7 ^ (uint32_t)(t7 >> 31);
-            } else {
-                int z[D];
-                float p[D];
-                nearest<D>(x, c, z, p, a2);
-#pragma unroll
-                for (int m = 0; m < D; m++) {
-                    int sv = z[m];
-                    if constexpr (D == 4) {
-                        if (m == D - 1) sv >>= 1;
-                    }
-                    uu[m] = zigzag(sv);
-                }
-            }
-            cbits |= (uint32_t)c << (run * VPR + q);
-        }
-    }
-    return cbits;
-}
-
-// OR `cnt` codes' k low bits (code i at bit pos + i k) into a zeroed image.
-template <int CNT>
-__device__ __forceinline__ void pack_low_run(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u)
-{
-    const uint32_t lowmask = (1u << k) - 1u;
-    if (k <= 4) {  // 8 codes per 32-bit word
-#pragma unroll
-        for (int r0 = 0; r0 < CNT; r0 += 8) {
-            uint32_t acc = 0;
-#pragma unroll
-            for (int m = 7; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-            or_bits32(tbuf, pos + (uint32_t)r0 * k, acc, 8 * k);
-        }
-    } else {
-#pragma unroll
-        for (int r0 = 0; r0 < CNT; r0 += 4) {
-            uint64_t acc = 0;
-#pragma unroll
-            for (int m = 3; m >= 0; m--) acc = (acc << k) | (u[r0 + m] & lowmask);
-            or_bits(tbuf, pos + (uint32_t)r0 * k, acc, 4 * k);
-        }
-    }
-}
-
-// OR `cnt` codes' unary parts (q = u >> k zeros, then a one), starting at bit
-// pos, into a zeroed image, eight codes at a time.
-template <int CNT>
-__device__ __forceinline__ void pack_unary_run(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u)
-{
-#pragma unroll
-    for (int r0 = 0; r0 < CNT; r0 += 8) {
-        uint32_t bm = 0, rel = 0;
-#pragma unroll
-        for (int m = 0; m < 8; m++) {
-            const uint32_t pbit = rel + (u[r0 + m] >> k);
-            bm |= shl32(1u, pbit);
-            rel = pbit + 1;
-        }
-        if (rel <= 32) {
-            or_bits32(tbuf, pos, bm, (int)rel);
-        } else {  // a long code: set the terminators one by one
-            uint32_t pr = pos;
-#pragma unroll
-            for (int m = 0; m < 8; m++) {
-                pr += u[r0 + m] >> k;
-                atomicOr(&tbuf[pr >> 5], 1u << (pr & 31));
-                ++pr;
-            }
-        }
-        pos += rel;
-    }
-}
-
-// Pack lane l's two runs into a zeroed shared-memory image: coset bits, low
-// parts, and unary parts starting uoffA / uoffB bits into the unary section.
-template <int N, int D, int EPL>
-__device__ __forceinline__ void pack_hx(uint32_t *tbuf, int l, int k, uint32_t cbits, const uint32_t (&u)[EPL],
-                                        uint32_t uoffA, uint32_t uoffB)
-{
-    constexpr int C = (D == 8 || D == 2) ? N / D : 0;
-    constexpr int RL = EPL / 2, VPR = RL / D;
-    if constexpr (C > 0) {
-        or_bits32(tbuf, (uint32_t)l * VPR, cbits & ((1u << VPR) - 1u), VPR);
-        or_bits32(tbuf, (uint32_t)(N / (2 * D)) + (uint32_t)l * VPR, cbits >> VPR, VPR);
-    }
-    if (k) {
-        pack_low_run<RL>(tbuf, (uint32_t)C + (uint32_t)l * RL * (uint32_t)k, k, u);
-        pack_low_run<RL>(tbuf, (uint32_t)C + ((uint32_t)N / 2 + (uint32_t)l * RL) * (uint32_t)k, k, u + RL);
-    }
-    const uint32_t ubase = (uint32_t)C + (uint32_t)N * (uint32_t)k;
-    pack_unary_run<RL>(tbuf, ubase + uoffA, k, u);
-    pack_unary_run<RL>(tbuf, ubase + uoffB, k, u + RL);
-}
-
-// The same as quantize_hx with the symbols as exact binary32 integers in
-// pairs (U[m]: symbols 2m, 2m + 1 of the lane's run-A-then-run-B order).  E8
-// uses e8_symbols (the fma pipe); a vector whose parity fix ties between
-// coordinates, and the other lattices, take the scalar nearest point.
+// v / Delta [+ dither], stripped and zigzagged, as exact binary32 integers in
+// pairs (U[m]: symbols 2m, 2m + 1 of the lane's run-A-then-run-B order, each
+// run in coordinate order).  sig: the transform's signs (bit 0: run A
+// negated, bit 1: run B).  Returns the coset bits (bit q: run A's vector q,
+// bit RL / D + q: run B's).  sb = 0: the all-zero tile.  E8 uses e8_symbols
+// (the fma pipe); a vector whose parity fix ties between coordinates, and the
+// other lattices, take the scalar nearest point.
 template <int N, int D, int EPL, bool DITHER>
 __device__ __forceinline__ uint32_t quantize_hx_f(const float2 (&P)[EPL / 2], uint32_t sb, uint32_t sig,
                                                   uint64_t tkey, int l, const A2Consts &a2, float2 (&U)[EPL / 2])
@@ -626,10 +296,11 @@ __device__ __forceinline__ void shifted_sums(const float2 (&U)[EPL / 2], int k, 
     sbv = b - kBiasRun;
 }
 
-// Rice parameter from float symbols: as rice_param (exact argmin of the
-// tile's coded length, smallest k on ties; one pass over k0-1, k0, k0+1, a
-// walk only if the optimum lies outside).  partA / partB: this lane's
-// sum(u >> k) over run A / run B at the returned k.
+// Rice parameter: the smallest k minimising sum(u >> k) + N (1 + k) over the
+// group's symbols.  One pass gives the sums at k0-1, k0, k0+1 (k0 = the
+// rate's typical k); the cost is convex in k, so k0 is optimal iff
+// C(k0-1) > C(k0) <= C(k0+1), and only otherwise does the search walk on.
+// partA / partB: this lane's sum(u >> k) over run A / run B at the returned k.
 template <int N, int EPL, int LPT>
 __device__ __forceinline__ int rice_param_f(const float2 (&U)[EPL / 2], unsigned mask, int k_hint, uint32_t &partA,
                                             uint32_t &partB)
@@ -702,8 +373,8 @@ __device__ __forceinline__ void run_words8(const float2 *U, int k, uint32_t &low
     unary = bm;
 }
 
-// OR `cnt` codes' k low bits into a zeroed image, writes confined to the
-// image's first `limit` words (as pack_low_run).
+// OR `cnt` codes' k low bits (code i at bit pos + i k) into a zeroed image,
+// four codes at a time, writes confined to the image's first `limit` words.
 template <int CNT>
 __device__ __forceinline__ void pack_low_run_lim(uint32_t *tbuf, uint32_t pos, int k, const uint32_t *u, uint32_t limit)
 {
@@ -733,8 +404,9 @@ __device__ __forceinline__ void pack_unary_run_lim(uint32_t *tbuf, uint32_t pos,
     }
 }
 
-// Pack lane l's two runs of float symbols into a zeroed shared-memory image
-// (as pack_hx).  spanA / spanB: the runs' unary bits (sum of q + 1); limit:
+// Pack lane l's two runs of float symbols into a zeroed shared-memory image:
+// coset bits, low parts, and unary parts starting uoffA / uoffB bits into the
+// unary section.  spanA / spanB: the runs' unary bits (sum of q + 1); limit:
 // the words of the group's image from tbuf on (no write goes past them).
 template <int N, int D, int EPL>
 __device__ __forceinline__ void pack_hx_f(uint32_t *tbuf, int l, int k, uint32_t cbits, const float2 (&U)[EPL / 2],
@@ -941,7 +613,15 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
                         const uint32_t gw = g < 32 ? __shfl_sync(FULL, mine, g) : __shfl_sync(FULL, mine2, g - 32);
                         const uint32_t *src = stage + (size_t)g * gstride;
                         uint32_t *dst = a.payload + base + go;
-                        for (uint32_t i = lane; i < gw; i += 32) dst[i] = src[i];
+                        uint32_t i = lane;
+                        for (; i + 96 < gw; i += 128) {  // four loads in flight per lane
+                            const uint32_t w0 = src[i], w1 = src[i + 32], w2 = src[i + 64], w3 = src[i + 96];
+                            dst[i] = w0;
+                            dst[i + 32] = w1;
+                            dst[i + 64] = w2;
+                            dst[i + 96] = w3;
+                        }
+                        for (; i < gw; i += 32) dst[i] = src[i];
                     }
                 }
                 if (lane < GPB) s_goff[lane] = gexcl;
@@ -983,8 +663,9 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 constexpr int kFixedWarps = 8, kFixedThreads = kFixedWarps * 32;
 // Resident blocks the registers are budgeted for: the rotated tile, the
 // next tile's raw words and a probe's symbols are live together.  At 80
-// registers (3 blocks per SM) E8 spills a few words, yet measured faster
-// than 128 registers without spills (2 blocks) and no slower than 64 (4).
+// registers (3 blocks per SM) E8 spills a few words, yet the Llama layer
+// encodes faster than with 128 registers and no spills (2 blocks: 2.04 vs
+// 1.87 ms) and level with 64 (4 blocks: 1.88 ms).
 constexpr int fixed_min_blocks(int epl) { return epl >= 32 ? 1 : 3; }
 constexpr int kFixedMaxProbes = 64;  // the search needs at most about 20
 enum { kPredict, kStart, kDown, kUp, kBisect, kFinal };  // scale search phases
@@ -994,30 +675,31 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
     encode_fixed_kernel(const EncodeArgs a)
 {
     constexpr int LPT = N / EPL, TPW = 32 / LPT, GPB = kFixedWarps * TPW;
-    constexpr int WPT = N / 64 > 0 ? N / 64 : 1;
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
-    static_assert(EPL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32, "layout");
+    constexpr int NP = EPL / 2, RL = EPL / 2;
+    static_assert(EPL % D == 0 && RL % D == 0 && LPT <= 32 && (32 % LPT) == 0 && EPL <= 32 && LPT >= 2, "layout");
     const uint32_t S = a.slot_words;
     const uint32_t istride = (S + 1 + 3) & ~3u;  // slot image + a guard word, 16-byte multiple
+    const int ywords = a.sign_words ? (int)a.tiles_per_row * LPT : 0;  // sign words cached per block
     extern __shared__ __align__(16) uint32_t smem[];
-    unsigned long long *sign_tab = reinterpret_cast<unsigned long long *>(smem);
-    uint32_t *images = smem + 2 * ((a.sign_words + 1) & ~1);
-    uint32_t *sym = images + (size_t)GPB * istride;  // [EPL + 3][threads]: the last fitting probe's symbols
+    uint32_t *ytab = smem;                                       // [tiles_per_row][LPT]
+    uint32_t *images = smem + ((ywords + 3) & ~3);
+    float *sym = reinterpret_cast<float *>(images + (size_t)GPB * istride);  // [NP * 2 + 4][threads]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < a.sign_words; i += kFixedWarps * 32) {
-        const uint64_t j = (uint64_t)(i / WPT), m = (uint64_t)(i % WPT);
-        sign_tab[i] = mix64(mix64(a.sign_key ^ j) ^ m);
-    }
+    for (int i = tid; i < ywords; i += kFixedThreads)
+        ytab[i] = encode_sign_word<N, EPL>(a.sign_key, (uint64_t)(i / LPT), i % LPT);
     __syncthreads();
 
     const int l = lane % LPT;
     const int gid = warp * TPW + lane / LPT;
     const unsigned mask = group_mask<LPT>(lane);
+    const uint32_t sig = hx_sigma_bits<LPT>(l);
     uint32_t *img = images + (size_t)gid * istride;
     const int64_t npairs = (a.ntiles + 1) >> 1;
     const uint32_t tpr = (uint32_t)a.tiles_per_row;
     const uint32_t budget = 32u * S;
+    uint32_t *keep = reinterpret_cast<uint32_t *>(sym);
 
     for (int64_t p = (int64_t)blockIdx.x * GPB + gid; p < npairs; p += (int64_t)gridDim.x * GPB) {
         uint32_t kbyte = 0;
@@ -1029,22 +711,16 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
         for (int h = 0; h < 2; h++) {
             const int64_t t = tp + h;
             if (t >= a.ntiles) break;  // group-uniform
-            // ---- signs, then prefetch the pair's second tile
-            const uint32_t i0 = (uint32_t)l * EPL;
-            const uint64_t sw = a.sign_words ? sign_tab[(uint64_t)jj * WPT + (i0 >> 6)]
-                                             : mix64(mix64(a.sign_key ^ (uint64_t)jj) ^ (uint64_t)(i0 >> 6));
-            const uint32_t sbits = (uint32_t)(sw >> (i0 & 63));
-            float v[EPL];
-            unpack_raw<EPL, F32IN>(raw, v);
-#pragma unroll
-            for (int r = 0; r < EPL; r++)
-                v[r] = __uint_as_float(__float_as_uint(v[r]) ^ ((sbits << (31 - r)) & 0x80000000u));
+            // ---- signs (as pairs), then prefetch the pair's second tile
+            const uint32_t Y = ywords ? ytab[jj * LPT + l] : encode_sign_word<N, EPL>(a.sign_key, jj, l);
+            float2 v[NP];
+            unpack_signed<EPL, F32IN>(raw, Y, v);
             if (h == 0 && t + 1 < a.ntiles) load_raw<EPL, F32IN>(a.x, (t + 1) * N + (int64_t)l * EPL, raw);
             if (++jj == tpr) jj = 0;
 
             // ---- rotation, closed-form start, scale search
-            const float Ssq = sumsq<EPL, LPT>(v, mask);
-            fwht<EPL, LPT>(v, mask, l);
+            const float Ssq = sumsq_pairs<EPL, LPT, !F32IN>(v, mask);
+            fwht_hx<EPL, LPT>(v, mask, l);
             bool nonfinite;
             const uint32_t c0 = tile_scale_bits(Ssq, a.c, nonfinite);
             if (nonfinite && l == 0 && a.status) atomicOr(a.status, kStatusNonfinite);
@@ -1058,20 +734,25 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             const int lo_lim = (int)c0 - 512 > 0x0080 ? (int)c0 - 512 : 0x0080;
             const int hi_lim = (int)c0 + 512 < 0x7f7f ? (int)c0 + 512 : 0x7f7f;
             int phase = c0 ? kPredict : kFinal, lo = 0, hi = (int)c0, step = 1, c = (int)c0;
-            uint32_t u[EPL], cbits, part;
+            float2 U[NP];
+            uint32_t cbits, partA, partB;
             int k;
             for (int probe = 0;; probe++) {
-                cbits = quantize_lane<D, EPL, DITHER>(v, (uint32_t)c, tkey, l, a.a2, u);
-                k = rice_param<N, EPL, LPT>(u, mask, a.k_hint, part);
+                cbits = quantize_hx_f<N, D, EPL, DITHER>(v, (uint32_t)c, sig, tkey, l, a.a2, U);
+                k = rice_param_f<N, EPL, LPT>(U, mask, a.k_hint, partA, partB);
                 if (phase == kFinal) break;
-                const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, part);
+                const uint32_t bits = (uint32_t)C + (uint32_t)N * (uint32_t)(k + 1) + group_sum<LPT>(mask, partA + partB);
                 const bool f = bits <= budget;
                 if (f) {  // keep a fitting probe's symbols: the search's answer is its last fitting probe
 #pragma unroll
-                    for (int r = 0; r < EPL; r++) sym[r * kFixedThreads + tid] = u[r];
-                    sym[(EPL + 0) * kFixedThreads + tid] = cbits;
-                    sym[(EPL + 1) * kFixedThreads + tid] = (uint32_t)k;
-                    sym[(EPL + 2) * kFixedThreads + tid] = part;
+                    for (int m = 0; m < NP; m++) {
+                        sym[(2 * m) * kFixedThreads + tid] = U[m].x;
+                        sym[(2 * m + 1) * kFixedThreads + tid] = U[m].y;
+                    }
+                    keep[(EPL + 0) * kFixedThreads + tid] = cbits;
+                    keep[(EPL + 1) * kFixedThreads + tid] = (uint32_t)k;
+                    keep[(EPL + 2) * kFixedThreads + tid] = partA;
+                    keep[(EPL + 3) * kFixedThreads + tid] = partB;
                 }
                 if (phase == kPredict) {
                     // a pattern step moves the size by about N / 128 bits: start
@@ -1114,10 +795,12 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
                     c = answer;
                     if (answer != 0) {  // an earlier fitting probe: its kept symbols
 #pragma unroll
-                        for (int r = 0; r < EPL; r++) u[r] = sym[r * kFixedThreads + tid];
-                        cbits = sym[(EPL + 0) * kFixedThreads + tid];
-                        k = (int)sym[(EPL + 1) * kFixedThreads + tid];
-                        part = sym[(EPL + 2) * kFixedThreads + tid];
+                        for (int m = 0; m < NP; m++)
+                            U[m] = make_float2(sym[(2 * m) * kFixedThreads + tid], sym[(2 * m + 1) * kFixedThreads + tid]);
+                        cbits = keep[(EPL + 0) * kFixedThreads + tid];
+                        k = (int)keep[(EPL + 1) * kFixedThreads + tid];
+                        partA = keep[(EPL + 2) * kFixedThreads + tid];
+                        partB = keep[(EPL + 3) * kFixedThreads + tid];
                         break;
                     }
                     phase = kFinal;  // the all-zero tile
@@ -1125,11 +808,14 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             }
             const uint32_t sb = (uint32_t)c;
 
-            // ---- pack the chosen symbols, store the slot
-            const uint32_t uoff = group_excl_scan<LPT>(mask, part + EPL, l);
+            // ---- pack the chosen symbols (run A's unary parts precede run B's), store the slot
+            const uint32_t ulA = partA + RL, ulB = partB + RL;
+            const uint32_t totA = group_sum<LPT>(mask, ulA);
+            const uint32_t uoffA = group_excl_scan<LPT>(mask, ulA, l);
+            const uint32_t uoffB = totA + group_excl_scan<LPT>(mask, ulB, l);
             for (uint32_t i = l; i < istride; i += LPT) img[i] = 0u;
             __syncwarp(mask);
-            pack_lane<N, D, EPL>(img, l, k, cbits, u, uoff);
+            pack_hx_f<N, D, EPL>(img, l, k, cbits, U, uoffA, uoffB, ulA, ulB, istride);
             __syncwarp(mask);
             uint32_t *dst = a.payload + (uint64_t)t * S;
             for (uint32_t i = l; i < S; i += LPT) dst[i] = img[i];
@@ -1144,10 +830,8 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
 // ------------------------------------------------------------------ launch
 namespace {
 
-// coordinates per lane: 8 for n = 64, 16 for 128 and 256, 32 above
-template <int N>
-constexpr int epl_for() { return N == 64 ? 8 : (N <= 256 ? 16 : 32); }
-// the variable-rate encoder: at least 16 per lane, so a run holds whole E8 vectors
+// coordinates per lane (both encoders): at least 16, so each of a lane's two
+// runs after the half-exchange transform holds whole E8 vectors
 template <int N>
 constexpr int epl_var() { return N <= 256 ? 16 : 32; }
 
@@ -1198,10 +882,11 @@ cudaError_t launch_encode_n(int lattice, bool dither, int dtype, const EncodeArg
 template <int N, int D, bool DITHER, bool F32IN>
 cudaError_t launch_encode_fixed_t(const EncodeArgs &a, cudaStream_t s)
 {
-    constexpr int EPL = epl_for<N>(), GPB = kFixedWarps * (32 / (N / EPL));
+    constexpr int EPL = epl_var<N>(), GPB = kFixedWarps * (32 / (N / EPL));
     const size_t istride = (a.slot_words + 1 + 3) & ~(size_t)3;
-    const size_t smem = (size_t)((a.sign_words + 1) & ~1) * 8 + (size_t)GPB * istride * 4 +
-                        (size_t)(EPL + 3) * kFixedThreads * 4;
+    const size_t ywords = a.sign_words ? (size_t)a.tiles_per_row * (N / EPL) : 0;
+    const size_t smem = ((ywords + 3) & ~(size_t)3) * 4 + (size_t)GPB * istride * 4 +
+                        (size_t)(EPL + 4) * kFixedThreads * 4;
     auto kern = encode_fixed_kernel<N, D, EPL, DITHER, F32IN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -193,87 +193,28 @@ __host__ __device__ __forceinline__ uint32_t sign_word(F neg)
 }
 
 // ------------------------------------------------------------- E8
-// Fast E8 nearest point of one vector (4 pairs of x = v / Delta [+ dither]):
-// the same decision as the Conway-Sloane two-coset rule with the exact
-// distance identity (see nearest<8> in hq_device.cuh), in a branch-free form.
-//   R = x + 1.5 2^23 rounded to nearest (bits: B + rint x), F = the same add
-//   rounded down (B + floor x), e = x - rint x, all exact for |x| < 2^22.
+constexpr int32_t kMagicBias = 0x4B400000;  // bits of 1.5 * 2^23: B + k is the float 1.5 2^23 + k
+
+// E8 nearest point and symbols of one vector (4 pairs of x = v / Delta
+// [+ dither]): the Conway-Sloane two-coset rule with the exact distance
+// identity (see nearest<8> in hq_device.cuh), branch-free and in binary32
+// arithmetic on exact small integers (the fma pipe).
+//   R = x + 1.5 2^23 rounded to nearest (rint x, biased), F = the same add
+//   rounded down (floor x, biased), e = x - rint x, all exact for |x| < 2^22.
 //   d0 - d1 = sum|e| - 2 + [sum rint odd](1 - 2 max|e|) - [sum floor odd] 2 min|e|
 //   (binary32, this order); d0 - d1 <= 0 keeps the integer coset.
 //   The parity fix moves the coordinate of largest |e| (integer coset) or
 //   smallest |e| (half-integer coset) one step towards x.  With C = F - R
-//   (-1 where rint = floor + 1, i.e. e < 0) and H = -1 at the moved coordinate:
-//     integer coset:      z = F - (C ^ H)
-//     half-integer coset: z = F - ((C & H) + (H & ~C & 1))
-//   (z = the stored integer y - c/2, biased by B).  When |e| == T holds for
-//   more than one coordinate the first index must move; `tie` reports that
-//   case and the caller decodes the vector with the sequential rule instead.
-//   Returns the coset bit; zb gets the biased integers.
-__device__ __forceinline__ int e8_fast(const float2 (&X)[4], int32_t (&zb)[8], bool &tie)
-{
-    constexpr float kM = 12582912.0f;  // 1.5 * 2^23
-    const float2 M2 = splat2(kM);
-    float2 R[4], F[4], E[4];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        R[i] = add2(X[i], M2);
-        F[i] = add2_rd(X[i], M2);
-        E[i] = sub2(X[i], sub2(R[i], M2));
-    }
-    const float ae[8] = { fabsf(E[0].x), fabsf(E[0].y), fabsf(E[1].x), fabsf(E[1].y),
-                          fabsf(E[2].x), fabsf(E[2].y), fabsf(E[3].x), fabsf(E[3].y) };
-    float s = ae[0], mx = ae[0], mn = ae[0];
-#pragma unroll
-    for (int i = 1; i < 8; i++) {
-        s = __fadd_rn(s, ae[i]);
-        mx = fmaxf(mx, ae[i]);
-        mn = fminf(mn, ae[i]);
-    }
-    const int32_t r[8] = { __float_as_int(R[0].x), __float_as_int(R[0].y), __float_as_int(R[1].x),
-                           __float_as_int(R[1].y), __float_as_int(R[2].x), __float_as_int(R[2].y),
-                           __float_as_int(R[3].x), __float_as_int(R[3].y) };
-    const int32_t f[8] = { __float_as_int(F[0].x), __float_as_int(F[0].y), __float_as_int(F[1].x),
-                           __float_as_int(F[1].y), __float_as_int(F[2].x), __float_as_int(F[2].y),
-                           __float_as_int(F[3].x), __float_as_int(F[3].y) };
-    const int32_t px = r[0] ^ r[1] ^ r[2] ^ r[3] ^ r[4] ^ r[5] ^ r[6] ^ r[7];
-    const int32_t py = f[0] ^ f[1] ^ f[2] ^ f[3] ^ f[4] ^ f[5] ^ f[6] ^ f[7];
-    const bool odd0 = px & 1, odd1 = py & 1;
-    float dd = __fsub_rn(s, 2.0f);
-    if (odd0) dd = __fadd_rn(dd, __fmaf_rn(mx, -2.0f, 1.0f));  // 1 - 2 max|e|: one rounding
-    if (odd1) dd = __fmaf_rn(mn, -2.0f, dd);                    // dd - 2 min|e|: one rounding
-    const bool one = dd > 0.0f;
-    const bool fix = one ? odd1 : odd0;
-    const float T = fix ? (one ? mn : mx) : -1.0f;
-    int32_t H[8], cnt = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        H[i] = ae[i] == T ? -1 : 0;
-        cnt += H[i];
-    }
-    tie = cnt < -1;
-    // one 3-input logic op picks the coset's formula per coordinate
-    const int32_t Q = one ? -1 : 0, Q1 = Q & 1;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const int32_t C = f[i] - r[i];
-        const int32_t p = ((C ^ H[i]) & ~Q) | (C & H[i] & Q);
-        zb[i] = f[i] - p - (H[i] & ~C & Q1);
-    }
-    return one ? 1 : 0;
-}
-
-constexpr int32_t kMagicBias = 0x4B400000;  // bits of 1.5 * 2^23: B + k is the float 1.5 2^23 + k
-
-// The same decision with the per-coordinate selection, the parity fix and
-// the strip + zigzag done in binary32 arithmetic on exact small integers (the
-// fma pipe) instead of integer logic: with C = F - R (0, or -1 where rint =
-// floor + 1) and h = +1 (integer coset) or -1 (half-integer coset) at the
-// moved coordinate, 0 elsewhere,
-//   z = F - [integer coset] C + h (1 + 2C)   (biased by 1.5 2^23, then removed),
-// and the zigzag of an integer z is |2z + 1/2| - 1/2 (2z for z >= 0, -2z - 1
-// below).  The last coordinate is stored as floor(z / 2) (an fma rounded
-// down against 1.5 2^23).  U gets the 8 symbols as exact binary32 integers.
-// Returns the coset bit; tie as in e8_fast.
+//   (0, or -1 where rint = floor + 1) and h = +1 (integer coset) or -1
+//   (half-integer coset) at the moved coordinate, 0 elsewhere,
+//     z = F - [integer coset] C + h (1 + 2C)   (biased by 1.5 2^23, then removed)
+//   is the stored integer y - c/2, and the zigzag of an integer z is
+//   |2z + 1/2| - 1/2 (2z for z >= 0, -2z - 1 below).  The last coordinate is
+//   stored as floor(z / 2) (an fma rounded down against 1.5 2^23).
+// U gets the 8 symbols as exact binary32 integers; returns the coset bit.
+// When |e| == T holds for more than one coordinate the first index must
+// move: `tie` reports that case, and the caller decodes the vector with the
+// sequential rule instead.
 __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4], bool &tie)
 {
     constexpr float kM = 12582912.0f;  // 1.5 * 2^23
