@@ -149,6 +149,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 16-byte global -> shared copy through L2 (cp.async, no registers held)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -292,6 +300,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
                     break;
                 }
             }
+            // B: X~ rows b0 .. b0 + NB - 1 of tile j (consecutive threads:
+            // consecutive rows), copied asynchronously while A is parsed
+            for (int e = tid; e < NB * 32; e += kGemmThreads) {
+                const int n = e % NB, kc = e / NB;
+                cp_async16(aB + (uint32_t)((n & 7) + 8 * (n >> 3)) * 16u + (uint32_t)kc * LBO_B,
+                           a.xt + (int64_t)(b0 + n) * a.cols + j * N + kc * 8);
+            }
+            cp_async_commit();
             // A: rows r0 .. r0 + 127 of column tile j, lane l's chunks 2l and 2l + 1
             for (int m = gid; m < kGemmM; m += GPB) {
                 const int64_t r = r0 + m;
@@ -315,13 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
                 }
                 if (bad && l == 0 && a.status) atomicOr(a.status, kStatusCorrupt);
             }
-            // B: X~ rows b0 .. b0 + NB - 1 of tile j (consecutive threads: consecutive rows)
-            for (int e = tid; e < NB * 32; e += kGemmThreads) {
-                const int n = e % NB, kc = e / NB;
-                const uint4 v =
-                    __ldg(reinterpret_cast<const uint4 *>(a.xt + (int64_t)(b0 + n) * a.cols + j * N + kc * 8));
-                *reinterpret_cast<uint4 *>(sB + (uint32_t)((n & 7) + 8 * (n >> 3)) * 16u + (uint32_t)kc * LBO_B) = v;
-            }
+            cp_async_wait_all();  // this thread's B chunks have landed
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
