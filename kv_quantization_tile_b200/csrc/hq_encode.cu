@@ -197,8 +197,7 @@ __device__ __forceinline__ void dither_at(uint64_t tile_key, uint32_t c0, float 
 // run in coordinate order).  sig: the transform's signs (bit 0: run A
 // negated, bit 1: run B).  Returns the coset bits (bit q: run A's vector q,
 // bit RL / D + q: run B's).  sb = 0: the all-zero tile.  E8 uses e8_symbols
-// (the fma pipe); a vector whose parity fix ties between coordinates, and the
-// other lattices, take the scalar nearest point.
+// (the fma pipe), the other lattices the scalar nearest point.
 template <int N, int D, int EPL, bool DITHER>
 __device__ __forceinline__ uint32_t quantize_hx_f(const float2 (&P)[EPL / 2], uint32_t sb, uint32_t sig,
                                                   uint64_t tkey, int l, const A2Consts &a2, float2 (&U)[EPL / 2])
@@ -233,21 +232,17 @@ __device__ __forceinline__ uint32_t quantize_hx_f(const float2 (&P)[EPL / 2], ui
             }
             float us[D];
             int c = 0;
-            bool slow = true;
             if constexpr (D == 8) {
                 float2 V[4], W[4];
 #pragma unroll
                 for (int i = 0; i < 4; i++) V[i] = make_float2(x[2 * i], x[2 * i + 1]);
-                bool tie;
-                c = e8_symbols(V, W, tie);
+                c = e8_symbols(V, W);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     us[2 * i] = W[i].x;
                     us[2 * i + 1] = W[i].y;
                 }
-                slow = tie;  // several coordinates tie for the parity fix: the sequential rule
-            }
-            if (slow) {
+            } else {
                 int z[D];
                 float p[D];
                 nearest<D>(x, c, z, p, a2);

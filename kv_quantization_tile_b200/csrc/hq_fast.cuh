@@ -212,10 +212,9 @@ constexpr int32_t kMagicBias = 0x4B400000;  // bits of 1.5 * 2^23: B + k is the 
 //   |2z + 1/2| - 1/2 (2z for z >= 0, -2z - 1 below).  The last coordinate is
 //   stored as floor(z / 2) (an fma rounded down against 1.5 2^23).
 // U gets the 8 symbols as exact binary32 integers; returns the coset bit.
-// When |e| == T holds for more than one coordinate the first index must
-// move: `tie` reports that case, and the caller decodes the vector with the
-// sequential rule instead.
-__device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4], bool &tie)
+// When |e| == T holds for more than one coordinate, the rule moves the first
+// of them (index order), so h keeps only the first hit.
+__device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4])
 {
     constexpr float kM = 12582912.0f;  // 1.5 * 2^23
     const float2 M2 = splat2(kM);
@@ -247,12 +246,22 @@ __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4], 
     const bool fix = one ? odd1 : odd0;
     const float T = fix ? (one ? mn : mx) : -1.0f;
     const float sc = one ? -1.0f : 1.0f;
-    // H: 1 at the coordinates whose |e| is T, else 0; more than one hit is a tie
+    // H: 1 at the coordinates whose |e| is T, else 0
     float2 H[4];
 #pragma unroll
     for (int i = 0; i < 4; i++) H[i] = make_float2(eq1f(ae[2 * i], T), eq1f(ae[2 * i + 1], T));
     const float2 hs = add2(add2(H[0], H[1]), add2(H[2], H[3]));
-    tie = __fadd_rn(hs.x, hs.y) > 1.5f;
+    if (__fadd_rn(hs.x, hs.y) > 1.5f) {  // a tie: only the first hit (in index order) moves
+        float seen = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float hx = H[i].x, hy = H[i].y;
+            H[i].x = hx * (1.0f - seen);
+            seen = fmaxf(seen, hx);
+            H[i].y = hy * (1.0f - seen);
+            seen = fmaxf(seen, hy);
+        }
+    }
     const float2 mq0 = splat2(one ? 0.0f : -1.0f), two = splat2(2.0f), half = splat2(0.5f);
     const float2 sc2 = splat2(2.0f * sc), sc1 = splat2(sc);
 #pragma unroll
