@@ -402,15 +402,24 @@ __device__ __forceinline__ void pack_unary_run_lim(uint32_t *tbuf, uint32_t pos,
 // Pack lane l's two runs of float symbols into a zeroed shared-memory image:
 // coset bits, low parts, and unary parts starting uoffA / uoffB bits into the
 // unary section.  spanA / spanB: the runs' unary bits (sum of q + 1); limit:
-// the words of the group's image from tbuf on (no write goes past them).
+// the words of the group's image from tbuf on (no write goes past them);
+// mask: the group's lanes (all of them call this together).
 template <int N, int D, int EPL>
 __device__ __forceinline__ void pack_hx_f(uint32_t *tbuf, int l, int k, uint32_t cbits, const float2 (&U)[EPL / 2],
                                           uint32_t uoffA, uint32_t uoffB, uint32_t spanA, uint32_t spanB,
-                                          uint32_t limit)
+                                          uint32_t limit, unsigned mask)
 {
     constexpr int C = (D == 8 || D == 2) ? N / D : 0;
-    constexpr int RL = EPL / 2, VPR = RL / D, HP = EPL / 4;
-    if constexpr (C > 0) {
+    constexpr int RL = EPL / 2, VPR = RL / D, HP = EPL / 4, LPT = N / EPL;
+    if constexpr (C > 0 && VPR == 1 && 2 * LPT <= 32) {
+        // one coset bit per run and lane: the group's bits by two ballots,
+        // run A's in lane order, then run B's, OR-ed in by the first lane
+        const int base = (threadIdx.x & 31) & ~(LPT - 1);
+        const uint32_t gm = LPT == 32 ? 0xffffffffu : (1u << LPT) - 1u;
+        const uint32_t ba = (__ballot_sync(mask, cbits & 1u) >> base) & gm;
+        const uint32_t bb = (__ballot_sync(mask, cbits & 2u) >> base) & gm;
+        if (l == 0) or_bits32_lim(tbuf, 0u, ba | (bb << LPT), C, limit);
+    } else if constexpr (C > 0) {
         or_bits32_lim(tbuf, (uint32_t)l * VPR, cbits & ((1u << VPR) - 1u), VPR, limit);
         or_bits32_lim(tbuf, (uint32_t)(N / (2 * D)) + (uint32_t)l * VPR, cbits >> VPR, VPR, limit);
     }
@@ -555,7 +564,7 @@ __global__ void __launch_bounds__(kEncodeWarps * 32, encode_min_blocks(EPL, D, D
 
                 // ---- pack into the group's image (zeroed at chunk start)
                 uint32_t *tbuf = gstage + goff;
-                if (active && !overflow) pack_hx_f<N, D, EPL>(tbuf, l, k, cbits, U, uoffA, uoffB, ulA, ulB, gstride - goff);
+                if (active && !overflow) pack_hx_f<N, D, EPL>(tbuf, l, k, cbits, U, uoffA, uoffB, ulA, ulB, gstride - goff, mask);
                 if (overflow && l == 0 && a.status) atomicOr(a.status, kStatusCapacity);
                 if (l == 0) {
                     tile_w[gid * G + gi] = goff;
@@ -810,7 +819,7 @@ __global__ void __launch_bounds__(kFixedWarps * 32, fixed_min_blocks(EPL))
             const uint32_t uoffB = totA + group_excl_scan<LPT>(mask, ulB, l);
             for (uint32_t i = l; i < istride; i += LPT) img[i] = 0u;
             __syncwarp(mask);
-            pack_hx_f<N, D, EPL>(img, l, k, cbits, U, uoffA, uoffB, ulA, ulB, istride);
+            pack_hx_f<N, D, EPL>(img, l, k, cbits, U, uoffA, uoffB, ulA, ulB, istride, mask);
             __syncwarp(mask);
             uint32_t *dst = a.payload + (uint64_t)t * S;
             for (uint32_t i = l; i < S; i += LPT) dst[i] = img[i];
