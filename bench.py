@@ -49,7 +49,7 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip GEMV/KV/e2e/CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", default=None, help="comma-separated matrix names (profiling cases)")
-    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "configs", "dit", "kv_attention", "fixed"],
+    p.add_argument("--leg", default=None, choices=["gemv", "gemm", "configs", "dit", "kv_attention", "fixed", "profile"],
                    help="run one side leg alone on cuda:0 and print its JSON (profiling cases)")
     p.add_argument("--group", type=int, default=4, help="query heads per KV head for --leg kv_attention")
     p.add_argument("--batch", type=int, default=None, help="one batch size for --leg gemm")
@@ -832,6 +832,43 @@ def fixed_leg(dev, peak):
     return res
 
 
+def profile_leg(dev):
+    """One cold launch each of the decode-GEMV (14336 x 4096, E8 4 bps), the
+    fixed-rate encode of the Llama gate matrix (31-word slots) and the KV
+    attention of 32 query heads over the 8 x 32768 x 128 E8 4-bps K and V
+    streams: the launches the path profiles capture."""
+    import torch
+
+    from kv_quantization_tile_b200 import hq, workloads
+
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    w1, _, x1, _ = workloads.gemv_case(dev)
+    r, c = w1.shape
+    s = hq.alloc_stream(r, c, TILE, LAT, BPS, dev)
+    hq.hq_encode(w1, TILE, LAT, BPS, SEED, s, hq.alloc_workspace(r, c, TILE, dev), st)
+    y = torch.empty(r, dtype=torch.float32, device=dev)
+    hq.hq_decode_gemv(s, r, c, TILE, LAT, BPS, SEED, x1, y, st)
+    gate = workloads.llama_layer(dev, names=["gate"])[0][1]
+    slot = hq.hq_fixed_slot_words(TILE, LAT, BPS)
+    fs = hq.alloc_fixed_stream(gate.shape[0], gate.shape[1], TILE, slot, dev)
+    hq.hq_encode_fixed(gate, TILE, LAT, SEED, fs, st)
+    k, v = workloads.kv_layer(dev)
+    heads, tokens, d = workloads.KV_HEADS, workloads.KV_TOKENS, workloads.KV_HEAD_DIM
+    streams = []
+    for x, seed in ((k, SEED), (v, SEED + 1)):
+        sx = hq.alloc_stream(heads * tokens, d, d, LAT, BPS, dev)
+        hq.hq_kv_encode(x, d, LAT, BPS, seed, sx, hq.alloc_workspace(heads * tokens, d, d, dev), st)
+        streams.append(sx)
+    q = torch.randn(4 * heads, d, generator=torch.Generator(device=dev).manual_seed(5000), device=dev).to(torch.bfloat16)
+    out = torch.empty(4 * heads, d, dtype=torch.float32, device=dev)
+    aws = hq.alloc_attention_workspace(heads, tokens, d, 4, dev)
+    hq.hq_kv_attention(streams[0], streams[1], heads, tokens, d, LAT, BPS, BPS, SEED, SEED + 1, q, 1.0 / math.sqrt(d),
+                       out, aws, group=4, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return {"launches": ["gemv_kernel 14336x4096", "encode_fixed_kernel gate", "kv_attention_kernel 32 query heads"]}
+
+
 def run_leg(args):
     peak, _ = peaks()
     if args.leg == "gemv":
@@ -843,6 +880,8 @@ def run_leg(args):
         res = configs_leg("cuda", peak, [m for _, m in workloads.llama_layer("cuda")])
     elif args.leg == "dit":
         res = dit_leg("cuda", peak)
+    elif args.leg == "profile":
+        res = profile_leg("cuda")
     elif args.leg == "fixed":
         res = fixed_leg("cuda", peak)
     else:
