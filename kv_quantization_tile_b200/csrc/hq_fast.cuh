@@ -56,27 +56,6 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b)
 }
 __device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
 
-// three-input max / min (one instruction each on sm_100)
-__device__ __forceinline__ float max3f(float a, float b, float c)
-{
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-__device__ __forceinline__ float min3f(float a, float b, float c)
-{
-    float d;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-// 1.0f if a == b, else 0.0f
-__device__ __forceinline__ float eq1f(float a, float b)
-{
-    float d;
-    asm("set.eq.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-    return d;
-}
-
 // ------------------------------------------------------------- transform
 // Forward transform of one tile held as EPL / 2 pairs per lane (see above).
 // l is the lane's index in its group, mask the group's lanes.
@@ -230,8 +209,12 @@ __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4])
     float s = ae[0];
 #pragma unroll
     for (int i = 1; i < 8; i++) s = __fadd_rn(s, ae[i]);  // in index order: the rounding is part of the rule
-    const float mx = max3f(max3f(ae[0], ae[1], ae[2]), max3f(ae[3], ae[4], ae[5]), fmaxf(ae[6], ae[7]));
-    const float mn = min3f(min3f(ae[0], ae[1], ae[2]), min3f(ae[3], ae[4], ae[5]), fminf(ae[6], ae[7]));
+    float mx = ae[0], mn = ae[0];
+#pragma unroll
+    for (int i = 1; i < 8; i++) {
+        mx = fmaxf(mx, ae[i]);
+        mn = fminf(mn, ae[i]);
+    }
     const int32_t px = __float_as_int(R[0].x) ^ __float_as_int(R[0].y) ^ __float_as_int(R[1].x) ^
                        __float_as_int(R[1].y) ^ __float_as_int(R[2].x) ^ __float_as_int(R[2].y) ^
                        __float_as_int(R[3].x) ^ __float_as_int(R[3].y);
@@ -249,7 +232,7 @@ __device__ __forceinline__ int e8_symbols(const float2 (&X)[4], float2 (&U)[4])
     // H: 1 at the coordinates whose |e| is T, else 0
     float2 H[4];
 #pragma unroll
-    for (int i = 0; i < 4; i++) H[i] = make_float2(eq1f(ae[2 * i], T), eq1f(ae[2 * i + 1], T));
+    for (int i = 0; i < 4; i++) H[i] = make_float2(ae[2 * i] == T ? 1.0f : 0.0f, ae[2 * i + 1] == T ? 1.0f : 0.0f);
     const float2 hs = add2(add2(H[0], H[1]), add2(H[2], H[3]));
     if (__fadd_rn(hs.x, hs.y) > 1.5f) {  // a tie: only the first hit (in index order) moves
         float seen = 0.0f;
