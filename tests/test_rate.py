@@ -64,3 +64,36 @@ def test_rate_report_itemizes_the_bits():
     h1 = 1.0
     assert r["symbol_entropy_bits_per_coord"] == round((14 * h0 + 2 * h1) / 16, 4)
     assert r["rice_gap_bits_per_coord"] == round(36 / 16 - (14 * h0 + 2 * h1) / 16, 4)
+
+
+@pytest.mark.parametrize("bps", [3.0, 4.0, 5.0])
+def test_e8_rice_gap_per_tile(bps):
+    """Per tile: the tile's Rice bits minus its symbols' code length under the
+    pooled empirical distribution (cross-entropy, stripped coordinates apart),
+    per coordinate.  Every tile's excess is positive and small; their mean is
+    the pooled gap.  Measured on 400 tiles: 0.02 .. 0.20 bits, mean 0.11 at
+    4 bps."""
+    rng = np.random.default_rng(7)
+    n, ntiles = 256, 400
+    x = (rng.standard_normal((ntiles, n)) * 0.02).astype(np.float32)
+    x = (x.view(np.uint32) & 0xFFFF0000).view(np.float32)
+    last = np.arange(n) % 8 == 7
+    rice, us = [], []
+    for t in range(ntiles):
+        r = oracle.encode_tile(x[t], "E8", bps, 42, j=t % 16, t=t)
+        st, _, u = oracle.unpack_tile("E8", n, r["k"], r["words"])
+        assert st == 0
+        rice.append(n * r["k"] + int((u.astype(np.int64) >> r["k"]).sum()) + n)
+        us.append(u.astype(np.int64))
+    U = np.stack(us)
+
+    def code_len(vals):
+        c = np.bincount(vals.ravel())
+        with np.errstate(divide="ignore"):
+            return -np.log2(c / c.sum())
+
+    L0, L1 = code_len(U[:, ~last]), code_len(U[:, last])
+    ce = np.array([L0[U[t, ~last]].sum() + L1[U[t, last]].sum() for t in range(ntiles)])
+    gap = (np.array(rice) - ce) / n
+    assert gap.min() > 0.0 and gap.max() < 0.3, (gap.min(), gap.max())
+    assert 0.05 < gap.mean() < 0.15, gap.mean()
