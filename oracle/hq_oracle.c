@@ -25,6 +25,11 @@
  * stated reading; the same readings are listed, with reasons, in the design
  * notes that ship with the repository.
  *
+ * Parity unpinned: the stream layout (hqo_pack_tile / the unpacker) -- no
+ * page prints a stream, so it is checked only against layouts worked out by
+ * hand from this file's own specification (tests/golden/rice_layout.json)
+ * and by round trips, not against anything the pages fix.
+ *
  * Precision: every step whose floating-point result decides an integer (the
  * lattice point, the Rice parameter, the stream) runs in IEEE binary32 with
  * round-to-nearest-even, one rounding per operation (compile with
