@@ -172,6 +172,38 @@ def test_every_tile_of_the_llama_and_kv_layers_is_bit_exact():
     assert flipped == 0
 
 
+def test_every_tile_of_one_dit_block_is_bit_exact():
+    """Whole streams of one DiT block (its ten matrices, 268 M weights, E8 4
+    bps, tile 256) and of its two FFN matrices with D4, A2 and Z at 4 bps,
+    against the oracle's encode of the same inputs: offsets, scales, Rice
+    parameters and every payload word equal."""
+    import os
+    from gpu_util import fetch
+    threads = max(1, os.cpu_count() or 1)
+    ntiles = 0
+    for name, x in workloads.dit_block(0, DEV):
+        rows, cols = x.shape
+        lats = ["E8"] + (["D4", "A2", "Z"] if name.startswith("ffn") else [])
+        xh = host_input(x)
+        for lat in lats:
+            s = hq.alloc_stream(rows, cols, 256, lat, 4.0, DEV)
+            st = torch.zeros(1, dtype=torch.int32, device=DEV)
+            hq.hq_encode(x, 256, lat, 4.0, 42, s, hq.alloc_workspace(rows, cols, 256, DEV), st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            g = fetch(s)
+            ref = oracle.encode(xh, 256, lat, 4.0, 42, threads=threads)
+            assert np.array_equal(g["off"], ref["off"]), (name, lat)
+            assert np.array_equal(g["scale"], ref["scale"]), (name, lat)
+            assert np.array_equal(g["k"], ref["k"]), (name, lat)
+            assert np.array_equal(g["payload"], ref["payload"]), (name, lat)
+            ntiles += g["k"].size
+            del s, g, ref
+        del x, xh
+        torch.cuda.empty_cache()
+    assert ntiles == (8 * 4096 * 16 + 2 * (16384 * 16)) + 3 * 2 * (16384 * 16)
+
+
 @pytest.mark.parametrize("case", ["llama_layer", "kv_layer"])
 def test_fixed_rate_full_size_sampled_tiles(case):
     """Fixed-rate streams at full size (31-word slots for the Llama layer at
